@@ -1,0 +1,275 @@
+"""fp64 CPU oracle of the Grouped Query Experts (GQE) attention forward pass.
+
+TEST INFRASTRUCTURE. Only the tests, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` use this module. The CUDA library never imports,
+links or calls it, and it imports nothing from the CUDA library. It is a plain,
+slow, obviously correct restatement of what the layer computes, in float64,
+taking the bf16 input values (exact in float64).
+
+Sources (the method is described in prose only; no formula or code is printed):
+  [GS]  "Grouped Query Experts: Mixture-of-Experts on GQA Self-Attention",
+        gist.science technical summary (zh / it / es editions), section
+        "Architecture and routing" (grouped expert pool, conditional activation,
+        dense KV path, output construction: hard concatenation, renormalised
+        weighted sum, always-on shared head).
+  [AT]  animattoys.com article on the same paper ("讓AI的注意力學會偷懶…"),
+        section 4 "How GQE works": per-group router scores, top-k activation,
+        each selected expert attends independently, concat + weighted-average
+        slot + shared head merged and passed through the output projection.
+  [WK]  aiboss88.com wiki "Grouped-Query Attention": query heads of one group
+        share one KV head; G = 1 is MQA, G = H is MHA.
+
+Readings where the pages are silent (each one is listed with its reason in the
+design notes of this repository):
+  * router = linear map of the layer input, logits = x Wr + br, no noise;
+  * probabilities = softmax over the M experts of each group;
+  * top-k by probability, exact ties broken toward the lower expert index; the
+    selected set is concatenated in ascending expert order;
+  * renormalised weights w = p_sel / sum(p_sel) over the selected set;
+  * one weighted slot per group;
+  * shared head attends KV head 0;
+  * scale 1/sqrt(dh), causal mask s <= t, no positional encoding or biases;
+  * Wo rows: [concat (g-major, slot j) | slot g | shared].
+
+Layout conventions (match the ones ``gqe_inputs`` draws): x [B*T, D],
+Wq [D, (G*M+1)*dh] with routed head h = g*M + e and the shared head last,
+Wk/Wv [D, G*dh], Wr [D, G*M], br [G*M], Wo [(G*k+G+1)*dh, D],
+Wo_dense [G*M*dh, D]. Token n = b*T + t.
+
+Every function here is pinned by tests/test_oracle.py against hand-worked
+examples, brute force and closed-form invariants.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+F64 = np.float64
+
+
+def _f64(a) -> np.ndarray:
+    """bf16/fp32 torch tensor or array -> float64 numpy (exact)."""
+    if hasattr(a, "detach"):
+        a = a.detach().to("cpu").float().numpy()
+    return np.asarray(a, dtype=F64)
+
+
+# ---------------------------------------------------------------------------
+# Router: [GS] "Conditional activation"; [AT] section 4, routing decision.
+# ---------------------------------------------------------------------------
+def route(x, Wr, br, G: int, M: int, k: int, forced_sel=None) -> dict:
+    """Per-token, per-group expert choice.
+
+    logits[n, g, e] = x[n] . Wr[:, g*M + e] + br[g*M + e]
+    p[n, g, :]      = softmax over the M experts of group g
+    sel[n, g, :]    = the k experts with the largest p (ties: lower index),
+                      listed in ascending expert index
+    w[n, g, j]      = p[sel_j] / sum_j' p[sel_j']     (renormalised)
+    margin[n, g]    = logit of the k-th ranked expert minus that of the
+                      (k+1)-th (+inf when k == M): how far the choice is from
+                      flipping.
+    ``forced_sel`` replaces the choice (the weights follow it).
+    """
+    X = _f64(x)
+    logits = X @ _f64(Wr)
+    if br is not None:
+        logits = logits + _f64(br)[None, :]
+    n = X.shape[0]
+    logits = logits.reshape(n, G, M)
+    mx = logits.max(axis=2, keepdims=True)
+    ex = np.exp(logits - mx)
+    p = ex / ex.sum(axis=2, keepdims=True)
+
+    # rank experts: larger logit first (same order as p), exact ties -> lower e
+    idx = np.broadcast_to(np.arange(M), logits.shape)
+    order = np.lexsort((idx, -logits), axis=-1)          # [n, G, M]
+    ranked = np.take_along_axis(logits, order, axis=2)
+    if k < M:
+        margin = ranked[:, :, k - 1] - ranked[:, :, k]
+    else:
+        margin = np.full((n, G), np.inf)
+
+    if forced_sel is None:
+        sel = np.sort(order[:, :, :k], axis=2)
+    else:
+        sel = np.sort(np.asarray(forced_sel, dtype=np.int64).reshape(n, G, k), axis=2)
+    psel = np.take_along_axis(p, sel, axis=2)
+    w = psel / psel.sum(axis=2, keepdims=True)
+    return {"logits": logits, "p": p, "sel": sel.astype(np.int64), "w": w, "margin": margin}
+
+
+def compact(sel, B: int, T: int, G: int, M: int):
+    """Token lists per segment s = (b*G + g)*M + e, tokens ascending.
+
+    seg_off [B*G*M + 1]: exclusive prefix of the segment lengths.
+    seg_tok [B*T*G*k]  : flat token index n = b*T + t of each compacted row.
+    row_map [B*T, G, k]: compacted row of (n, g, slot j).
+    This is the bookkeeping that lets the query projection run only for the
+    selected experts ([GS] "Conditional activation"; [AT] section 4).
+    """
+    sel = np.asarray(sel).reshape(B * T, G, -1)
+    k = sel.shape[2]
+    seg_off = np.zeros(B * G * M + 1, dtype=np.int64)
+    seg_tok = np.zeros(B * T * G * k, dtype=np.int64)
+    row_map = np.zeros((B * T, G, k), dtype=np.int64)
+    pos = 0
+    for b in range(B):
+        for g in range(G):
+            for e in range(M):
+                s = (b * G + g) * M + e
+                seg_off[s] = pos
+                toks_local, slots = np.nonzero(sel[b * T:(b + 1) * T, g, :] == e)
+                toks = toks_local + b * T                      # ascending
+                seg_tok[pos:pos + len(toks)] = toks
+                row_map[toks, g, slots] = pos + np.arange(len(toks))
+                pos += len(toks)
+    seg_off[B * G * M] = pos
+    return seg_off, seg_tok, row_map
+
+
+# ---------------------------------------------------------------------------
+# Causal scaled dot-product attention of one head against one KV head.
+# [AT] section 4: each selected expert computes attention independently
+# against its group's (shared, dense) K/V; [GS] "Dense KV path".
+# ---------------------------------------------------------------------------
+def attention_weights(q, pos, Kb, scale: float) -> np.ndarray:
+    """softmax_s(q_r . K_s * scale) over s <= pos_r; zeros for s > pos_r."""
+    q = np.asarray(q, F64)
+    pos = np.asarray(pos, dtype=np.int64)
+    tmax = int(pos.max()) + 1
+    S = (q @ Kb[:tmax].T) * scale
+    S[np.arange(tmax)[None, :] > pos[:, None]] = -np.inf
+    S = S - S.max(axis=1, keepdims=True)
+    P = np.exp(S)
+    return P / P.sum(axis=1, keepdims=True)
+
+
+def causal_attention(q, pos, Kb, Vb, scale: float, chunk_elems: int = 1 << 24) -> np.ndarray:
+    """o_r = sum_{s <= pos_r} softmax(q_r . K_s * scale) V_s, row by row."""
+    q = np.asarray(q, F64)
+    pos = np.asarray(pos, dtype=np.int64)
+    out = np.zeros((q.shape[0], Vb.shape[1]), dtype=F64)
+    if q.shape[0] == 0:
+        return out
+    tmax = int(pos.max()) + 1
+    step = max(1, chunk_elems // tmax)
+    for r0 in range(0, q.shape[0], step):
+        sl = slice(r0, r0 + step)
+        P = attention_weights(q[sl], pos[sl], Kb, scale)
+        out[sl] = P @ Vb[:P.shape[1]]
+    return out
+
+
+def _rows_of(rows, B, T):
+    if rows is None:
+        return np.arange(B * T, dtype=np.int64)
+    return np.asarray(rows, dtype=np.int64)
+
+
+def _project_kv(X, Wk, Wv, B, T, G, dh):
+    K = (X @ _f64(Wk)).reshape(B, T, G, dh)
+    V = (X @ _f64(Wv)).reshape(B, T, G, dh)
+    return K, V
+
+
+# ---------------------------------------------------------------------------
+# GQE layer forward: [GS] "Architecture and routing", [AT] section 4.
+# ---------------------------------------------------------------------------
+def gqe_forward(x, Wq, Wk, Wv, Wr, br, Wo, dims, rows=None, forced_sel=None) -> dict:
+    """The whole layer for the query tokens ``rows`` (flat n = b*T + t).
+
+    Steps, in the pages' order:
+      1. router: logits, in-group softmax, top-k, renormalised weights;
+      2. dense K/V projection of every token (K/V stay dense);
+      3. query projection for the selected experts (+ the shared head);
+      4. each selected expert attends causally to its group's K/V; the
+         shared head attends KV head 0;
+      5. A = [hard concat of selected outputs | per-group weighted slot |
+         shared head];  6. y = A Wo.
+    Returns the intermediate values too (all float64, rows in ``rows`` order).
+    ``forced_sel`` ([len(rows), G, k]) overrides the router's choice.
+    """
+    B, T, D, G, M, k, dh = dims.B, dims.T, dims.D, dims.G, dims.M, dims.k, dims.dh
+    X = _f64(x).reshape(B * T, D)
+    rows = _rows_of(rows, B, T)
+    scale = 1.0 / math.sqrt(dh)
+    R = route(X[rows], Wr, br, G, M, k, forced_sel=forced_sel)
+    sel, w = R["sel"], R["w"]
+
+    K, V = _project_kv(X, Wk, Wv, B, T, G, dh)
+    WQ = _f64(Wq)
+    Xr = X[rows]
+    bidx, tpos = rows // T, rows % T
+    nr = len(rows)
+    Ha = G * k + 1
+    Q = np.zeros((nr, Ha, dh))
+    O = np.zeros((nr, Ha, dh))
+
+    for g in range(G):
+        for j in range(k):
+            e_col = sel[:, g, j]
+            for e in range(M):
+                m = e_col == e
+                if not m.any():
+                    continue
+                h = g * M + e
+                Q[m, g * k + j] = Xr[m] @ WQ[:, h * dh:(h + 1) * dh]
+    Q[:, G * k] = Xr @ WQ[:, G * M * dh:(G * M + 1) * dh]
+
+    for b in range(B):
+        mb = bidx == b
+        if not mb.any():
+            continue
+        for g in range(G):
+            for j in range(k):
+                O[mb, g * k + j] = causal_attention(Q[mb, g * k + j], tpos[mb], K[b, :, g], V[b, :, g], scale)
+        O[mb, G * k] = causal_attention(Q[mb, G * k], tpos[mb], K[b, :, 0], V[b, :, 0], scale)
+
+    concat = O[:, :G * k].reshape(nr, G * k * dh)
+    slot = np.einsum("ngj,ngjd->ngd", w, O[:, :G * k].reshape(nr, G, k, dh)).reshape(nr, G * dh)
+    shared = O[:, G * k]
+    A = np.concatenate([concat, slot, shared], axis=1)
+    y = A @ _f64(Wo)
+    return {"rows": rows, "sel": sel, "w": w, "margin": R["margin"], "logits": R["logits"],
+            "p": R["p"], "K": K, "V": V, "Q": Q, "O": O, "A": A, "y": y}
+
+
+def gqa_dense_forward(x, Wq, Wk, Wv, Wo_dense, dims, rows=None) -> dict:
+    """All G*M query heads active (the GQA baseline of [GS] "Experimental
+    results", 16 query heads over 8 KV groups); head h attends KV group h // M
+    ([WK]); y = concat_h O_h Wo_dense."""
+    B, T, D, G, M, dh = dims.B, dims.T, dims.D, dims.G, dims.M, dims.dh
+    X = _f64(x).reshape(B * T, D)
+    rows = _rows_of(rows, B, T)
+    scale = 1.0 / math.sqrt(dh)
+    K, V = _project_kv(X, Wk, Wv, B, T, G, dh)
+    WQ = _f64(Wq)[:, :G * M * dh]
+    Xr = X[rows]
+    bidx, tpos = rows // T, rows % T
+    nr = len(rows)
+    H = G * M
+    Q = (Xr @ WQ).reshape(nr, H, dh)
+    O = np.zeros((nr, H, dh))
+    for b in range(B):
+        mb = bidx == b
+        if not mb.any():
+            continue
+        for h in range(H):
+            g = h // M
+            O[mb, h] = causal_attention(Q[mb, h], tpos[mb], K[b, :, g], V[b, :, g], scale)
+    y = O.reshape(nr, H * dh) @ _f64(Wo_dense)
+    return {"rows": rows, "K": K, "V": V, "Q": Q, "O": O, "y": y}
+
+
+def sample_rows(B: int, T: int, n_uniform: int, seed: int, n_last: int = 64, n_first: int = 16) -> np.ndarray:
+    """Query positions for sampled parity at sizes the full oracle cannot
+    finish: the first and last positions of every sequence plus uniform
+    draws (flat n = b*T + t, sorted, unique)."""
+    rng = np.random.default_rng(seed)
+    picks = []
+    for b in range(B):
+        picks.append(b * T + np.arange(min(n_first, T)))
+        picks.append(b * T + np.arange(max(0, T - n_last), T))
+    picks.append(rng.integers(0, B * T, size=n_uniform))
+    return np.unique(np.concatenate(picks))

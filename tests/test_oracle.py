@@ -1,0 +1,373 @@
+"""Pins of the fp64 oracle against things other than itself (CPU only).
+
+* hand-worked examples (tests/golden/*.txt, closed forms in e);
+* brute force: pure-Python attention loops, subset enumeration for top-k;
+* library special case: torch's scaled_dot_product_attention in fp64;
+* closed-form invariants: rows of the attention matrix sum to 1, causality,
+  k = M reduces to dense GQA plus the slot and shared terms, G = 1 is MQA,
+  M = k = 1, T = 1;
+* planted mistakes: perturbing the oracle in plausible ways makes a pin fail.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.gqe_ref as ref
+from gqe_inputs import Dims, make_inputs
+
+from _golden import load
+
+
+def _as_inputs(gold):
+    return {k: gold[k] for k in ("x", "Wq", "Wk", "Wv", "Wr", "br", "Wo")}
+
+
+def _run_golden(gold):
+    d = gold["dims"]
+    inp = _as_inputs(gold)
+    return ref.gqe_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"], inp["Wo"], d)
+
+
+def _check_golden(gold, out):
+    d = gold["dims"]
+    np.testing.assert_array_equal(out["sel"], gold["expect.sel"].astype(np.int64))
+    np.testing.assert_allclose(out["margin"], gold["expect.margin"], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(out["w"], gold["expect.w"], rtol=0, atol=1e-12)
+    O = out["O"].reshape(d.B * d.T, -1)
+    np.testing.assert_allclose(O, gold["expect.O"], rtol=0, atol=1e-12)
+    if "expect.A" in gold:
+        np.testing.assert_allclose(out["A"], gold["expect.A"], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(out["y"], gold["expect.y"], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("name", ["worked_example_k1.txt", "worked_example_k2.txt"])
+def test_worked_example(name):
+    gold = load(name)
+    d = gold["dims"]
+    out = _run_golden(gold)
+    _check_golden(gold, out)
+    if "expect.p_t0" in gold:
+        np.testing.assert_allclose(out["p"][0], gold["expect.p_t0"], rtol=0, atol=1e-12)
+    seg_off, seg_tok, row_map = ref.compact(out["sel"], d.B, d.T, d.G, d.M)
+    np.testing.assert_array_equal(seg_off, gold["expect.seg_off"].astype(np.int64))
+    np.testing.assert_array_equal(seg_tok, gold["expect.seg_tok"].astype(np.int64))
+    np.testing.assert_array_equal(row_map, gold["expect.row_map"].astype(np.int64))
+
+
+def test_tie_breaks_to_lower_expert():
+    # two equal logits: the lower expert index is chosen, margin is exactly 0
+    x = np.array([[1.0, 1.0]])
+    Wr = np.array([[1.0, 0.0], [0.0, 1.0]])
+    r = ref.route(x, Wr, None, G=1, M=2, k=1)
+    assert r["sel"][0, 0, 0] == 0
+    assert r["margin"][0, 0] == 0.0
+    # three-way tie with k = 2 picks {0, 1}
+    Wr3 = np.zeros((2, 3))
+    r3 = ref.route(x, Wr3, None, G=1, M=3, k=2)
+    np.testing.assert_array_equal(r3["sel"][0, 0], [0, 1])
+
+
+@pytest.mark.parametrize("M,k", [(2, 1), (3, 2), (4, 2), (5, 3), (4, 4)])
+def test_topk_matches_subset_enumeration(M, k):
+    rng = np.random.default_rng(M * 10 + k)
+    N, D, G = 64, 8, 3
+    x = rng.standard_normal((N, D))
+    Wr = rng.standard_normal((D, G * M))
+    br = rng.standard_normal(G * M)
+    r = ref.route(x, Wr, br, G, M, k)
+    logits = x @ Wr + br
+    for n in range(N):
+        for g in range(G):
+            lg = [float(v) for v in logits[n, g * M:(g + 1) * M]]
+            z = sum(math.exp(v) for v in lg)
+            p = [math.exp(v) / z for v in lg]
+            best = max(itertools.combinations(range(M), k), key=lambda c: sum(p[i] for i in c))
+            assert tuple(r["sel"][n, g]) == best
+            tot = sum(p[i] for i in best)
+            np.testing.assert_allclose(r["w"][n, g], [p[i] / tot for i in best], rtol=1e-12)
+            np.testing.assert_allclose(r["p"][n, g], p, rtol=1e-12)
+            srt = sorted(lg, reverse=True)
+            exp_margin = srt[k - 1] - srt[k] if k < M else math.inf
+            assert r["margin"][n, g] == pytest.approx(exp_margin, abs=1e-12)
+
+
+def _attn_pure_python(q, K, V, t, scale):
+    """Brute force: loops over s <= t with math.exp, no numpy arithmetic."""
+    sc = [scale * sum(q[d] * K[s][d] for d in range(len(q))) for s in range(t + 1)]
+    m = max(sc)
+    ws = [math.exp(v - m) for v in sc]
+    z = sum(ws)
+    return [sum(ws[s] * V[s][d] for s in range(t + 1)) / z for d in range(len(V[0]))]
+
+
+@pytest.mark.parametrize("T,dh", [(1, 4), (7, 3), (16, 8)])
+def test_attention_matches_pure_python_bruteforce(T, dh):
+    rng = np.random.default_rng(T * 100 + dh)
+    Q = rng.standard_normal((T, dh))
+    K = rng.standard_normal((T, dh))
+    V = rng.standard_normal((T, dh))
+    scale = 1.0 / math.sqrt(dh)
+    O = ref.causal_attention(Q, np.arange(T), K, V, scale)
+    for t in range(T):
+        bf = _attn_pure_python(Q[t].tolist(), K.tolist(), V.tolist(), t, scale)
+        np.testing.assert_allclose(O[t], bf, rtol=0, atol=1e-12)
+
+
+def test_attention_rows_sum_to_one_and_are_causal():
+    rng = np.random.default_rng(7)
+    T, dh = 40, 16
+    Q = rng.standard_normal((T, dh)) * 3
+    K = rng.standard_normal((T, dh))
+    P = ref.attention_weights(Q, np.arange(T), K, 0.25)
+    np.testing.assert_allclose(P.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+    assert np.all(P[np.triu_indices(T, 1)] == 0.0)
+    assert np.all(P[np.tril_indices(T)] > 0.0)
+
+
+def test_attention_matches_torch_sdpa_fp64():
+    rng = np.random.default_rng(11)
+    T, dh = 96, 64
+    Q = rng.standard_normal((T, dh))
+    K = rng.standard_normal((T, dh))
+    V = rng.standard_normal((T, dh))
+    O = ref.causal_attention(Q, np.arange(T), K, V, 1.0 / math.sqrt(dh))
+    tq, tk, tv = (torch.from_numpy(a)[None, None] for a in (Q, K, V))
+    Ot = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True)[0, 0].numpy()
+    np.testing.assert_allclose(O, Ot, rtol=0, atol=1e-12)
+
+
+def _small(B=2, T=24, D=32, G=2, M=2, k=1, dh=8, bias0=0.0, seed=3):
+    d = Dims(B=B, T=T, D=D, G=G, M=M, k=k, dh=dh, bias0=bias0)
+    inp = make_inputs(d, seed=seed)
+    # small D: raise the weight scale so routing and attention are not flat
+    for key in ("Wq", "Wk", "Wv", "Wr", "Wo", "Wo_dense"):
+        inp[key] = (inp[key].float() * 20).to(torch.bfloat16)
+    return d, inp
+
+
+def _fwd(d, inp, **kw):
+    return ref.gqe_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"], inp["Wo"], d, **kw)
+
+
+def _sdpa_heads(Qh, Kg, Vg, dh):
+    """torch SDPA in fp64: Qh [T, H, dh], Kg/Vg [T, H, dh] (already expanded)."""
+    q = torch.from_numpy(np.ascontiguousarray(Qh.transpose(1, 0, 2)))[None]
+    kk = torch.from_numpy(np.ascontiguousarray(Kg.transpose(1, 0, 2)))[None]
+    vv = torch.from_numpy(np.ascontiguousarray(Vg.transpose(1, 0, 2)))[None]
+    o = torch.nn.functional.scaled_dot_product_attention(q, kk, vv, is_causal=True, scale=1.0 / math.sqrt(dh))
+    return o[0].numpy().transpose(1, 0, 2)
+
+
+def test_dense_gqa_matches_sdpa_with_expanded_kv():
+    d, inp = _small(B=2, T=20, G=2, M=3)
+    out = ref.gqa_dense_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wo_dense"], d)
+    X = inp["x"].double().numpy()
+    H = d.G * d.M
+    for b in range(d.B):
+        xb = X[b * d.T:(b + 1) * d.T]
+        Q = (xb @ inp["Wq"].double().numpy()[:, :H * d.dh]).reshape(d.T, H, d.dh)
+        K = (xb @ inp["Wk"].double().numpy()).reshape(d.T, d.G, d.dh)
+        V = (xb @ inp["Wv"].double().numpy()).reshape(d.T, d.G, d.dh)
+        kv_of_head = np.arange(H) // d.M
+        O = _sdpa_heads(Q, K[:, kv_of_head], V[:, kv_of_head], d.dh)
+        np.testing.assert_allclose(out["O"][b * d.T:(b + 1) * d.T], O, rtol=0, atol=1e-12)
+        y = O.reshape(d.T, H * d.dh) @ inp["Wo_dense"].double().numpy()
+        np.testing.assert_allclose(out["y"][b * d.T:(b + 1) * d.T], y, rtol=0, atol=1e-11)
+
+
+def test_gqe_attention_matches_sdpa_per_selected_head():
+    d, inp = _small(B=2, T=20, G=2, M=4, k=2)
+    out = _fwd(d, inp)
+    X = inp["x"].double().numpy()
+    Wq = inp["Wq"].double().numpy()
+    for b in range(d.B):
+        xb = X[b * d.T:(b + 1) * d.T]
+        K = (xb @ inp["Wk"].double().numpy()).reshape(d.T, d.G, d.dh)
+        V = (xb @ inp["Wv"].double().numpy()).reshape(d.T, d.G, d.dh)
+        Qall = (xb @ Wq).reshape(d.T, d.G * d.M + 1, d.dh)
+        Oall = _sdpa_heads(Qall, K[:, list(np.arange(d.G * d.M) // d.M) + [0]],
+                           V[:, list(np.arange(d.G * d.M) // d.M) + [0]], d.dh)
+        for t in range(d.T):
+            n = b * d.T + t
+            for g in range(d.G):
+                for j in range(d.k):
+                    h = g * d.M + out["sel"][n, g, j]
+                    np.testing.assert_allclose(out["O"][n, g * d.k + j], Oall[t, h], rtol=0, atol=1e-12)
+            np.testing.assert_allclose(out["O"][n, d.G * d.k], Oall[t, d.G * d.M], rtol=0, atol=1e-12)
+
+
+def test_causality_future_tokens_do_not_change_outputs():
+    d, inp = _small(B=1, T=32)
+    base = _fwd(d, inp)
+    t0 = 17
+    pert = dict(inp)
+    x = inp["x"].clone()
+    x[t0 + 1:] = torch.randn(x[t0 + 1:].shape, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    pert["x"] = x
+    out = _fwd(d, pert)
+    # bitwise: routing is per token and masked scores contribute exact zeros
+    assert np.array_equal(out["y"][:t0 + 1], base["y"][:t0 + 1])
+    assert not np.array_equal(out["y"][t0 + 1:], base["y"][t0 + 1:])
+
+
+def test_k_equals_m_is_dense_gqa_plus_slot_and_shared():
+    d, inp = _small(B=2, T=16, G=2, M=3, k=3)
+    out = _fwd(d, inp)
+    cdim = d.G * d.k * d.dh
+    Wo = inp["Wo"].double().numpy()
+    dense = ref.gqa_dense_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], torch.from_numpy(Wo[:cdim]), d)
+    # slot = sum_e p_e O_e over all experts (renormalisation over the full pool is p itself)
+    O = dense["O"].reshape(-1, d.G, d.M, d.dh)
+    slot = np.einsum("nge,nged->ngd", out["p"], O).reshape(-1, d.G * d.dh)
+    shared = out["O"][:, d.G * d.k]
+    expect = dense["y"] + slot @ Wo[cdim:cdim + d.G * d.dh] + shared @ Wo[cdim + d.G * d.dh:]
+    np.testing.assert_allclose(out["y"], expect, rtol=0, atol=1e-11)
+    # zero slot and shared rows: exactly the dense layer with Wo_dense = concat rows
+    Wo0 = Wo.copy()
+    Wo0[cdim:] = 0
+    out0 = ref.gqe_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"], Wo0, d)
+    np.testing.assert_allclose(out0["y"], dense["y"], rtol=0, atol=1e-12)
+
+
+def test_g1_is_multi_query_attention():
+    d, inp = _small(B=1, T=20, G=1, M=3, k=3)
+    out = _fwd(d, inp)
+    X = inp["x"].double().numpy()
+    K = (X @ inp["Wk"].double().numpy()).reshape(d.T, 1, d.dh)
+    V = (X @ inp["Wv"].double().numpy()).reshape(d.T, 1, d.dh)
+    Q = (X @ inp["Wq"].double().numpy()).reshape(d.T, d.M + 1, d.dh)
+    O = _sdpa_heads(Q, np.repeat(K, d.M + 1, axis=1), np.repeat(V, d.M + 1, axis=1), d.dh)
+    np.testing.assert_allclose(out["O"], O, rtol=0, atol=1e-12)
+
+
+def test_m1_k1_every_token_routes_to_its_only_expert():
+    d, inp = _small(B=1, T=16, G=3, M=1, k=1)
+    out = _fwd(d, inp)
+    assert np.all(out["sel"] == 0)
+    assert np.all(out["w"] == 1.0)
+    cdim = d.G * d.dh
+    # slot equals the concat part exactly
+    np.testing.assert_array_equal(out["A"][:, cdim:2 * cdim], out["A"][:, :cdim])
+
+
+def test_t1_every_head_returns_v0_of_its_kv_group():
+    d, inp = _small(B=3, T=1, G=2, M=2, k=1)
+    out = _fwd(d, inp)
+    X = inp["x"].double().numpy()
+    V = (X @ inp["Wv"].double().numpy()).reshape(d.B, d.G, d.dh)
+    for n in range(d.B):
+        for g in range(d.G):
+            np.testing.assert_allclose(out["O"][n, g], V[n, g], rtol=0, atol=1e-14)
+        np.testing.assert_allclose(out["O"][n, d.G], V[n, 0], rtol=0, atol=1e-14)
+    A = np.concatenate([V.reshape(d.B, -1), V.reshape(d.B, -1), V[:, 0]], axis=1)
+    np.testing.assert_allclose(out["y"], A @ inp["Wo"].double().numpy(), rtol=0, atol=1e-13)
+
+
+def test_rows_subset_equals_full_run():
+    d, inp = _small(B=2, T=24, G=2, M=2, k=1)
+    full = _fwd(d, inp)
+    rows = np.array([0, 5, 23, 24, 31, 47])
+    sub = _fwd(d, inp, rows=rows)
+    np.testing.assert_allclose(sub["y"], full["y"][rows], rtol=0, atol=1e-13)
+    np.testing.assert_array_equal(sub["sel"], full["sel"][rows])
+
+
+def test_forced_selection_follows_the_given_experts():
+    d, inp = _small(B=1, T=12, G=2, M=3, k=2)
+    full = _fwd(d, inp)
+    same = _fwd(d, inp, forced_sel=full["sel"])
+    np.testing.assert_array_equal(same["y"], full["y"])
+    flipped = full["sel"].copy()
+    flipped[3, 1] = [0, 1] if tuple(flipped[3, 1]) != (0, 1) else [1, 2]
+    out = _fwd(d, inp, forced_sel=flipped)
+    p = full["p"][3, 1, flipped[3, 1]]
+    np.testing.assert_allclose(out["w"][3, 1], p / p.sum(), rtol=1e-13)
+    assert not np.allclose(out["y"][3], full["y"][3])
+
+
+def test_compaction_is_a_permutation_in_ascending_token_order():
+    rng = np.random.default_rng(2)
+    B, T, G, M, k = 3, 50, 4, 4, 2
+    sel = np.sort(np.stack([np.stack([rng.choice(M, k, replace=False) for _ in range(G)]) for _ in range(B * T)]), axis=2)
+    seg_off, seg_tok, row_map = ref.compact(sel, B, T, G, M)
+    assert seg_off[-1] == B * T * G * k
+    seen = np.zeros(B * T * G * k, dtype=int)
+    for n in range(B * T):
+        for g in range(G):
+            for j in range(k):
+                r = row_map[n, g, j]
+                s = (n // T * G + g) * M + sel[n, g, j]
+                assert seg_off[s] <= r < seg_off[s + 1]
+                assert seg_tok[r] == n
+                seen[r] += 1
+    assert np.all(seen == 1)
+    for s in range(B * G * M):
+        assert np.all(np.diff(seg_tok[seg_off[s]:seg_off[s + 1]]) > 0)
+
+
+def test_sample_rows_cover_ends_of_every_sequence():
+    rows = ref.sample_rows(B=2, T=1000, n_uniform=50, seed=0)
+    for b in range(2):
+        assert b * 1000 in rows and b * 1000 + 999 in rows
+    assert np.all(np.diff(rows) > 0)
+
+
+# --- planted mistakes: each plausible slip in the oracle trips a pin ---------
+
+def _golden_fails(monkeypatch, name, attr, fake):
+    monkeypatch.setattr(ref, attr, fake)
+    gold = load(name)
+    with pytest.raises(AssertionError):
+        _check_golden(gold, _run_golden(gold))
+
+
+def test_planted_no_causal_mask_is_caught(monkeypatch):
+    orig = ref.attention_weights
+
+    def no_mask(q, pos, Kb, scale):
+        return orig(q, np.full_like(np.asarray(pos), Kb.shape[0] - 1), Kb, scale)
+    _golden_fails(monkeypatch, "worked_example_k1.txt", "attention_weights", no_mask)
+
+
+def test_planted_k_v_swap_is_caught(monkeypatch):
+    orig = ref._project_kv
+
+    def swapped(X, Wk, Wv, B, T, G, dh):
+        K, V = orig(X, Wk, Wv, B, T, G, dh)
+        return V, K
+    _golden_fails(monkeypatch, "worked_example_k1.txt", "_project_kv", swapped)
+
+
+def test_planted_missing_renormalisation_is_caught(monkeypatch):
+    orig = ref.route
+
+    def raw_p(*a, **kw):
+        r = orig(*a, **kw)
+        r["w"] = np.take_along_axis(r["p"], r["sel"], axis=2)
+        return r
+    _golden_fails(monkeypatch, "worked_example_k2.txt", "route", raw_p)
+
+
+def test_planted_descending_concat_order_is_caught(monkeypatch):
+    orig = ref.route
+
+    def desc(*a, **kw):
+        r = orig(*a, **kw)
+        r["sel"] = r["sel"][:, :, ::-1].copy()
+        r["w"] = r["w"][:, :, ::-1].copy()
+        return r
+    _golden_fails(monkeypatch, "worked_example_k2.txt", "route", desc)
+
+
+def test_planted_wrong_softmax_scale_is_caught():
+    rng = np.random.default_rng(1)
+    Q, K, V = (rng.standard_normal((12, 16)) for _ in range(3))
+    good = ref.causal_attention(Q, np.arange(12), K, V, 0.25)
+    bad = ref.causal_attention(Q, np.arange(12), K, V, 1.0 / 16)
+    Ot = torch.nn.functional.scaled_dot_product_attention(
+        *(torch.from_numpy(a)[None, None] for a in (Q, K, V)), is_causal=True)[0, 0].numpy()
+    np.testing.assert_allclose(good, Ot, atol=1e-12)
+    assert not np.allclose(bad, Ot, atol=1e-6)
