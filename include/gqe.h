@@ -1,0 +1,214 @@
+/*
+ * gqe.h -- C ABI of libgqe: the Grouped Query Experts (GQE) attention-layer
+ * forward pass on NVIDIA B200 (sm_100a).
+ *
+ * The method ("Grouped Query Experts: Mixture-of-Experts on GQA
+ * Self-Attention"; gist.science technical summary, section "Architecture and
+ * routing"; animattoys.com article on the same paper, section 4 "How GQE
+ * works"): inside every GQA group the M query heads form a pool of experts; a
+ * per-token router activates the top-k of them; K/V projections and K/V heads
+ * stay dense; every selected expert attends causally to its group's K/V; the
+ * layer output is the output projection of [hard concatenation of the selected
+ * experts | per-group weighted slot (router probabilities renormalised over
+ * the selected set) | one always-on shared head].
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers (cudaMalloc'd or torch-owned),
+ *    except where a name ends in `_host`. The caller owns every buffer and the
+ *    workspace; the library never allocates or frees device memory.
+ *  - Tensors are dense row-major. "bf16" = IEEE bfloat16 stored as uint16.
+ *    Weights are [in, out]. Token index n = b*T + t.
+ *  - Every pointer must be 16-byte aligned; D and dh multiples of 64.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
+ *    asynchronous: they validate arguments on the host, enqueue kernels and
+ *    return. Invalid arguments return an error code before any launch.
+ *  - `ws`/`ws_bytes`: caller-provided device workspace of at least
+ *    gqe_workspace_bytes(dims, op) bytes, 256-byte aligned. Contents on entry
+ *    are ignored.
+ *  - Device-side failures (a pipeline wait that exceeded its time limit) are
+ *    recorded in a sticky per-device error word read by gqe_check_error().
+ *
+ * Supported shapes (others return GQE_ERR_UNSUPPORTED): dh == 64;
+ * D % 64 == 0; 1 <= k <= M; G*M a power of two <= 64; k and M in {1,2,4,8}
+ * (128 must be a multiple of the rows each token contributes to one
+ * attention tile); B*T < 2^31 / (G*k+1) / 64.
+ */
+#ifndef GQE_H_
+#define GQE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Layer dimensions: batch, tokens per sequence, d_model, KV groups, experts
+ * per group, experts selected per group, head dim. The shared head is always
+ * on. */
+typedef struct gqe_dims {
+  int32_t B, T, D, G, M, k, dh;
+} gqe_dims;
+
+enum gqe_status {
+  GQE_OK = 0,
+  GQE_ERR_INVALID_ARG = -1,  /* null/misaligned pointer, bad dims          */
+  GQE_ERR_UNSUPPORTED = -2,  /* shape outside the supported set above      */
+  GQE_ERR_WORKSPACE = -3,    /* ws too small or misaligned                  */
+  GQE_ERR_CUDA = -4,         /* a CUDA runtime call or launch failed        */
+  GQE_ERR_TIMEOUT = -5,      /* a device pipeline wait hit its time limit   */
+  GQE_ERR_NO_DEVICE = -6,    /* no sm_100 device current                    */
+  GQE_ERR_DEVICE_CHECK = -7  /* a device-side index check failed; the
+                                offending access was skipped               */
+};
+
+/* Operation selector for gqe_workspace_bytes. */
+enum gqe_op {
+  GQE_OP_ROUTE = 1,
+  GQE_OP_QPROJ = 2,
+  GQE_OP_ATTN = 3,
+  GQE_OP_COMBINE = 4,
+  GQE_OP_FORWARD = 5,
+  GQE_OP_DENSE = 6,
+  GQE_OP_FORWARD_HOST = 7
+};
+
+/* Workspace bytes the operation needs for these dims (0 if none); returns 0
+ * and nothing else for invalid dims (check with gqe_validate_dims). */
+size_t gqe_workspace_bytes(const gqe_dims* d, int op);
+
+/* GQE_OK if the dims are supported, else the error code a call would give. */
+int gqe_validate_dims(const gqe_dims* d);
+
+/*
+ * gqe_route -- the per-token router and the token compaction.
+ * Method: gist.science summary, "Architecture and routing", conditional
+ * activation (per token, top-k experts of every group) and the renormalised
+ * weighted sum (router probabilities renormalised over the selected set);
+ * animattoys.com article, section 4 (router scores each expert of each group,
+ * activates the k best).
+ *
+ *   logits[n,g,e] = sum_d x[n,d] * Wr[d, g*M+e] + br[g*M+e]    (fp32 accumulate)
+ *   p = softmax over e within the group; top-k by p (exact ties -> lower e)
+ *
+ * In : x  [B*T, D] bf16; Wr [D, G*M] bf16; br [G*M] fp32 or NULL (zeros).
+ * Out: sel     [B*T, G, k] int32  selected experts, ascending
+ *      w       [B*T, G, k] fp32   p_sel / sum(p_sel), same order as sel
+ *      margin  [B*T, G]    fp32   logit of k-th ranked minus (k+1)-th
+ *                                 (+inf when k == M); NULL to skip
+ *      seg_off [B*G*M + 1] int32  segment s = (b*G + g)*M + e starts at
+ *                                 seg_off[s]; seg_off[B*G*M] = B*T*G*k
+ *      seg_tok [B*T*G*k]   int32  token n of every compacted row, ascending
+ *                                 within each segment
+ *      row_map [B*T, G, k] int32  compacted row of (n, g, slot); NULL to skip
+ * ws: gqe_workspace_bytes(d, GQE_OP_ROUTE) (per-chunk expert counts).
+ */
+int gqe_route(const gqe_dims* d, const void* x, const void* Wr, const float* br,
+              int32_t* sel, float* w, float* margin, int32_t* seg_off,
+              int32_t* seg_tok, int32_t* row_map, void* ws, size_t ws_bytes,
+              void* stream);
+
+/*
+ * gqe_qproj -- dense K/V projection and the query projection of the selected
+ * experts only (plus the shared head), on tcgen05 tensor cores.
+ * Method: gist.science summary, "Architecture and routing", dense KV path
+ * (K/V projections unchanged from GQA) and sparsity on the query side only;
+ * animattoys.com article, section 4 (each expert has its own query
+ * projection; the group's experts read the same K/V).
+ *
+ * In : x [B*T, D]; Wq [D, (G*M+1)*dh] (routed head h = g*M+e, shared head
+ *      last); Wk, Wv [D, G*dh]; sel/seg_off/seg_tok from gqe_route.
+ * Out: Q [B*T, G*k+1, dh] bf16: Q[n, g*k+j] = x[n] Wq[:, head of sel[n,g,j]],
+ *        Q[n, G*k] = x[n] Wq[:, shared];
+ *      K, V [B*T, G, dh] bf16.
+ * ws: none (0 bytes). Segment sizes are read on the device: no host sync.
+ */
+int gqe_qproj(const gqe_dims* d, const void* x, const void* Wq, const void* Wk,
+              const void* Wv, const int32_t* sel, const int32_t* seg_off,
+              const int32_t* seg_tok, void* Q, void* K, void* V, void* ws,
+              size_t ws_bytes, void* stream);
+
+/*
+ * gqe_attn -- routed causal attention (FlashAttention-style, tcgen05 + TMEM,
+ * K/V tiles streamed by TMA).
+ * Method: animattoys.com article, section 4 (every selected expert computes
+ * attention on its own against its group's shared K/V; the shared head is
+ * always computed); gist.science summary, "Architecture and routing".
+ * The shared head attends KV head 0 (the pages do not say which; this is the
+ * library's fixed choice).
+ *
+ *   O[n, g*k+j] = sum_{s<=t} softmax_s(Q[n,g*k+j] . K[b,s,g] / sqrt(dh)) V[b,s,g]
+ *   O[n, G*k]   = same with Q[n, G*k] against KV head 0
+ *
+ * In : Q [B*T, G*k+1, dh]; K, V [B*T, G, dh]. Out: O [B*T, G*k+1, dh] bf16.
+ * Arithmetic: S and O accumulate in fp32 (TMEM), P rounded to bf16.
+ */
+int gqe_attn(const gqe_dims* d, const void* Q, const void* K, const void* V,
+             void* O, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * gqe_combine -- output construction and output projection.
+ * Method: gist.science summary, "Architecture and routing", output
+ * construction (hard concatenation; renormalised weighted sum; always-on
+ * shared head); animattoys.com article, section 4 (the three parts are merged
+ * and passed through the final output projection).
+ *
+ *   A[n] = [O[n,0..G*k-1] (concat) | sum_j w[n,g,j] O[n,g*k+j] for g (slot)
+ *           | O[n,G*k] (shared)]           width (G*k + G + 1)*dh
+ *   y    = A Wo,   Wo [(G*k+G+1)*dh, D] bf16, y [B*T, D] bf16.
+ * ws: gqe_workspace_bytes(d, GQE_OP_COMBINE).
+ */
+int gqe_combine(const gqe_dims* d, const void* O, const float* w,
+                const void* Wo, void* y, void* ws, size_t ws_bytes,
+                void* stream);
+
+/*
+ * gqe_forward -- route -> qproj -> attn -> combine on one stream.
+ * ws: gqe_workspace_bytes(d, GQE_OP_FORWARD); it holds every intermediate
+ * (sel, w, margin, segments, Q, K, V, O, ...).
+ */
+int gqe_forward(const gqe_dims* d, const void* x, const void* Wq,
+                const void* Wk, const void* Wv, const void* Wr,
+                const float* br, const void* Wo, void* y, void* ws,
+                size_t ws_bytes, void* stream);
+
+/*
+ * gqe_forward_host -- gqe_forward with the activations in HOST memory: the
+ * call enqueues the copy of x_host into the workspace, the forward pass and
+ * the copy of y back to y_host, all on `stream` (pin both host buffers for the
+ * copies to be asynchronous). Weights are device pointers.
+ * ws: gqe_workspace_bytes(d, GQE_OP_FORWARD_HOST).
+ */
+int gqe_forward_host(const gqe_dims* d, const void* x_host, const void* Wq,
+                     const void* Wk, const void* Wv, const void* Wr,
+                     const float* br, const void* Wo, void* y_host, void* ws,
+                     size_t ws_bytes, void* stream);
+
+/*
+ * gqa_dense_forward -- the all-heads GQA baseline the method is compared with
+ * (gist.science summary, "Experimental results": 16 query heads over 8 KV
+ * groups, all active). Head h = g*M+e attends KV group g; k is ignored.
+ *   y = concat_h O_h Wo_dense,  Wq's first G*M*dh columns, Wo_dense [G*M*dh, D].
+ * ws: gqe_workspace_bytes(d, GQE_OP_DENSE).
+ */
+int gqa_dense_forward(const gqe_dims* d, const void* x, const void* Wq,
+                      const void* Wk, const void* Wv, const void* Wo_dense,
+                      void* y, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, then read and clear the current device's sticky
+ * error word: GQE_OK, GQE_ERR_TIMEOUT, GQE_ERR_DEVICE_CHECK, or GQE_ERR_CUDA
+ * if the stream itself reported an error. */
+int gqe_check_error(void* stream);
+
+/* Static description of a status code. */
+const char* gqe_status_string(int status);
+
+/* Library ABI version (major*100 + minor). */
+int gqe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQE_H_ */

@@ -1,0 +1,539 @@
+// gqe_api.cu -- the C ABI of libgqe (declared in include/gqe.h): argument
+// validation, TMA tensor-map construction, workspace carving and kernel
+// launches for the GQE forward pass and the dense GQA baseline. Every step of
+// the computation runs in the kernels of this translation unit.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "gqe.h"
+#include "sm100.cuh"
+#include "route.cuh"
+#include "gemm.cuh"
+#include "attn.cuh"
+#include "combine.cuh"
+
+using namespace gqe;
+
+namespace {
+
+constexpr int kGemmStages = 4;
+constexpr int kQProjStages = 4;
+
+inline bool pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int check_dims(const gqe_dims* d) {
+  if (d == nullptr) return GQE_ERR_INVALID_ARG;
+  if (d->B < 1 || d->T < 1 || d->D < 1 || d->G < 1 || d->M < 1 || d->k < 1 || d->dh < 1) return GQE_ERR_INVALID_ARG;
+  if (d->k > d->M) return GQE_ERR_INVALID_ARG;
+  if (d->dh != 64) return GQE_ERR_UNSUPPORTED;
+  if (d->D % 64 != 0) return GQE_ERR_UNSUPPORTED;
+  const int GM = d->G * d->M;
+  if (GM < 2 || GM > 64 || !pow2(GM)) return GQE_ERR_UNSUPPORTED;
+  if (!pow2(d->M) || d->M > 8 || !pow2(d->k) || d->k > 8) return GQE_ERR_UNSUPPORTED;
+  if ((long long)d->D * GM * 2 > kRouteMaxWrBytes) return GQE_ERR_UNSUPPORTED;
+  if ((long long)d->B * GM > 8192) return GQE_ERR_UNSUPPORTED;
+  const long long N = (long long)d->B * d->T;
+  if (N * d->G * d->k >= (1ll << 31) || N * (d->G * d->M + 1) >= (1ll << 31)) return GQE_ERR_UNSUPPORTED;
+  return GQE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// TMA tensor maps (driver entry point fetched through the runtime)
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// bf16 tensor, 128-byte swizzle; dims/strides innermost first; strides in bytes
+// for dims 1..rank-1.
+int make_tmap(CUtensorMap* tm, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
+              const uint32_t* box) {
+  auto fn = encode_fn();
+  if (!fn) return GQE_ERR_CUDA;
+  cuuint64_t gd[5], gs[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides[i];
+  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bx, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? GQE_OK : GQE_ERR_CUDA;
+}
+
+// row-major [rows, cols] bf16 with row stride ld (elements); box 64 cols x box_rows
+int tmap_rows(CUtensorMap* tm, const void* base, long long rows, long long cols, long long ld, int box_rows) {
+  const uint64_t dims[2] = {(uint64_t)cols, (uint64_t)rows};
+  const uint64_t strides[1] = {(uint64_t)ld * 2};
+  const uint32_t box[2] = {64, (uint32_t)box_rows};
+  return make_tmap(tm, base, 2, dims, strides, box);
+}
+
+// [N, H, 64] bf16; box (64, bh, bn)
+int tmap_heads(CUtensorMap* tm, const void* base, long long N, int H, int bh, int bn) {
+  const uint64_t dims[3] = {64, (uint64_t)H, (uint64_t)N};
+  const uint64_t strides[2] = {128, (uint64_t)H * 128};
+  const uint32_t box[3] = {64, (uint32_t)bh, (uint32_t)bn};
+  return make_tmap(tm, base, 3, dims, strides, box);
+}
+
+// ---------------------------------------------------------------------------
+// Launch helpers
+// ---------------------------------------------------------------------------
+template <typename K>
+int set_smem(K kernel, int bytes) {
+  // cheap after the first call on a device; keeps multi-device use correct
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
+             ? GQE_OK
+             : GQE_ERR_CUDA;
+}
+
+inline int launch_status() { return cudaGetLastError() == cudaSuccess ? GQE_OK : GQE_ERR_CUDA; }
+
+template <int BN, int AMODE>
+int launch_gemm(const GemmParams& p, long long grid, cudaStream_t st) {
+  constexpr int STAGES = AMODE == kATma ? kGemmStages : kQProjStages;
+  auto kern = gemm_bf16_kernel<BN, STAGES, AMODE>;
+  const int smem = GemmSmem<BN, STAGES>::kBytes;
+  if (int e = set_smem(kern, smem)) return e;
+  if (grid <= 0) return GQE_OK;
+  if (grid > 0x7fffffffll) return GQE_ERR_UNSUPPORTED;
+  kern<<<(unsigned)grid, kGemmThreads, smem, st>>>(p);
+  return launch_status();
+}
+
+// Dense multi-segment projection: A [rows, K] times up to three weights.
+struct DenseSeg {
+  const void* W;     // [K, w_cols]
+  int w_cols;        // columns of the weight tensor
+  int b_col0;        // first column used
+  int n_cols;        // columns used
+  void* C;
+  long long ldc;
+  int c_col0;
+};
+
+int gemm_dense(const void* A, long long rows, int K, const DenseSeg* segs, int nseg, cudaStream_t st) {
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  if (int e = tmap_rows(&p.tmA, A, rows, K, K, kGemmBM)) return e;
+  int nt = 0;
+  for (int s = 0; s < nseg; ++s) {
+    if (int e = tmap_rows(&p.tmB[s], segs[s].W, K, segs[s].w_cols, segs[s].w_cols, 64)) return e;
+    p.seg[s].n_cols = segs[s].n_cols;
+    p.seg[s].b_col0 = segs[s].b_col0;
+    p.seg[s].c_col0 = segs[s].c_col0;
+    p.seg[s].ldc = segs[s].ldc;
+    p.seg[s].C = static_cast<__nv_bfloat16*>(segs[s].C);
+    p.seg[s].tile_start = nt;
+    nt += (int)cdiv(segs[s].n_cols, 128);
+  }
+  p.nseg = nseg;
+  p.ntn = nt;
+  p.rows = (int)rows;
+  p.K = K;
+  return launch_gemm<128, kATma>(p, cdiv(rows, kGemmBM) * nt, st);
+}
+
+// ---------------------------------------------------------------------------
+// Workspace carving
+// ---------------------------------------------------------------------------
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  template <typename T>
+  T* take(size_t count) {
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off = align256(off + count * sizeof(T));
+    return p;
+  }
+};
+
+struct RouteWs {
+  int32_t* counts;
+  int32_t* chunk_base;
+};
+RouteWs carve_route(Carver& c, const gqe_dims* d) {
+  const long long nch = cdiv(d->T, kRouteChunk);
+  const size_t n = (size_t)d->B * nch * d->G * d->M;
+  RouteWs r;
+  r.counts = c.take<int32_t>(n);
+  r.chunk_base = c.take<int32_t>(n);
+  return r;
+}
+
+struct FwdWs {
+  int32_t *sel, *seg_off, *seg_tok, *row_map;
+  float *w, *margin;
+  RouteWs route;
+  __nv_bfloat16 *Q, *K, *V, *O, *A;
+};
+FwdWs carve_forward(Carver& c, const gqe_dims* d) {
+  const size_t N = (size_t)d->B * d->T;
+  const int Ha = d->G * d->k + 1;
+  FwdWs f;
+  f.sel = c.take<int32_t>(N * d->G * d->k);
+  f.w = c.take<float>(N * d->G * d->k);
+  f.margin = c.take<float>(N * d->G);
+  f.seg_off = c.take<int32_t>((size_t)d->B * d->G * d->M + 1);
+  f.seg_tok = c.take<int32_t>(N * d->G * d->k);
+  f.row_map = c.take<int32_t>(N * d->G * d->k);
+  f.route = carve_route(c, d);
+  f.Q = c.take<__nv_bfloat16>(N * Ha * 64);
+  f.K = c.take<__nv_bfloat16>(N * d->G * 64);
+  f.V = c.take<__nv_bfloat16>(N * d->G * 64);
+  f.O = c.take<__nv_bfloat16>(N * Ha * 64);
+  f.A = c.take<__nv_bfloat16>(N * (size_t)(d->G * d->k + d->G + 1) * 64);
+  return f;
+}
+
+size_t combine_ws_bytes(const gqe_dims* d) {
+  return align256((size_t)d->B * d->T * (d->G * d->k + d->G + 1) * 64 * 2);
+}
+
+struct DenseWs {
+  __nv_bfloat16 *Q, *K, *V, *O;
+};
+DenseWs carve_dense(Carver& c, const gqe_dims* d) {
+  const size_t N = (size_t)d->B * d->T;
+  DenseWs w;
+  w.Q = c.take<__nv_bfloat16>(N * d->G * d->M * 64);
+  w.K = c.take<__nv_bfloat16>(N * d->G * 64);
+  w.V = c.take<__nv_bfloat16>(N * d->G * 64);
+  w.O = c.take<__nv_bfloat16>(N * d->G * d->M * 64);
+  return w;
+}
+
+int check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (need == 0) return GQE_OK;
+  if (ws == nullptr || ws_bytes < need) return GQE_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255) != 0) return GQE_ERR_WORKSPACE;
+  return GQE_OK;
+}
+
+int check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GQE_ERR_NO_DEVICE;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return GQE_ERR_NO_DEVICE;
+  if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return GQE_ERR_NO_DEVICE;
+  return (major == 10 && minor == 0) ? GQE_OK : GQE_ERR_NO_DEVICE;
+}
+
+#define GQE_TRY(expr)          \
+  do {                         \
+    const int _e = (expr);     \
+    if (_e != GQE_OK) return _e; \
+  } while (0)
+
+// ---------------------------------------------------------------------------
+// Stage implementations (arguments already validated)
+// ---------------------------------------------------------------------------
+template <int GM>
+int launch_route_select(const RouteParams& rp, long long grid, cudaStream_t st) {
+  constexpr int TPW = (64 / GM) < 1 ? 1 : ((64 / GM) > 16 ? 16 : (64 / GM));
+  constexpr int V = TPW * GM;
+  const int smem = rp.D * GM * 2 + kRouteWarps * V * 4 + GM * 4;
+  auto kern = route_select_kernel<GM>;
+  GQE_TRY(set_smem(kern, smem));
+  kern<<<(unsigned)grid, kRouteWarps * 32, smem, st>>>(rp);
+  return launch_status();
+}
+
+int do_route(const gqe_dims* d, const void* x, const void* Wr, const float* br, int32_t* sel, float* w,
+             float* margin, int32_t* seg_off, int32_t* seg_tok, int32_t* row_map, RouteWs rw, cudaStream_t st) {
+  RouteParams rp;
+  rp.x = static_cast<const __nv_bfloat16*>(x);
+  rp.Wr = static_cast<const __nv_bfloat16*>(Wr);
+  rp.br = br;
+  rp.sel = sel;
+  rp.w = w;
+  rp.margin = margin;
+  rp.counts = rw.counts;
+  rp.chunk_base = rw.chunk_base;
+  rp.seg_off = seg_off;
+  rp.seg_tok = seg_tok;
+  rp.row_map = row_map;
+  rp.B = d->B;
+  rp.T = d->T;
+  rp.D = d->D;
+  rp.G = d->G;
+  rp.M = d->M;
+  rp.k = d->k;
+  rp.nch = (int)cdiv(d->T, kRouteChunk);
+  const long long grid = (long long)d->B * rp.nch;
+  switch (d->G * d->M) {
+    case 2: GQE_TRY(launch_route_select<2>(rp, grid, st)); break;
+    case 4: GQE_TRY(launch_route_select<4>(rp, grid, st)); break;
+    case 8: GQE_TRY(launch_route_select<8>(rp, grid, st)); break;
+    case 16: GQE_TRY(launch_route_select<16>(rp, grid, st)); break;
+    case 32: GQE_TRY(launch_route_select<32>(rp, grid, st)); break;
+    case 64: GQE_TRY(launch_route_select<64>(rp, grid, st)); break;
+    default: return GQE_ERR_UNSUPPORTED;
+  }
+  const int nseg = d->B * d->G * d->M;
+  route_scan_kernel<<<1, 1024, nseg * 4, st>>>(rp);
+  GQE_TRY(launch_status());
+  route_scatter_kernel<<<(unsigned)grid, kRouteChunk, 0, st>>>(rp);
+  return launch_status();
+}
+
+int do_qproj(const gqe_dims* d, const void* x, const void* Wq, const void* Wk, const void* Wv, const int32_t* sel,
+             const int32_t* seg_off, const int32_t* seg_tok, void* Q, void* K, void* V, cudaStream_t st) {
+  const long long N = (long long)d->B * d->T;
+  const int G = d->G, M = d->M, k = d->k, Ha = G * k + 1;
+  const int wq_cols = (G * M + 1) * 64;
+  // dense part: K, V and the shared head's query, one launch over x
+  const DenseSeg segs[3] = {
+      {Wk, G * 64, 0, G * 64, K, (long long)G * 64, 0},
+      {Wv, G * 64, 0, G * 64, V, (long long)G * 64, 0},
+      {Wq, wq_cols, G * M * 64, 64, Q, (long long)Ha * 64, G * k * 64},
+  };
+  GQE_TRY(gemm_dense(x, N, d->D, segs, 3, st));
+  // selected experts: one segment per (b, g, e), rows gathered by seg_tok
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  GQE_TRY(tmap_rows(&p.tmB[0], Wq, d->D, wq_cols, wq_cols, 64));
+  p.K = d->D;
+  p.x = static_cast<const __nv_bfloat16*>(x);
+  p.seg_off = seg_off;
+  p.seg_tok = seg_tok;
+  p.sel = sel;
+  p.Q = static_cast<__nv_bfloat16*>(Q);
+  p.nsegs_q = d->B * G * M;
+  p.G = G;
+  p.M = M;
+  p.k = k;
+  p.Ha = Ha;
+  p.ntok = (int)N;
+  const long long tiles_max = cdiv(N * G * k, kGemmBM) + p.nsegs_q;
+  return launch_gemm<64, kAGather>(p, tiles_max, st);
+}
+
+int do_attn(const gqe_dims* d, const void* Q, int Hq, const void* K, const void* V, void* O, bool dense,
+            cudaStream_t st) {
+  const long long N = (long long)d->B * d->T;
+  AttnParams p;
+  memset(&p, 0, sizeof(p));
+  const int rr = dense ? d->M : d->k;
+  GQE_TRY(tmap_heads(&p.tmQ[0], Q, N, Hq, rr, 128 / rr));
+  GQE_TRY(tmap_heads(&p.tmQ[1], Q, N, Hq, 1, 128));
+  GQE_TRY(tmap_heads(&p.tmK, K, N, d->G, 1, 128));
+  GQE_TRY(tmap_heads(&p.tmV, V, N, d->G, 1, 128));
+  p.O = static_cast<__nv_bfloat16*>(O);
+  p.B = d->B;
+  p.T = d->T;
+  p.Ha = Hq;
+  int nrs = 0;
+  for (int g = 0; g < d->G; ++g) p.rs[nrs++] = AttnRowSet{g * rr, rr, g, 0};
+  if (!dense) p.rs[nrs++] = AttnRowSet{d->G * d->k, 1, 0, 1};
+  p.nrs = nrs;
+  p.nqt_max = (int)cdiv((long long)d->T * rr, 128);
+  p.scale_log2 = 1.4426950408889634f / sqrtf(64.f);
+  GQE_TRY(set_smem(attn_fwd_kernel, AttnSmem::kBytes));
+  const long long gx = (long long)d->B * nrs;
+  if (gx > 0x7fffffffll || p.nqt_max > 65535) return GQE_ERR_UNSUPPORTED;
+  dim3 grid((unsigned)gx, (unsigned)p.nqt_max);
+  attn_fwd_kernel<<<grid, kAttnThreads, AttnSmem::kBytes, st>>>(p);
+  return launch_status();
+}
+
+int do_combine(const gqe_dims* d, const void* O, const float* w, const void* Wo, void* y, __nv_bfloat16* A,
+               cudaStream_t st) {
+  const long long N = (long long)d->B * d->T;
+  const int KA = (d->G * d->k + d->G + 1) * 64;
+  CombineParams cp{static_cast<const __nv_bfloat16*>(O), w, A, N, d->G, d->k};
+  const long long warps = N;
+  const long long blocks = std::min<long long>(cdiv(warps * 32, 256), 148ll * 16);
+  combine_build_kernel<<<(unsigned)blocks, 256, 0, st>>>(cp);
+  GQE_TRY(launch_status());
+  const DenseSeg seg = {Wo, d->D, 0, d->D, y, (long long)d->D, 0};
+  return gemm_dense(A, N, KA, &seg, 1, st);
+}
+
+int check_ptrs(std::initializer_list<const void*> ps) {
+  for (const void* p : ps)
+    if (p == nullptr || !aligned16(p)) return GQE_ERR_INVALID_ARG;
+  return GQE_OK;
+}
+
+}  // namespace
+
+// ===========================================================================
+// exported C ABI
+// ===========================================================================
+extern "C" {
+
+int gqe_version(void) { return 100; }
+
+int gqe_validate_dims(const gqe_dims* d) { return check_dims(d); }
+
+size_t gqe_workspace_bytes(const gqe_dims* d, int op) {
+  if (check_dims(d) != GQE_OK) return 0;
+  Carver c{nullptr};
+  switch (op) {
+    case GQE_OP_ROUTE: carve_route(c, d); return c.off;
+    case GQE_OP_QPROJ: return 0;
+    case GQE_OP_ATTN: return 0;
+    case GQE_OP_COMBINE: return combine_ws_bytes(d);
+    case GQE_OP_FORWARD: carve_forward(c, d); return c.off;
+    case GQE_OP_FORWARD_HOST: {
+      carve_forward(c, d);
+      c.take<__nv_bfloat16>((size_t)d->B * d->T * d->D);
+      c.take<__nv_bfloat16>((size_t)d->B * d->T * d->D);
+      return c.off;
+    }
+    case GQE_OP_DENSE: carve_dense(c, d); return c.off;
+    default: return 0;
+  }
+}
+
+int gqe_route(const gqe_dims* d, const void* x, const void* Wr, const float* br, int32_t* sel, float* w,
+              float* margin, int32_t* seg_off, int32_t* seg_tok, int32_t* row_map, void* ws, size_t ws_bytes,
+              void* stream) {
+  GQE_TRY(check_dims(d));
+  GQE_TRY(check_ptrs({x, Wr, sel, w, seg_off, seg_tok}));
+  if (br && !aligned16(br)) return GQE_ERR_INVALID_ARG;
+  if (margin && !aligned16(margin)) return GQE_ERR_INVALID_ARG;
+  if (row_map && !aligned16(row_map)) return GQE_ERR_INVALID_ARG;
+  GQE_TRY(check_ws(ws, ws_bytes, gqe_workspace_bytes(d, GQE_OP_ROUTE)));
+  GQE_TRY(check_device());
+  Carver c{static_cast<uint8_t*>(ws)};
+  RouteWs rw = carve_route(c, d);
+  return do_route(d, x, Wr, br, sel, w, margin, seg_off, seg_tok, row_map, rw, static_cast<cudaStream_t>(stream));
+}
+
+int gqe_qproj(const gqe_dims* d, const void* x, const void* Wq, const void* Wk, const void* Wv, const int32_t* sel,
+              const int32_t* seg_off, const int32_t* seg_tok, void* Q, void* K, void* V, void* ws, size_t ws_bytes,
+              void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  GQE_TRY(check_dims(d));
+  GQE_TRY(check_ptrs({x, Wq, Wk, Wv, sel, seg_off, seg_tok, Q, K, V}));
+  GQE_TRY(check_device());
+  return do_qproj(d, x, Wq, Wk, Wv, sel, seg_off, seg_tok, Q, K, V, static_cast<cudaStream_t>(stream));
+}
+
+int gqe_attn(const gqe_dims* d, const void* Q, const void* K, const void* V, void* O, void* ws, size_t ws_bytes,
+             void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  GQE_TRY(check_dims(d));
+  GQE_TRY(check_ptrs({Q, K, V, O}));
+  GQE_TRY(check_device());
+  return do_attn(d, Q, d->G * d->k + 1, K, V, O, false, static_cast<cudaStream_t>(stream));
+}
+
+int gqe_combine(const gqe_dims* d, const void* O, const float* w, const void* Wo, void* y, void* ws, size_t ws_bytes,
+                void* stream) {
+  GQE_TRY(check_dims(d));
+  GQE_TRY(check_ptrs({O, w, Wo, y}));
+  GQE_TRY(check_ws(ws, ws_bytes, gqe_workspace_bytes(d, GQE_OP_COMBINE)));
+  GQE_TRY(check_device());
+  return do_combine(d, O, w, Wo, y, static_cast<__nv_bfloat16*>(ws), static_cast<cudaStream_t>(stream));
+}
+
+int gqe_forward(const gqe_dims* d, const void* x, const void* Wq, const void* Wk, const void* Wv, const void* Wr,
+                const float* br, const void* Wo, void* y, void* ws, size_t ws_bytes, void* stream) {
+  GQE_TRY(check_dims(d));
+  GQE_TRY(check_ptrs({x, Wq, Wk, Wv, Wr, Wo, y}));
+  if (br && !aligned16(br)) return GQE_ERR_INVALID_ARG;
+  GQE_TRY(check_ws(ws, ws_bytes, gqe_workspace_bytes(d, GQE_OP_FORWARD)));
+  GQE_TRY(check_device());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Carver c{static_cast<uint8_t*>(ws)};
+  FwdWs f = carve_forward(c, d);
+  GQE_TRY(do_route(d, x, Wr, br, f.sel, f.w, f.margin, f.seg_off, f.seg_tok, f.row_map, f.route, st));
+  GQE_TRY(do_qproj(d, x, Wq, Wk, Wv, f.sel, f.seg_off, f.seg_tok, f.Q, f.K, f.V, st));
+  GQE_TRY(do_attn(d, f.Q, d->G * d->k + 1, f.K, f.V, f.O, false, st));
+  return do_combine(d, f.O, f.w, Wo, y, f.A, st);
+}
+
+int gqe_forward_host(const gqe_dims* d, const void* x_host, const void* Wq, const void* Wk, const void* Wv,
+                     const void* Wr, const float* br, const void* Wo, void* y_host, void* ws, size_t ws_bytes,
+                     void* stream) {
+  GQE_TRY(check_dims(d));
+  if (x_host == nullptr || y_host == nullptr) return GQE_ERR_INVALID_ARG;
+  GQE_TRY(check_ws(ws, ws_bytes, gqe_workspace_bytes(d, GQE_OP_FORWARD_HOST)));
+  Carver c{static_cast<uint8_t*>(ws)};
+  carve_forward(c, d);
+  const size_t xbytes = (size_t)d->B * d->T * d->D * 2;
+  void* x_dev = c.take<__nv_bfloat16>((size_t)d->B * d->T * d->D);
+  void* y_dev = c.take<__nv_bfloat16>((size_t)d->B * d->T * d->D);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(x_dev, x_host, xbytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return GQE_ERR_CUDA;
+  GQE_TRY(gqe_forward(d, x_dev, Wq, Wk, Wv, Wr, br, Wo, y_dev, ws, ws_bytes, stream));
+  if (cudaMemcpyAsync(y_host, y_dev, xbytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return GQE_ERR_CUDA;
+  return GQE_OK;
+}
+
+int gqa_dense_forward(const gqe_dims* d, const void* x, const void* Wq, const void* Wk, const void* Wv,
+                      const void* Wo_dense, void* y, void* ws, size_t ws_bytes, void* stream) {
+  GQE_TRY(check_dims(d));
+  GQE_TRY(check_ptrs({x, Wq, Wk, Wv, Wo_dense, y}));
+  GQE_TRY(check_ws(ws, ws_bytes, gqe_workspace_bytes(d, GQE_OP_DENSE)));
+  GQE_TRY(check_device());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Carver c{static_cast<uint8_t*>(ws)};
+  DenseWs w = carve_dense(c, d);
+  const long long N = (long long)d->B * d->T;
+  const int G = d->G, M = d->M, H = G * M;
+  const int wq_cols = (G * M + 1) * 64;
+  const DenseSeg segs[3] = {
+      {Wq, wq_cols, 0, H * 64, w.Q, (long long)H * 64, 0},
+      {Wk, G * 64, 0, G * 64, w.K, (long long)G * 64, 0},
+      {Wv, G * 64, 0, G * 64, w.V, (long long)G * 64, 0},
+  };
+  GQE_TRY(gemm_dense(x, N, d->D, segs, 3, st));
+  GQE_TRY(do_attn(d, w.Q, H, w.K, w.V, w.O, true, st));
+  const DenseSeg so = {Wo_dense, d->D, 0, d->D, y, (long long)d->D, 0};
+  return gemm_dense(w.O, N, H * 64, &so, 1, st);
+}
+
+int gqe_check_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return GQE_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(int)) != cudaSuccess) return GQE_ERR_CUDA;
+  if (word != 0) {
+    const int zero = 0;
+    cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int));
+    return word == kDevErrTimeout ? GQE_ERR_TIMEOUT : GQE_ERR_DEVICE_CHECK;
+  }
+  return GQE_OK;
+}
+
+const char* gqe_status_string(int status) {
+  switch (status) {
+    case GQE_OK: return "ok";
+    case GQE_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, or bad dims)";
+    case GQE_ERR_UNSUPPORTED: return "unsupported shape";
+    case GQE_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case GQE_ERR_CUDA: return "CUDA runtime error";
+    case GQE_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case GQE_ERR_NO_DEVICE: return "no sm_100 device is current";
+    case GQE_ERR_DEVICE_CHECK: return "a device-side index check failed (access skipped)";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

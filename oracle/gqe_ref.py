@@ -173,6 +173,46 @@ def _project_kv(X, Wk, Wv, B, T, G, dh):
     return K, V
 
 
+def attend_selected(Q, rows, K, V, dims) -> np.ndarray:
+    """Attention step of the GQE layer for query rows ``rows`` (flat n).
+
+    Q [len(rows), G*k+1, dh]: slot g*k+j is the j-th selected expert of group
+    g, slot G*k the shared head. Each routed slot attends its group's K/V; the
+    shared head attends KV head 0 ([AT] section 4; KV head 0 is this
+    library's reading). K, V: [B, T, G, dh]."""
+    B, T, G, k, dh = dims.B, dims.T, dims.G, dims.k, dims.dh
+    rows = np.asarray(rows, dtype=np.int64)
+    Q = np.asarray(Q, F64)
+    K = np.asarray(K, F64).reshape(B, T, G, dh)
+    V = np.asarray(V, F64).reshape(B, T, G, dh)
+    scale = 1.0 / math.sqrt(dh)
+    bidx, tpos = rows // T, rows % T
+    O = np.zeros(Q.shape)
+    for b in range(B):
+        mb = bidx == b
+        if not mb.any():
+            continue
+        for g in range(G):
+            for j in range(k):
+                O[mb, g * k + j] = causal_attention(Q[mb, g * k + j], tpos[mb], K[b, :, g], V[b, :, g], scale)
+        O[mb, G * k] = causal_attention(Q[mb, G * k], tpos[mb], K[b, :, 0], V[b, :, 0], scale)
+    return O
+
+
+def combine(O, w, dims) -> np.ndarray:
+    """Output construction ([GS] "Architecture and routing", output
+    construction; [AT] section 4, merge of the three parts):
+    A = [hard concat of the selected outputs (g-major, ascending expert)
+         | per-group slot sum_j w[g,j] O[g,j] | shared head]."""
+    G, k, dh = dims.G, dims.k, dims.dh
+    O = np.asarray(O, F64)
+    w = np.asarray(w, F64)
+    nr = O.shape[0]
+    concat = O[:, :G * k].reshape(nr, G * k * dh)
+    slot = np.einsum("ngj,ngjd->ngd", w, O[:, :G * k].reshape(nr, G, k, dh)).reshape(nr, G * dh)
+    return np.concatenate([concat, slot, O[:, G * k]], axis=1)
+
+
 # ---------------------------------------------------------------------------
 # GQE layer forward: [GS] "Architecture and routing", [AT] section 4.
 # ---------------------------------------------------------------------------
@@ -193,18 +233,15 @@ def gqe_forward(x, Wq, Wk, Wv, Wr, br, Wo, dims, rows=None, forced_sel=None) -> 
     B, T, D, G, M, k, dh = dims.B, dims.T, dims.D, dims.G, dims.M, dims.k, dims.dh
     X = _f64(x).reshape(B * T, D)
     rows = _rows_of(rows, B, T)
-    scale = 1.0 / math.sqrt(dh)
     R = route(X[rows], Wr, br, G, M, k, forced_sel=forced_sel)
     sel, w = R["sel"], R["w"]
 
     K, V = _project_kv(X, Wk, Wv, B, T, G, dh)
     WQ = _f64(Wq)
     Xr = X[rows]
-    bidx, tpos = rows // T, rows % T
     nr = len(rows)
     Ha = G * k + 1
     Q = np.zeros((nr, Ha, dh))
-    O = np.zeros((nr, Ha, dh))
 
     for g in range(G):
         for j in range(k):
@@ -217,19 +254,8 @@ def gqe_forward(x, Wq, Wk, Wv, Wr, br, Wo, dims, rows=None, forced_sel=None) -> 
                 Q[m, g * k + j] = Xr[m] @ WQ[:, h * dh:(h + 1) * dh]
     Q[:, G * k] = Xr @ WQ[:, G * M * dh:(G * M + 1) * dh]
 
-    for b in range(B):
-        mb = bidx == b
-        if not mb.any():
-            continue
-        for g in range(G):
-            for j in range(k):
-                O[mb, g * k + j] = causal_attention(Q[mb, g * k + j], tpos[mb], K[b, :, g], V[b, :, g], scale)
-        O[mb, G * k] = causal_attention(Q[mb, G * k], tpos[mb], K[b, :, 0], V[b, :, 0], scale)
-
-    concat = O[:, :G * k].reshape(nr, G * k * dh)
-    slot = np.einsum("ngj,ngjd->ngd", w, O[:, :G * k].reshape(nr, G, k, dh)).reshape(nr, G * dh)
-    shared = O[:, G * k]
-    A = np.concatenate([concat, slot, shared], axis=1)
+    O = attend_selected(Q, rows, K, V, dims)
+    A = combine(O, w, dims)
     y = A @ _f64(Wo)
     return {"rows": rows, "sel": sel, "w": w, "margin": R["margin"], "logits": R["logits"],
             "p": R["p"], "K": K, "V": V, "Q": Q, "O": O, "A": A, "y": y}

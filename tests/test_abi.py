@@ -1,0 +1,86 @@
+"""The C-ABI library: it loads, exports every entry point include/gqe.h
+declares, and validates arguments on the host before touching a device (so
+these checks run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import moe_gqa_query_gqe_b200 as gqe
+from moe_gqa_query_gqe_b200 import lib
+from gqe_inputs import CONFIGS, Dims
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if not fn.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", fn)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w\s\*]*?\b(\w+)\s*\([^;{]*\)\s*;", src, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_library_exports_every_declared_symbol():
+    declared = _declared_functions()
+    assert "gqe_route" in declared and "gqa_dense_forward" in declared
+    so = lib.load()
+    for name in declared:
+        assert hasattr(so, name), f"{name} declared in include/ but not exported"
+    assert set(declared) == set(lib.EXPORTS)
+
+
+def test_version_and_status_strings():
+    assert gqe.gqe_version() == 100
+    for code in range(-7, 1):
+        assert gqe.gqe_status_string(code) != "unknown status"
+
+
+def test_all_workloads_are_supported_and_sized():
+    for name, d in CONFIGS.items():
+        assert gqe.validate_dims(d) == 0, name
+        assert gqe.workspace_bytes(d, gqe.OP_FORWARD) > 0
+        assert gqe.workspace_bytes(d, gqe.OP_FORWARD_HOST) > gqe.workspace_bytes(d, gqe.OP_FORWARD)
+        assert gqe.workspace_bytes(d, gqe.OP_DENSE) > 0
+        assert gqe.workspace_bytes(d, gqe.OP_QPROJ) == 0
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(dh=32), -2), (dict(D=1000), -2), (dict(k=3, M=2), -1), (dict(M=3, k=1), -2),
+    (dict(G=3, M=2), -2), (dict(T=0), -1), (dict(G=1, M=1), -2), (dict(k=0), -1),
+])
+def test_unsupported_and_invalid_dims(bad, code):
+    d = Dims(B=1, T=64, D=256, G=4, M=2, k=1).with_(**bad)
+    assert gqe.validate_dims(d) == code
+    assert gqe.workspace_bytes(d, gqe.OP_FORWARD) == 0
+
+
+def _raw(name, *args):
+    so = lib.load()
+    return getattr(so, name)(*args)
+
+
+def test_null_and_misaligned_pointers_are_rejected_before_any_launch():
+    d = lib.dims_struct(Dims(B=1, T=64, D=256, G=4, M=2, k=1))
+    P = 1 << 20  # aligned fake address: never dereferenced, validation fails first
+    dp = ctypes.byref(d)
+    assert _raw("gqe_attn", dp, None, P, P, P, None, 0, None) == -1
+    assert _raw("gqe_attn", dp, P + 2, P, P, P, None, 0, None) == -1
+    assert _raw("gqe_route", dp, P, P, None, P, P, None, P, P, None, None, 0, None) == -3  # no workspace
+    small = 256
+    assert _raw("gqe_route", dp, P, P, None, P, P, None, P, P, None, P, small, None) == -3
+    assert _raw("gqe_route", dp, P, P, None, P, P, None, P, P, None, P + 16, 1 << 30, None) == -3  # ws misaligned
+    assert _raw("gqa_dense_forward", dp, P, P, P, P, P, None, P, 1 << 30, None) == -1
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device answer")
+def test_valid_call_without_a_device_reports_no_device():
+    d = lib.dims_struct(Dims(B=1, T=64, D=256, G=4, M=2, k=1))
+    P = 1 << 20
+    assert _raw("gqe_attn", ctypes.byref(d), P, P, P, P, None, 0, None) == -6

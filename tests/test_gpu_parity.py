@@ -1,0 +1,189 @@
+"""GPU parity: every stage of the CUDA path against the fp64 oracle, element by
+element, on the same seeded inputs, through the C ABI.
+
+Bars: selections bit-exact except near-tie decisions (oracle margin < 1e-4,
+accepted either way, reported); compaction (segment offsets, token lists, row
+map) bit-exact against the oracle's compaction of the GPU's selections; bf16
+tensors within rel-L2 <= 5e-3 and max-abs <= 1e-2 of the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.gqe_ref as ref
+from gqe_inputs import CONFIGS, Dims, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from _gpu import (assert_close_bf16, check_selection, errors, f64, reference_attention, run_dense,
+                      run_forward, run_stages, to_dev)
+
+# sizes the oracle finishes in seconds; several tiles and ragged tails
+SMALL = {
+    "tiny_b2_t256": CONFIGS["tiny_b2_t256"],
+    "ragged_b3_t300": Dims(B=3, T=300, D=256, G=4, M=2, k=1),
+    "pool4_k2_skewed_t384": Dims(B=1, T=384, D=512, G=8, M=4, k=2, bias0=2.0),
+    "single_token_b4": Dims(B=4, T=1, D=128, G=2, M=2, k=1),
+    "one_group_g1_m4_k2": Dims(B=2, T=200, D=192, G=1, M=4, k=2),
+    "k_equals_m_t260": Dims(B=1, T=260, D=128, G=4, M=2, k=2),
+    "pool8_k4_t136": Dims(B=2, T=136, D=256, G=8, M=8, k=4),
+}
+
+
+@pytest.fixture(scope="module")
+def cases():
+    out = {}
+    for name, d in SMALL.items():
+        inp = make_inputs(d, seed=0)
+        dev = to_dev(inp)
+        st = run_stages(d, dev)
+        out[name] = (d, inp, dev, st)
+    return out
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_route_selection_and_compaction(cases, name):
+    d, inp, dev, st = cases[name]
+    assert st["status"] == 0
+    chk = check_selection(d, inp["x"], inp["Wr"], inp["br"], st["sel"])
+    r = chk["oracle"]
+    same = np.all(st["sel"].numpy() == r["sel"], axis=2)
+    np.testing.assert_allclose(st["w"].numpy()[same], r["w"][same], rtol=0, atol=2e-6)
+    fin = np.isfinite(r["margin"])
+    m_gpu = st["margin"].numpy()
+    np.testing.assert_allclose(m_gpu[fin & same], r["margin"][fin & same], rtol=0, atol=5e-5)
+    assert np.all(np.isinf(m_gpu[~fin]))
+    seg_off, seg_tok, row_map = ref.compact(st["sel"].numpy(), d.B, d.T, d.G, d.M)
+    np.testing.assert_array_equal(st["seg_off"].numpy(), seg_off)
+    np.testing.assert_array_equal(st["seg_tok"].numpy(), seg_tok)
+    np.testing.assert_array_equal(st["row_map"].numpy(), row_map)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_projection_stage(cases, name):
+    d, inp, dev, st = cases[name]
+    full = ref.gqe_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"], inp["Wo"], d,
+                           forced_sel=st["sel"].numpy())
+    N = d.B * d.T
+    assert_close_bf16(st["K"], full["K"].reshape(N, d.G, 64), "K")
+    assert_close_bf16(st["V"], full["V"].reshape(N, d.G, 64), "V")
+    assert_close_bf16(st["Q"], full["Q"], "Q (selected experts + shared head)")
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_attention_stage(cases, name):
+    d, inp, dev, st = cases[name]
+    rows = np.arange(d.B * d.T)
+    want = reference_attention(d, st["Q"], st["K"], st["V"], rows)
+    assert_close_bf16(st["O"], want, "O")
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_combine_stage(cases, name):
+    d, inp, dev, st = cases[name]
+    A = ref.combine(f64(st["O"]), f64(st["w"]), d)
+    want = A @ f64(inp["Wo"])
+    assert_close_bf16(st["y"], want, "y from GPU O and w")
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_layer_end_to_end(cases, name):
+    d, inp, dev, st = cases[name]
+    y, _, status = run_forward(d, dev)
+    assert status == 0
+    # the one-call forward runs the same kernels on the same inputs: identical bits
+    assert torch.equal(y.cpu(), st["y"])
+    full = ref.gqe_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"], inp["Wo"], d,
+                           forced_sel=st["sel"].numpy())
+    assert_close_bf16(y, full["y"], "GQE y vs oracle")
+
+
+@pytest.mark.parametrize("name", ["tiny_b2_t256", "ragged_b3_t300", "pool4_k2_skewed_t384", "pool8_k4_t136",
+                                  "single_token_b4"])
+def test_dense_gqa_baseline(cases, name):
+    d, inp, dev, st = cases[name]
+    y, _, status = run_dense(d, dev)
+    assert status == 0
+    want = ref.gqa_dense_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wo_dense"], d)
+    assert_close_bf16(y, want["y"], "dense GQA y vs oracle")
+
+
+def test_causality_bitwise_on_gpu(cases):
+    d, inp, dev, st = cases["ragged_b3_t300"]
+    t0 = 171
+    x = inp["x"].clone().view(d.B, d.T, d.D)
+    g = torch.Generator().manual_seed(9)
+    x[:, t0 + 1:] = torch.randn(x[:, t0 + 1:].shape, generator=g).to(torch.bfloat16)
+    dev2 = dict(dev)
+    dev2["x"] = x.view(d.B * d.T, d.D).cuda()
+    y2, _, status = run_forward(d, dev2)
+    assert status == 0
+    y1 = st["y"].view(d.B, d.T, d.D)
+    y2 = y2.cpu().view(d.B, d.T, d.D)
+    assert torch.equal(y1[:, :t0 + 1], y2[:, :t0 + 1])
+    assert not torch.equal(y1[:, t0 + 1:], y2[:, t0 + 1:])
+
+
+def test_repeat_calls_are_deterministic(cases):
+    d, inp, dev, st = cases["pool4_k2_skewed_t384"]
+    y1, _, _ = run_forward(d, dev)
+    y2, _, _ = run_forward(d, dev)
+    assert torch.equal(y1, y2)
+
+
+# ---- the workloads at full size: sampled query rows against the oracle ----
+
+def _sampled_parity(d, n_uniform, seed=0, dense=True):
+    inp = make_inputs(d, seed=0, device="cpu")
+    dev = to_dev(inp)
+    y, ws, status = run_forward(d, dev)
+    assert status == 0
+    import moe_gqa_query_gqe_b200 as gqe
+    views = gqe.forward_views(d, ws)
+    sel = views["sel"].cpu()
+    rows = ref.sample_rows(d.B, d.T, n_uniform=n_uniform, seed=seed)
+    chk = check_selection(d, inp["x"], inp["Wr"], inp["br"], sel, rows=rows)
+    seg_off = views["seg_off"].cpu().numpy()
+    assert seg_off[-1] == d.B * d.T * d.G * d.k
+    counts = np.diff(seg_off)
+    full = ref.gqe_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"], inp["Wo"], d,
+                           rows=rows, forced_sel=sel.numpy()[rows])
+    e = assert_close_bf16(y.cpu()[rows], full["y"], "GQE y (sampled rows)")
+    out = {"gqe": e, "near_ties": chk["near_ties"], "segments": counts}
+    if dense:
+        yd, _, status = run_dense(d, dev)
+        assert status == 0
+        want = ref.gqa_dense_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wo_dense"], d, rows=rows)
+        out["dense"] = assert_close_bf16(yd.cpu()[rows], want["y"], "dense y (sampled rows)")
+    return out
+
+
+def test_main_layer_b8_t2048_full_rows():
+    d = CONFIGS["main_b8_t2048"]
+    inp = make_inputs(d, seed=0)
+    dev = to_dev(inp)
+    y, ws, status = run_forward(d, dev)
+    assert status == 0
+    import moe_gqa_query_gqe_b200 as gqe
+    sel = gqe.forward_views(d, ws)["sel"].cpu()
+    check_selection(d, inp["x"], inp["Wr"], inp["br"], sel)
+    full = ref.gqe_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"], inp["Wo"], d,
+                           forced_sel=sel.numpy())
+    assert_close_bf16(y, full["y"], "GQE y, main layer")
+
+
+def test_long_context_t32768_sampled():
+    _sampled_parity(CONFIGS["long_b1_t32768"], n_uniform=256)
+
+
+def test_skewed_pool4_k2_t131072_sampled():
+    out = _sampled_parity(CONFIGS["skewed_b1_t131072_m4k2"], n_uniform=128, dense=False)
+    seg = out["segments"].reshape(8, 4)
+    # expert 0 carries the +2.0 router bias: it is in the top-2 of most tokens
+    assert np.all(seg[:, 0] > 0.9 * 131072)
+
+
+@pytest.mark.slow
+def test_million_tokens_sampled():
+    _sampled_parity(CONFIGS["million_b1_t1048576"], n_uniform=96, dense=False)
