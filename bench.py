@@ -1,0 +1,359 @@
+"""Throughput of the GQE attention-layer forward pass on B200.
+
+One step = one full forward pass of the layer (route -> selected-expert and
+K/V projections -> routed causal attention -> combine + output projection)
+over one batch of the main workload (8 sequences x 2048 tokens, d_model 1024,
+8 KV groups x 2 experts, k = 1, shared head, head dim 64), inputs resident in
+HBM. Prints one JSON line.
+
+  python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl reference]
+
+Timing: CUDA events on the launching stream around every step, an L2 flush
+(256 MiB write) between steps outside the events, max over ranks. With N > 1
+every rank runs its own batch (weak scaling, no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GQE fwd tokens/s, TFLOP/s % BF16 peak, speedup vs dense GQA at 2K–1M tokens"
+DEFAULT_WORKLOAD = "main_b8_t2048"
+
+
+def flops_model(d) -> dict:
+    """Algorithmic flops of one forward pass (what the method must compute;
+    masked halves of diagonal tiles are not counted)."""
+    N = d.B * d.T
+    Ha = d.G * d.k + 1
+    causal_pairs = d.B * d.T * (d.T + 1) // 2           # sum over rows of (t + 1), per row set
+    f = {
+        "router": 2 * N * d.D * d.G * d.M,
+        "q_proj": 2 * N * d.D * d.dh * Ha,
+        "kv_proj": 2 * N * d.D * 2 * d.G * d.dh,
+        "attention": 4 * d.dh * Ha * causal_pairs,
+        "wo": 2 * N * (d.G * d.k + d.G + 1) * d.dh * d.D,
+    }
+    dense = {
+        "qkv_proj": 2 * N * d.D * (d.G * d.M + 2 * d.G) * d.dh,
+        "attention": 4 * d.dh * d.G * d.M * causal_pairs,
+        "wo": 2 * N * d.G * d.M * d.dh * d.D,
+    }
+    return {"gqe": f, "gqe_total": sum(f.values()), "dense": dense, "dense_total": sum(dense.values())}
+
+
+def load_peaks() -> dict:
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            p = json.load(fh)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p["bf16_tflops_sustained"], "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_hash(name: str) -> str:
+    with open(os.path.join(ROOT, "moe_gqa_query_gqe_b200", "csrc", name), "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, src: str) -> float | None:
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as fh:
+            rec = json.load(fh)
+        r = rec.get(workload, {}).get(src)
+        if r and r.get("source_hash") == kernel_source_hash(src):
+            return float(r["bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.samples = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(gpu_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append((time.time(), parts))
+
+    def wait_first(self, timeout=3.0):
+        t0 = time.time()
+        while self.proc and not self.samples and time.time() - t0 < timeout:
+            time.sleep(0.05)
+
+    def stop(self, t_begin, t_end) -> dict:
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=2)
+            except Exception:
+                self.proc.kill()
+        window = [s for (t, s) in self.samples if t_begin - 0.2 <= t <= t_end + 0.2]
+        scope = "timed"
+        if not window:
+            window = [s for (_, s) in self.samples]
+            scope = "run"
+        if not window:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no-samples"], "samples": 0}
+        sm = [float(s[1]) for s in window if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in window for i in range(4) if s[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(window[0][2]) if window[0][2].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(window), "scope": scope}
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(d, budget_s: float, max_steps: int | None = None):
+    """Time the fp64 oracle on whole sequences of the workload (one sequence
+    per sample, all its rows), until ``budget_s`` of CPU work or ``max_steps``."""
+    import oracle.gqe_ref as ref
+    from gqe_inputs import make_inputs
+    d1 = d.with_(B=1)
+    inp = make_inputs(d1, seed=0)
+    times = []
+    t_all = time.time()
+    while True:
+        t0 = time.perf_counter()
+        ref.gqe_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"], inp["Wo"], d1)
+        times.append(time.perf_counter() - t0)
+        if max_steps is not None and len(times) >= max_steps:
+            break
+        if max_steps is None and time.time() - t_all >= budget_s:
+            break
+    return d1.T, times
+
+
+def run_reference(args, d, rank, world):
+    """The oracle arm: the fp64 CPU oracle as it stands, on host cores."""
+    if rank != 0:
+        return
+    tokens, times = oracle_sample(d, 0, max_steps=args.warmup + args.steps)
+    timed = times[args.warmup:] or times
+    sec = sum(timed) / len(timed)
+    value = tokens / sec
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, **{k: getattr(d, k) for k in ("B", "T", "D", "G", "M", "k", "dh")},
+                       "l2": "n/a (host)"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+                             "sample": f"one sequence ({tokens} tokens, all rows) of the workload per step"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="gqe", choices=["gqe", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle timing (rank 0, N=1)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    from gqe_inputs import CONFIGS
+    d = CONFIGS[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, d, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import moe_gqa_query_gqe_b200 as gqe
+    from gqe_inputs import make_inputs
+
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
+
+    inp = make_inputs(d, seed=rank, device="cuda")
+    N, G, M, k = d.B * d.T, d.G, d.M, d.k
+    Ha = G * k + 1
+    dev = "cuda"
+    sel = torch.empty(N, G, k, dtype=torch.int32, device=dev)
+    wts = torch.empty(N, G, k, dtype=torch.float32, device=dev)
+    margin = torch.empty(N, G, dtype=torch.float32, device=dev)
+    seg_off = torch.empty(d.B * G * M + 1, dtype=torch.int32, device=dev)
+    seg_tok = torch.empty(N * G * k, dtype=torch.int32, device=dev)
+    row_map = torch.empty(N, G, k, dtype=torch.int32, device=dev)
+    Q = torch.empty(N, Ha, 64, dtype=torch.bfloat16, device=dev)
+    K = torch.empty(N, G, 64, dtype=torch.bfloat16, device=dev)
+    V = torch.empty(N, G, 64, dtype=torch.bfloat16, device=dev)
+    O = torch.empty(N, Ha, 64, dtype=torch.bfloat16, device=dev)
+    y = torch.empty(N, d.D, dtype=torch.bfloat16, device=dev)
+    ws_route = gqe.workspace(d, gqe.OP_ROUTE)
+    ws_comb = gqe.workspace(d, gqe.OP_COMBINE)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev: ev[0].record(stream)
+        gqe.gqe_route(d, inp["x"], inp["Wr"], inp["br"], sel, wts, margin, seg_off, seg_tok, row_map, ws_route)
+        if ev: ev[1].record(stream)
+        gqe.gqe_qproj(d, inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], sel, seg_off, seg_tok, Q, K, V)
+        if ev: ev[2].record(stream)
+        gqe.gqe_attn(d, Q, K, V, O)
+        if ev: ev[3].record(stream)
+        gqe.gqe_combine(d, O, wts, inp["Wo"], y, ws_comb)
+        if ev: ev[4].record(stream)
+
+    launches_per_step = 3 + 2 + 1 + 2  # route 3, qproj 2, attention 1, combine 2
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # ---- warm-up, then K timed steps (L2 flushed between steps) -----------
+    sampler = ClockSampler(local_rank)
+    sampler.wait_first()
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    assert gqe.gqe_check_error() == 0
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    barrier()
+    t_begin = time.time()
+    for i in range(args.steps):
+        flush.fill_(1)
+        step(evs[i])
+    barrier()
+    t_end = time.time()
+    clocks = sampler.stop(t_begin, t_end)
+    status = gqe.gqe_check_error()
+    assert status == 0, gqe.gqe_status_string(status)
+    stage_ms = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)]
+    step_ms = [sum(s) for s in stage_ms]
+    total_ms = sum(step_ms)
+    attn_ms = sum(s[2] for s in stage_ms) / args.steps
+    stage_avg = {n: sum(s[j] for s in stage_ms) / args.steps for j, n in
+                 enumerate(("route", "qproj", "attention", "combine"))}
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * N / (ms_per_step / 1e3)
+
+    # ---- dense GQA baseline of the same library (speedup denominator) -------
+    ws_dense = gqe.workspace(d, gqe.OP_DENSE)
+    y_dense = torch.empty_like(y)
+    dense_ms = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        gqe.gqa_dense_forward(d, inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wo_dense"], y_dense, ws_dense)
+        e1.record(stream)
+        if i >= args.warmup:
+            dense_ms.append((e0, e1))
+    torch.cuda.synchronize()
+    dense_ms = sum(a.elapsed_time(b) for a, b in dense_ms) / args.steps
+
+    # ---- end to end through the host-buffer entry point ---------------------
+    x_host = inp["x"].cpu().pin_memory()
+    y_host = torch.empty(N, d.D, dtype=torch.bfloat16).pin_memory()
+    ws_host = gqe.workspace(d, gqe.OP_FORWARD_HOST)
+    e2e = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        gqe.gqe_forward_host(d, x_host, inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"], inp["Wo"], y_host,
+                             ws_host)
+        e1.record(stream)
+        if i >= args.warmup:
+            e2e.append((e0, e1))
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e) / args.steps
+    if world > 1:
+        t = torch.tensor([e2e_ms, dense_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms, dense_ms = (float(v) for v in t.tolist())
+    status = gqe.gqe_check_error()
+    assert status == 0, gqe.gqe_status_string(status)
+
+    fl = flops_model(d)
+    peaks = load_peaks()
+    attn_flops = fl["gqe"]["attention"]
+    attn_tflops = attn_flops / (attn_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": attn_tflops,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16_tflops"],
+                "peak_source": f"{peaks['source']} bf16 burst",
+                "traffic": recorded_traffic(args.workload, "attn.cuh"),
+                "algorithmic_flops_per_launch": attn_flops}
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) activations, N(0,0.02^2) weights)",
+            "config": {"workload": args.workload, **{kk: getattr(d, kk) for kk in ("B", "T", "D", "G", "M", "k", "dh")},
+                       "tokens_per_step_per_gpu": N, "l2": "flushed between steps (256 MiB write)",
+                       "parallelism": f"replicas x{world}"},
+            "tflops": fl["gqe_total"] / (ms_per_step / 1e3) / 1e12 * world,
+            "frac_bf16_peak": fl["gqe_total"] / (ms_per_step / 1e3) / 1e12 / peaks["bf16_tflops"],
+            "dense_gqa_ms_per_step": dense_ms, "speedup_vs_dense": dense_ms / ms_per_step,
+            "stage_ms": stage_avg, "roofline": roofline, "clocks": clocks,
+            "e2e": {"value": world * N / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": N * d.D * 2, "d2h_bytes_per_step": N * d.D * 2,
+                    "entry": "gqe_forward_host"},
+            "gpu_launches": launches_per_step * args.steps}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tokens, times = oracle_sample(d, args.cpu_budget)
+        sec = sum(times) / len(times)
+        line["cpu_baseline"] = {"value": tokens / sec, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+                                "sample": f"{len(times)} x one full sequence ({tokens} tokens) of the workload, fp64"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
