@@ -110,6 +110,35 @@ int gqe_route(const gqe_dims* d, const void* x, const void* Wr, const float* br,
               void* stream);
 
 /*
+ * gqe_route_noalloc -- gqe_route without a caller workspace. (The paper has no
+ * counterpart: this is a calling convenience of the library.)
+ *
+ * For callers that cannot allocate device memory on this path: for example
+ * code embedded in a host program that owns and pre-reserves all device
+ * memory, or a latency-critical loop where a cudaMalloc (which can
+ * synchronise the device) is not acceptable. The router's scratch (two int32
+ * arrays of B * ceil(T/128) * G*M counts) lives in a fixed 1 MiB array inside
+ * the library; every GPU that loads the library keeps those bytes reserved
+ * until the process exits. Arguments, outputs and results are exactly those
+ * of gqe_route.
+ *
+ * - Returns GQE_ERR_WORKSPACE, before any launch, when the scratch would
+ *   exceed 1 MiB, i.e. when 2 * B * ceil(T/128) * G*M * 4 bytes (each array
+ *   rounded up to 256 bytes) is larger than 1048576.
+ * - The first call on each device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ * - Every call on a device shares the one array and leaves its contents
+ *   behind. Nothing in it needs to start at zero (every entry is written
+ *   before it is read), but calls that overlap on the GPU (different streams
+ *   without ordering between them) race on it and give wrong token lists.
+ * - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+int gqe_route_noalloc(const gqe_dims* d, const void* x, const void* Wr,
+                      const float* br, int32_t* sel, float* w, float* margin,
+                      int32_t* seg_off, int32_t* seg_tok, int32_t* row_map,
+                      void* stream);
+
+/*
  * gqe_qproj -- dense K/V projection and the query projection of the selected
  * experts only (plus the shared head), on tcgen05 tensor cores.
  * Method: gist.science summary, "Architecture and routing", dense KV path

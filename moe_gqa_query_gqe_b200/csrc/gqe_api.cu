@@ -537,3 +537,58 @@ const char* gqe_status_string(int status) {
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// gqe_route_noalloc: gqe_route for callers that cannot allocate device memory
+// ===========================================================================
+// The router's only scratch (per-chunk expert counts and their scanned bases)
+// lives in this fixed array instead of a caller-provided workspace. Every GPU
+// that loads the library keeps these bytes reserved until the process exits.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 1u << 20;  // 1 MiB
+__device__ __align__(256) uint8_t g_route_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_route_scratch on the current device. In host code the
+// array's name only stands for it, so the address is looked up once per
+// device with that device current, then reused.
+int route_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GQE_ERR_NO_DEVICE;
+  if (dev < 0 || dev >= kMaxDevices) return GQE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || p == nullptr) return GQE_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return GQE_OK;
+}
+
+}  // namespace
+
+extern "C" int gqe_route_noalloc(const gqe_dims* d, const void* x, const void* Wr, const float* br, int32_t* sel,
+                                 float* w, float* margin, int32_t* seg_off, int32_t* seg_tok, int32_t* row_map,
+                                 void* stream) {
+  GQE_TRY(check_dims(d));
+  GQE_TRY(check_ptrs({x, Wr, sel, w, seg_off, seg_tok}));
+  if (br && !aligned16(br)) return GQE_ERR_INVALID_ARG;
+  if (margin && !aligned16(margin)) return GQE_ERR_INVALID_ARG;
+  if (row_map && !aligned16(row_map)) return GQE_ERR_INVALID_ARG;
+  Carver sizing{nullptr};
+  carve_route(sizing, d);
+  if (sizing.off > kNoAllocScratchBytes) return GQE_ERR_WORKSPACE;
+  GQE_TRY(check_device());
+  void* scratch = nullptr;
+  GQE_TRY(route_scratch(&scratch));
+  // No buffer needs zeroing: the select kernel writes every count and the
+  // scan kernel writes every base before they are read.
+  Carver c{static_cast<uint8_t*>(scratch)};
+  RouteWs rw = carve_route(c, d);
+  return do_route(d, x, Wr, br, sel, w, margin, seg_off, seg_tok, row_map, rw, static_cast<cudaStream_t>(stream));
+}

@@ -21,7 +21,7 @@ STATUS = {0: "GQE_OK", -1: "GQE_ERR_INVALID_ARG", -2: "GQE_ERR_UNSUPPORTED", -3:
 OP_ROUTE, OP_QPROJ, OP_ATTN, OP_COMBINE, OP_FORWARD, OP_DENSE, OP_FORWARD_HOST = 1, 2, 3, 4, 5, 6, 7
 
 # every symbol include/gqe.h declares
-EXPORTS = ("gqe_workspace_bytes", "gqe_validate_dims", "gqe_route", "gqe_qproj", "gqe_attn", "gqe_combine",
+EXPORTS = ("gqe_workspace_bytes", "gqe_validate_dims", "gqe_route", "gqe_route_noalloc", "gqe_qproj", "gqe_attn", "gqe_combine",
            "gqe_forward", "gqe_forward_host", "gqa_dense_forward", "gqe_check_error", "gqe_status_string",
            "gqe_version")
 
@@ -53,6 +53,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "gqe_workspace_bytes": (sz, [dp, ctypes.c_int]),
         "gqe_validate_dims": (ctypes.c_int, [dp]),
         "gqe_route": (ctypes.c_int, [dp, vp, vp, f32p, i32p, f32p, f32p, i32p, i32p, i32p, vp, sz, vp]),
+        "gqe_route_noalloc": (ctypes.c_int, [dp, vp, vp, f32p, i32p, f32p, f32p, i32p, i32p, i32p, vp]),
         "gqe_qproj": (ctypes.c_int, [dp, vp, vp, vp, vp, i32p, i32p, i32p, vp, vp, vp, vp, sz, vp]),
         "gqe_attn": (ctypes.c_int, [dp, vp, vp, vp, vp, vp, sz, vp]),
         "gqe_combine": (ctypes.c_int, [dp, vp, f32p, vp, vp, vp, sz, vp]),
@@ -118,6 +119,13 @@ def gqe_route(dims, x, Wr, br, sel, w, margin, seg_off, seg_tok, row_map, ws, st
     _call("gqe_route", ctypes.byref(dims_struct(dims)), _ptr(x), _ptr(Wr), _ptr(br), _ptr(sel), _ptr(w),
           _ptr(margin), _ptr(seg_off), _ptr(seg_tok), _ptr(row_map), _ptr(ws),
           ws.numel() if ws is not None else 0, _stream(stream))
+
+
+def gqe_route_noalloc(dims, x, Wr, br, sel, w, margin, seg_off, seg_tok, row_map, stream=None) -> None:
+    """gqe_route with its scratch in the library's fixed device array (for
+    callers that cannot allocate device memory); same outputs."""
+    _call("gqe_route_noalloc", ctypes.byref(dims_struct(dims)), _ptr(x), _ptr(Wr), _ptr(br), _ptr(sel), _ptr(w),
+          _ptr(margin), _ptr(seg_off), _ptr(seg_tok), _ptr(row_map), _stream(stream))
 
 
 def gqe_qproj(dims, x, Wq, Wk, Wv, sel, seg_off, seg_tok, Q, K, V, ws=None, stream=None) -> None:
