@@ -68,6 +68,8 @@ CONFIGS = {
     "long_b1_t32768": Dims(B=1, T=32768, D=1024, G=8, M=2, k=1),
     # 131072 tokens, pool of 4 experts per group, k = 2, skewed router.
     "skewed_b1_t131072_m4k2": Dims(B=1, T=131072, D=2048, G=8, M=4, k=2, bias0=2.0),
+    # one sequence of 8192 tokens: mid-size case for profiling captures.
+    "mid_b1_t8192": Dims(B=1, T=8192, D=1024, G=8, M=2, k=1),
     # one sequence of 1,048,576 tokens.
     "million_b1_t1048576": Dims(B=1, T=1048576, D=1024, G=8, M=2, k=1),
 }

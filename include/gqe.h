@@ -230,6 +230,10 @@ int gqa_dense_forward(const gqe_dims* d, const void* x, const void* Wq,
  * if the stream itself reported an error. */
 int gqe_check_error(void* stream);
 
+/* Description of the CUDA error behind the last GQE_ERR_CUDA returned on the
+ * calling host thread ("no error" if there was none). */
+const char* gqe_last_cuda_error(void);
+
 /* Static description of a status code. */
 const char* gqe_status_string(int status);
 

@@ -1,0 +1,446 @@
+// attn2.cuh -- causal attention of GQE's selected experts (and of the dense
+// GQA baseline), second-generation Blackwell kernel.
+//
+// Method: animattoys.com article on "Grouped Query Experts", section 4 (each
+// selected expert computes attention on its own against the K/V shared by its
+// group; the shared head is always computed); gist.science technical summary,
+// "Architecture and routing" (dense, unchanged K/V).
+//
+// Row sets (see attn.cuh): the query rows of one KV group, rr rows per token
+// (the k selected experts of the group, or all M heads in the dense baseline),
+// so the routed attention of a group is causal attention with rr rows per
+// position and stays balanced under any routing skew.
+//
+// Per CTA (persistent, one per SM, 384 threads), work item = two adjacent
+// 128-row Q tiles (A, B) of one row set; items are visited heaviest first:
+//   warp 0      TMA producer: Q_A, Q_B once per item, K/V blocks of 128
+//               positions through a STAGES-deep ring
+//   warp 1      TMEM owner; lane 0 issues, per K/V block j,
+//                 S_t(j+1) = Q_t K_{j+1}^T  (SS MMA, M=128 N=128 K=64)
+//                 O_t     += P_t(j) V_j     (TS MMA: P read from TMEM, N=64)
+//               for t = A, B
+//   warps 2..3  idle (they only hand their registers to the softmax warps)
+//   warps 4..7  softmax of tile A, warps 8..11 softmax of tile B: one thread
+//               per row; S read from TMEM (then released at once so the next
+//               S can be computed under this block's softmax), lazily
+//               rescaled online softmax in the exp2 domain, P written back to
+//               TMEM as bf16 pairs, final O / l stored as bf16.
+// TMEM columns: S_A [0,128) S_B [128,256) O_A [256,320) O_B [320,384)
+//               P_A [384,448) P_B [448,512).
+// Exponentials run on the MUFU ex2 unit. An FMA-pipe alternative for every
+// kA2PolyEvery-th column pair is kept (2^x = 2^j * p(x - j), j = round(x), p a
+// degree-3 minimax polynomial on [-1/2, 1/2], relative error 7.5e-5,
+// coefficients fitted by fit_exp2_poly.py in this directory); it is off
+// (kA2PolyEvery = 0) because every share tried measured slower here: the
+// softmax warps are latency-bound on the MMA round trips, not MUFU-bound.
+#pragma once
+
+#include "attn.cuh"
+#include "sm100.cuh"
+
+namespace gqe {
+
+constexpr int kA2Stages = 3;
+constexpr int kA2Threads = 384;
+// Register split after set-up: warpgroup 0 (TMA, MMA) gives registers back,
+// the two softmax warpgroups take them: 88*128 + 208*256 = 168*384, the
+// registers the block is launched with.
+constexpr int kA2RegsLow = 88;
+constexpr int kA2RegsHigh = 208;
+constexpr int kA2PolyEvery = 0;  // every n-th column pair uses the FMA-pipe exp2 (0: none)
+
+struct Attn2Params {
+  CUtensorMap tmQ[2];  // [B*T, Ha, 64] boxes (64, rr, 128/rr)
+  CUtensorMap tmK;     // [B*T, G, 64] box (64, 1, 128)
+  CUtensorMap tmV;
+  __nv_bfloat16* O;    // [B*T, Ha, 64]
+  int B, T, Ha, nrs, npairs_max, total_items;
+  float scale_log2;    // log2(e) / sqrt(dh)
+  AttnRowSet rs[kMaxRowSets];
+};
+
+struct A2Smem {
+  static constexpr int kQ = 0;  // Q_A, Q_B: 16 KB each
+  static constexpr int kK = 32768;
+  static constexpr int kV = kK + kA2Stages * 16384;
+  static constexpr int kBar = kV + kA2Stages * 16384;
+  static constexpr int kBytes = kBar + 512 + 1024;
+};
+
+// ---- packed fp32 helpers (sm_100 f32x2 instructions) ------------------------
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                      float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair on the FMA pipe: j = round(x) by the 1.5*2^23 shift, f = x - j
+// in [-1/2, 1/2], p(f) by Horner, exponent j added to p's bits. x is clamped
+// at -125 so the exponent add cannot underflow (2^-125 is zero for bf16 P).
+__device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 9.999280572e-01f, c1 = 6.932609677e-01f, c2 = 2.426111251e-01f, c3 = 5.517166853e-02f;
+  x0 = fmaxf(x0, -125.0f);
+  x1 = fmaxf(x1, -125.0f);
+  float t0, t1, j0, j1, f0, f1, p0, p1;
+  fadd2(t0, t1, x0, x1, kShift, kShift);
+  fadd2(j0, j1, t0, t1, -kShift, -kShift);
+  ffma2(f0, f1, j0, j1, -1.0f, -1.0f, x0, x1);
+  ffma2(p0, p1, f0, f1, c3, c3, c2, c2);
+  ffma2(p0, p1, p0, p1, f0, f1, c1, c1);
+  ffma2(p0, p1, p0, p1, f0, f1, c0, c0);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
+// 32 lanes x 64 columns store of packed bf16 pairs; waits in the same block.
+__device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,"
+      "%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,"
+      "%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]), "r"(r[32]),
+      "r"(r[33]), "r"(r[34]), "r"(r[35]), "r"(r[36]), "r"(r[37]), "r"(r[38]), "r"(r[39]), "r"(r[40]),
+      "r"(r[41]), "r"(r[42]), "r"(r[43]), "r"(r[44]), "r"(r[45]), "r"(r[46]), "r"(r[47]), "r"(r[48]),
+      "r"(r[49]), "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]), "r"(r[55]), "r"(r[56]),
+      "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]), "r"(r[63])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+struct A2Item {
+  int valid;         // 0: no work for this item index
+  int b, t0, tpt;    // batch, first token of tile A, tokens per tile
+  int nA, nB, nmax;  // K/V blocks of tile A, tile B (0 if empty), max
+  AttnRowSet rs;
+};
+
+__device__ __forceinline__ A2Item a2_decode(const Attn2Params& p, int item) {
+  A2Item it;
+  const int per_level = p.B * p.nrs;
+  const int level = item / per_level, rem = item % per_level;
+  const int rsi = rem % p.nrs;
+  it.b = rem / p.nrs;
+  it.rs = p.rs[rsi];
+  it.tpt = 128 / it.rs.rr;
+  const int npairs = (p.T + 2 * it.tpt - 1) / (2 * it.tpt);
+  const int pair = npairs - 1 - level;  // heaviest pair of every row set first
+  it.valid = pair >= 0;
+  if (!it.valid) return it;
+  it.t0 = pair * 2 * it.tpt;
+  it.nA = (min(it.t0 + it.tpt, p.T) - 1) / 128 + 1;
+  it.nB = (it.t0 + it.tpt < p.T) ? (min(it.t0 + 2 * it.tpt, p.T) - 1) / 128 + 1 : 0;
+  it.nmax = max(it.nA, it.nB);
+  return it;
+}
+
+// Static schedule over the heaviest-first item list: round r hands items
+// r*G .. r*G+G-1 to the G CTAs in forward order when r is even and in reverse
+// order when r is odd, so every CTA's heavy and light items pair up.
+__device__ __forceinline__ int a2_item_of(int round) {
+  const int g = gridDim.x;
+  return round * g + ((round & 1) ? (g - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+}
+
+__global__ void __launch_bounds__(kA2Threads, 1) attn2_fwd_kernel(const __grid_constant__ Attn2Params p) {
+  using L = A2Smem;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* k_full = bars + 2;                   // [STAGES]
+  uint64_t* v_full = k_full + kA2Stages;         // [STAGES]
+  uint64_t* kv_empty = v_full + kA2Stages;       // [STAGES]
+  uint64_t* s_full = kv_empty + kA2Stages;       // [2] (tile A, B)
+  uint64_t* s_free = s_full + 2;                 // [2]
+  uint64_t* p_full = s_free + 2;                 // [2]
+  uint64_t* pv_done = p_full + 2;                // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (tid == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < kA2Stages; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&s_free[t], 128);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&pv_done[t], 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tmQ[0]);
+    tma_prefetch_desc(&p.tmQ[1]);
+    tma_prefetch_desc(&p.tmK);
+    tma_prefetch_desc(&p.tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t sbase = smem_u32(smem);
+  if (warp < 4) {
+    setmaxnreg_dec<kA2RegsLow>();
+    if (warp == 0 && lane == 0) {
+      // ---- producer ------------------------------------------------------------
+      uint32_t kv = 0, n_items = 0;
+      bool ok = true;
+      for (int round = 0, item = a2_item_of(0); ok && item < p.total_items; item = a2_item_of(++round)) {
+        const A2Item it = a2_decode(p, item);
+        if (!it.valid) continue;
+        const int row0 = it.b * p.T;
+        if (!(ok = mbar_wait(q_empty, (n_items & 1) ^ 1, abort_flag))) break;
+        mbar_arrive_expect_tx(q_full, it.nB > 0 ? 32768 : 16384);
+        tma_load_3d(smem + L::kQ, &p.tmQ[it.rs.tm], q_full, 0, it.rs.h0, row0 + it.t0);
+        if (it.nB > 0) tma_load_3d(smem + L::kQ + 16384, &p.tmQ[it.rs.tm], q_full, 0, it.rs.h0, row0 + it.t0 + it.tpt);
+        for (int j = 0; j < it.nmax; ++j, ++kv) {
+          const int s = kv % kA2Stages;
+          if (!(ok = mbar_wait(&kv_empty[s], ((kv / kA2Stages) & 1) ^ 1, abort_flag))) break;
+          mbar_arrive_expect_tx(&k_full[s], 16384);
+          tma_load_3d(smem + L::kK + s * 16384, &p.tmK, &k_full[s], 0, it.rs.kvg, row0 + j * 128);
+          mbar_arrive_expect_tx(&v_full[s], 16384);
+          tma_load_3d(smem + L::kV + s * 16384, &p.tmV, &v_full[s], 0, it.rs.kvg, row0 + j * 128);
+        }
+        ++n_items;
+      }
+    } else if (warp == 1 && lane == 0) {
+      // ---- MMA issue -------------------------------------------------------------
+      constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false);  // Q, K both K-major
+      constexpr uint32_t idesc_o = idesc_bf16(128, 64, false, true);    // P from TMEM, V MN-major
+      uint32_t kv = 0, n_items = 0;
+      uint32_t s_cnt0 = 0, s_cnt1 = 0, pv_cnt0 = 0, pv_cnt1 = 0;  // issued so far, per tile
+      bool ok = true;
+      auto issue_s = [&](int t, uint32_t kvi) -> bool {
+        uint32_t& sc = t ? s_cnt1 : s_cnt0;
+        if (sc > 0 && !mbar_wait(&s_free[t], (sc - 1) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t qa = sbase + L::kQ + t * 16384;
+        const uint32_t ka = sbase + L::kK + (kvi % kA2Stages) * 16384;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_ss(tmem_base + t * 128, sdesc_sw128(qa + kk * 32, 16, 1024), sdesc_sw128(ka + kk * 32, 16, 1024),
+                  idesc_s, kk != 0);
+        umma_commit(&s_full[t]);
+        ++sc;
+        return true;
+      };
+      auto issue_pv = [&](int t, uint32_t kvi, bool acc) -> bool {
+        uint32_t& pc = t ? pv_cnt1 : pv_cnt0;
+        if (!mbar_wait(&p_full[t], pc & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t va = sbase + L::kV + (kvi % kA2Stages) * 16384;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tmem_base + 256 + t * 64, tmem_base + 384 + t * 64 + kk * 8, sdesc_sw128(va + kk * 2048, 8192, 1024),
+                  idesc_o, (acc || kk != 0) ? 1u : 0u);
+        umma_commit(&pv_done[t]);
+        ++pc;
+        return true;
+      };
+      for (int round = 0, item = a2_item_of(0); ok && item < p.total_items; item = a2_item_of(++round)) {
+        const A2Item it = a2_decode(p, item);
+        if (!it.valid) continue;
+        if (!(ok = mbar_wait(q_full, n_items & 1, abort_flag))) break;
+        const uint32_t kv0 = kv;
+        if (!(ok = mbar_wait(&k_full[kv0 % kA2Stages], (kv0 / kA2Stages) & 1, abort_flag))) break;
+        tc_fence_after();
+        ok = issue_s(0, kv0) && (it.nB == 0 || issue_s(1, kv0));
+        for (int j = 0; ok && j < it.nmax; ++j) {
+          const uint32_t kvj = kv0 + j;
+          if (j + 1 < it.nmax) {
+            if (!(ok = mbar_wait(&k_full[(kvj + 1) % kA2Stages], ((kvj + 1) / kA2Stages) & 1, abort_flag))) break;
+            if (j + 1 < it.nA && !(ok = issue_s(0, kvj + 1))) break;
+            if (j + 1 < it.nB && !(ok = issue_s(1, kvj + 1))) break;
+          }
+          if (!(ok = mbar_wait(&v_full[kvj % kA2Stages], (kvj / kA2Stages) & 1, abort_flag))) break;
+          if (j < it.nA && !(ok = issue_pv(0, kvj, j > 0))) break;
+          if (j < it.nB && !(ok = issue_pv(1, kvj, j > 0))) break;
+          umma_commit(&kv_empty[kvj % kA2Stages]);
+        }
+        umma_commit(q_empty);
+        kv += it.nmax;
+        ++n_items;
+      }
+    }
+  } else {
+    setmaxnreg_inc<kA2RegsHigh>();
+    // ---- softmax warpgroups: warps 4..7 -> tile A, 8..11 -> tile B --------------
+    const int t = (warp - 4) >> 2;
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int row = q * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t tm_s = tmem_base + lane_off + t * 128;
+    const uint32_t tm_o = tmem_base + lane_off + 256 + t * 64;
+    const uint32_t tm_p = tmem_base + lane_off + 384 + t * 64;
+    const float sl2 = p.scale_log2;
+    uint32_t cnt = 0;  // blocks processed by this tile so far (barrier phases)
+    bool ok = true;
+    for (int round = 0, item = a2_item_of(0); ok && item < p.total_items; item = a2_item_of(++round)) {
+      const A2Item it = a2_decode(p, item);
+      if (!it.valid) continue;
+      const int nblk = t == 0 ? it.nA : it.nB;
+      if (nblk == 0) continue;
+      const int tfirst = it.t0 + t * it.tpt;      // first token of this tile
+      const int tok = tfirst + row / it.rs.rr;    // token of this row (>= T: not stored)
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int j = 0; j < nblk; ++j, ++cnt) {
+        bool w_ok = mbar_wait(&s_full[t], cnt & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+        tc_fence_after();
+        float s[128];
+        tmem_ld128f(tm_s, s);
+        tc_fence_before();
+        mbar_arrive(&s_free[t]);  // S may be overwritten by the next block's QK^T now
+
+        const int kv0 = j * 128;
+        if (kv0 + 127 > tfirst) {
+          const int lim = tok - kv0;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c > lim) s[c] = -INFINITY;
+        }
+        float m4[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+        for (int c = 4; c < 128; c += 8) {
+          m4[0] = fmax3(m4[0], s[c], s[c + 1]);
+          m4[1] = fmax3(m4[1], s[c + 2], s[c + 3]);
+          m4[2] = fmax3(m4[2], s[c + 4], s[c + 5]);
+          m4[3] = fmax3(m4[3], s[c + 6], s[c + 7]);
+        }
+        const float mx = fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
+        const float m_new = fmaxf(m_run, mx * sl2);
+        const float m_use = (m_new > m_run + kRescaleThreshold) ? m_new : m_run;
+        const float alpha = ex2_approx(m_run - m_use);
+        const bool rescale = (j > 0) && (m_use != m_run);
+        m_run = m_use;
+
+        // x = s * scale_log2 - m, then 2^x: MUFU for most pairs, FMA pipe for some
+        float sm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 4 independent pair chains
+        uint32_t pk[64];
+#pragma unroll
+        for (int pi = 0; pi < 64; ++pi) {
+          float x0, x1, y0, y1;
+          ffma2(x0, x1, s[2 * pi], s[2 * pi + 1], sl2, sl2, -m_use, -m_use);
+          bool poly = false;
+          if constexpr (kA2PolyEvery > 0) poly = (pi % kA2PolyEvery) == kA2PolyEvery - 1;
+          if (poly) {
+            exp2_poly2(y0, y1, x0, x1);
+          } else {
+            y0 = ex2_approx(x0);
+            y1 = ex2_approx(x1);
+          }
+          fadd2(sm[2 * (pi & 3)], sm[2 * (pi & 3) + 1], sm[2 * (pi & 3)], sm[2 * (pi & 3) + 1], y0, y1);
+          pk[pi] = pack_bf16x2(y0, y1);
+        }
+        l_run = l_run * alpha + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
+
+        // P(j) overwrites P(j-1) and O may need rescaling: both need PV(j-1) done
+        if (j > 0) {
+          w_ok = mbar_wait(&pv_done[t], (cnt - 1) & 1, abort_flag);
+          if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              uint32_t o[16];
+              tmem_ld16(tm_o + h * 16, o);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+              tmem_st16(tm_o + h * 16, o);
+            }
+          }
+        }
+        tmem_st64(tm_p, pk);
+        tc_fence_before();
+        mbar_arrive(&p_full[t]);
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l -> bf16 ------------------------------------------------
+      const bool w_ok = mbar_wait(&pv_done[t], (cnt - 1) & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+      tc_fence_after();
+      const float inv = 1.f / l_run;
+      __nv_bfloat16* dst =
+          (tok < p.T) ? p.O + ((size_t)(it.b * p.T + tok) * p.Ha + it.rs.h0 + (row % it.rs.rr)) * 64 : nullptr;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t o[32];
+        tmem_ld32(tm_o + h * 32, o);
+        if (dst) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            st_global_v4(dst + h * 32 + i * 8, pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+      }
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    const unsigned long long t0n = globaltimer_ns();
+    while (globaltimer_ns() - t0n < 100000ull) {}
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace gqe

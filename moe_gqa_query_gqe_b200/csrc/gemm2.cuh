@@ -1,0 +1,340 @@
+// gemm2.cuh -- persistent tcgen05 GEMM for the GQE projections:
+// C = A * B, bf16 in, fp32 accumulate in TMEM, bf16 out.
+//
+//   A [rows, K] row-major (K-major operand): TMA tiles (dense rows), or rows
+//     gathered by a segment's token list with TMA tile::gather4 (the
+//     selected-expert query projection: only tokens that picked the expert are
+//     multiplied; each lane of the producer warp gathers 4 of the 128 rows).
+//   B [K, N] row-major weight (MN-major operand), 64 x 64 TMA boxes, 128-byte
+//     swizzle. The MMA N of a tile is the segment's remaining width rounded
+//     up to 64 (no work on columns past the segment).
+//   Tiles of 128 x BN; persistent CTAs walk the tile list round-robin. The
+//   TMEM accumulator is double-buffered (2 x BN columns), so the epilogue of
+//   one tile overlaps the main loop of the next.
+//
+// Warp roles (one CTA per SM, 192 threads):
+//   warp 0     : TMA producer (lane 0; all 32 lanes issue the row gathers)
+//   warp 1     : TMEM allocation + MMA issue (lane 0)
+//   warps 2..5 : epilogue (TMEM lanes 32*(warp%4) .. +31)
+#pragma once
+
+#include "gemm.cuh"
+#include "sm100.cuh"
+
+namespace gqe {
+
+constexpr int kG2MaxSegsSmem = 8192;  // gather mode: segment tile prefix kept in shared memory
+
+template <int BN, int STAGES, int AMODE>
+struct G2Cfg {
+  // kAGatherLsu: 8 more warps copy the gathered A rows with cp.async
+  static constexpr int kThreads = AMODE == kAGatherLsu ? 448 : 192;
+  static constexpr int kABytes = kGemmBM * kGemmBK * 2;  // 16 KB
+  static constexpr int kBBytes = BN * kGemmBK * 2;       // BN/64 boxes of 8 KB
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kBarOffset = STAGES * kStageBytes;
+  static constexpr int kPrefixOffset = kBarOffset + 256;
+  static constexpr int kBytesBase = kPrefixOffset + 1024;  // + (nsegs+1)*4 in gather mode
+};
+
+struct G2Tile {
+  int m0;        // first row (dense) / first compacted row offset within the segment (gather)
+  int seg;       // dense: output segment; gather: expert segment
+  int n0;        // first column of the segment
+  int nvalid;    // columns computed (multiple of 64, <= BN)
+  int row0, row_end;  // gather: compacted row range of the tile
+};
+
+template <int BN>
+__device__ __forceinline__ G2Tile g2_decode(const GemmParams& p, int tile, const int* s_prefix) {
+  G2Tile t;
+  if (s_prefix == nullptr) {
+    const int mt = tile / p.ntn, nt = tile % p.ntn;
+    t.m0 = mt * kGemmBM;
+    t.seg = 0;
+    for (int s = 1; s < p.nseg; ++s)
+      if (nt >= p.seg[s].tile_start) t.seg = s;
+    t.n0 = (nt - p.seg[t.seg].tile_start) * BN;
+    const int rem = p.seg[t.seg].n_cols - t.n0;
+    t.nvalid = rem >= BN ? BN : ((rem + 63) / 64) * 64;
+    t.row0 = t.row_end = 0;
+  } else {
+    // largest s with s_prefix[s] <= tile
+    int lo = 0, hi = p.nsegs_q - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_prefix[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    t.seg = lo;
+    const int mt = tile - s_prefix[lo];
+    t.m0 = mt * kGemmBM;
+    t.row0 = p.seg_off[lo] + t.m0;
+    t.row_end = min(p.seg_off[lo + 1], p.seg_off[p.nsegs_q]);
+    t.n0 = 0;
+    t.nvalid = 64;
+  }
+  return t;
+}
+
+template <int BN, int STAGES, int AMODE>
+__global__ void __launch_bounds__(G2Cfg<BN, STAGES, AMODE>::kThreads, 1)
+    gemm2_kernel(const __grid_constant__ GemmParams p, int total_tiles) {
+  using C = G2Cfg<BN, STAGES, AMODE>;
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;   // [2]
+  uint64_t* acc_empty = acc_full + 2;    // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_prefix = reinterpret_cast<int*>(smem + C::kPrefixOffset);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nk = (p.K + kGemmBK - 1) / kGemmBK;
+
+  if constexpr (AMODE != kATma) {
+    // tile prefix over the expert segments: s_prefix[s] = tiles before segment s
+    if (warp == 0) {
+      int before = 0;
+      for (int s0 = 0; s0 < p.nsegs_q; s0 += 32) {
+        const int s = s0 + lane;
+        const int len = s < p.nsegs_q ? p.seg_off[s + 1] - p.seg_off[s] : 0;
+        const int nt = (len + kGemmBM - 1) / kGemmBM;
+        int incl = nt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int u = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += u;
+        }
+        if (s < p.nsegs_q) s_prefix[s] = before + incl - nt;
+        before += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) s_prefix[p.nsegs_q] = before;
+    }
+  }
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], AMODE == kAGatherLsu ? 1 + 256 : 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 2 * BN);
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tmA);
+    for (int s = 0; s < (AMODE == kATma ? p.nseg : 1); ++s) tma_prefetch_desc(&p.tmB[s]);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t smem_base = smem_u32(smem);
+  int ntiles = total_tiles;
+  if constexpr (AMODE != kATma) ntiles = min(total_tiles, s_prefix[p.nsegs_q]);
+  const int* prefix = AMODE != kATma ? s_prefix : nullptr;
+
+  if (warp == 0) {
+    // ---- TMA producer: A tiles (dense rows or gathered rows) and B tiles -------
+    uint32_t it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+      const G2Tile t = g2_decode<BN>(p, tile, prefix);
+      int b_col;
+      const CUtensorMap* tmb;
+      int tk0 = 0, tk1 = 0, tk2 = 0, tk3 = 0;
+      if constexpr (AMODE == kATma) {
+        b_col = p.seg[t.seg].b_col0 + t.n0;
+        tmb = &p.tmB[t.seg];
+      } else if constexpr (AMODE == kAGatherLsu) {
+        b_col = (t.seg % (p.G * p.M)) * 64;
+        tmb = &p.tmB[0];
+      } else {
+        b_col = (t.seg % (p.G * p.M)) * 64;  // head h = g*M + e of segment (b, g, e)
+        tmb = &p.tmB[0];
+        // rows 4*lane .. 4*lane+3 of the tile; rows past the segment re-read its
+        // first token (their results are never stored)
+        int tk[4];
+        const int first = p.seg_tok[t.row0];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int ci = t.row0 + 4 * lane + i;
+          int v = ci < t.row_end ? p.seg_tok[ci] : first;
+          if (v < 0 || v >= p.ntok) {
+            flag_bounds_error();
+            v = 0;
+          }
+          tk[i] = v;
+        }
+        tk0 = tk[0];
+        tk1 = tk[1];
+        tk2 = tk[2];
+        tk3 = tk[3];
+      }
+      const int nbox = t.nvalid / 64;
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = it % STAGES;
+        bool w_ok = true;
+        if (lane == 0) w_ok = mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort_flag);
+        if (!(ok = __shfl_sync(0xffffffffu, w_ok, 0))) break;
+        uint8_t* a_s = smem + s * C::kStageBytes;
+        uint8_t* b_s = a_s + C::kABytes;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[s], (AMODE == kAGatherLsu ? 0 : C::kABytes) + nbox * 8192);
+          if constexpr (AMODE == kATma) tma_load_2d(a_s, &p.tmA, &full[s], kb * kGemmBK, t.m0);
+          for (int nb = 0; nb < nbox; ++nb)
+            tma_load_2d(b_s + nb * 8192, tmb, &full[s], b_col + nb * 64, kb * kGemmBK);
+        }
+        if constexpr (AMODE == kAGather) {
+          __syncwarp();
+          tma_gather4(a_s + lane * 512, &p.tmA, &full[s], kb * kGemmBK, tk0, tk1, tk2, tk3);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---- MMA issue ------------------------------------------------------------
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++tcount) {
+        const G2Tile t = g2_decode<BN>(p, tile, prefix);
+        const uint32_t a = tcount & 1;
+        if (!(ok = mbar_wait(&acc_empty[a], ((tcount >> 1) & 1) ^ 1, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + a * BN;
+        const uint32_t idesc = idesc_bf16(kGemmBM, t.nvalid, false, true);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (!(ok = mbar_wait(&full[s], (it / STAGES) & 1, abort_flag))) break;
+          // rows copied by cp.async (generic proxy) are read by the MMA (async proxy)
+          if constexpr (AMODE == kAGatherLsu) fence_proxy_async_smem();
+          tc_fence_after();
+          const uint32_t a_addr = smem_base + s * C::kStageBytes;
+          const uint32_t b_addr = a_addr + C::kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kGemmBK / 16; ++kk)
+            umma_ss(d_tmem, sdesc_sw128(a_addr + kk * 32, 16, 1024), sdesc_sw128(b_addr + kk * 2048, 8192, 1024),
+                    idesc, (kb | kk) != 0);
+          umma_commit(&empty[s]);
+        }
+        umma_commit(&acc_full[a]);
+      }
+    }
+  } else if (warp >= 6) {
+    if constexpr (AMODE == kAGatherLsu) {
+      // ---- A copiers (warps 6..13): 16-byte chunk c of rows r = i*32 + ct/8 -------
+      // The token rows of the next tile are fetched while this tile's copies run,
+      // so no copier waits on a token-list load at a tile boundary.
+      const int ct = tid - 192;  // 0..255
+      const int c = ct & 7;
+      uint32_t it = 0;
+      bool ok = true;
+      auto fetch_rows = [&](int tile, int (&tk)[4]) {
+        const G2Tile t = g2_decode<BN>(p, tile, prefix);
+        const int first = p.seg_tok[t.row0];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = i * 32 + (ct >> 3);
+          tk[i] = (t.row0 + r < t.row_end) ? p.seg_tok[t.row0 + r] : first;
+        }
+      };
+      int tk_cur[4] = {0, 0, 0, 0}, tk_next[4] = {0, 0, 0, 0};
+      if ((int)blockIdx.x < ntiles) fetch_rows(blockIdx.x, tk_cur);
+      for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+        if (tile + (int)gridDim.x < ntiles) fetch_rows(tile + gridDim.x, tk_next);
+        uint32_t dst_off[4];
+        const __nv_bfloat16* src[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = i * 32 + (ct >> 3);
+          int v = tk_cur[i];
+          if (v < 0 || v >= p.ntok) {
+            flag_bounds_error();
+            v = 0;
+          }
+          src[i] = p.x + (size_t)v * p.K + c * 8;
+          dst_off[i] = r * 128 + ((c ^ (r & 7)) << 4);
+        }
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (!(ok = mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort_flag))) break;
+          const uint32_t a_addr = smem_base + s * C::kStageBytes;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) cp_async_16_full(a_addr + dst_off[i], src[i] + kb * kGemmBK);
+          cp_async_mbar_arrive_noinc(&full[s]);  // arrives when these copies land; no wait here
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tk_cur[i] = tk_next[i];
+      }
+      asm volatile("cp.async.wait_all;" ::: "memory");  // nothing may be in flight when the CTA exits
+    }
+  } else {
+    // ---- epilogue ---------------------------------------------------------------
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    uint32_t tcount = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tcount) {
+      const G2Tile t = g2_decode<BN>(p, tile, prefix);
+      const uint32_t a = tcount & 1;
+      const bool ok = mbar_wait(&acc_full[a], (tcount >> 1) & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      __nv_bfloat16* dst_row = nullptr;
+      if constexpr (AMODE == kATma) {
+        const GemmSeg& sg = p.seg[t.seg];
+        if (t.m0 + row < p.rows) dst_row = sg.C + (size_t)(t.m0 + row) * sg.ldc + sg.c_col0 + t.n0;
+      } else {
+        const int ci = t.row0 + row;
+        if (ci < t.row_end) {
+          const int GM = p.G * p.M;
+          const int n = p.seg_tok[ci];
+          const int g = (t.seg % GM) / p.M, e = t.seg % p.M;
+          if (n >= 0 && n < p.ntok) {
+            int j = 0;
+            for (int jj = 0; jj < p.k; ++jj)
+              if (p.sel[((size_t)n * p.G + g) * p.k + jj] == e) j = jj;
+            dst_row = p.Q + ((size_t)n * p.Ha + g * p.k + j) * 64;
+          } else {
+            flag_bounds_error();
+          }
+        }
+      }
+      int ncols = t.nvalid;
+      if constexpr (AMODE == kATma) ncols = min(t.nvalid, p.seg[t.seg].n_cols - t.n0);
+      const uint32_t tm = tmem_base + a * BN + (static_cast<uint32_t>(q * 32) << 16);
+      for (int cc = 0; cc < t.nvalid / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tm + cc * 32, r);
+        if (dst_row != nullptr && cc * 32 < ncols) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+          __nv_bfloat16* d = dst_row + cc * 32;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) st_global_v4(d + i * 8, pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[a]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    const unsigned long long t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 100000ull) {}
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 2 * BN);
+  }
+}
+
+}  // namespace gqe

@@ -13,15 +13,14 @@
 #include "sm100.cuh"
 #include "route.cuh"
 #include "gemm.cuh"
+#include "gemm2.cuh"
 #include "attn.cuh"
+#include "attn2.cuh"
 #include "combine.cuh"
 
 using namespace gqe;
 
 namespace {
-
-constexpr int kGemmStages = 4;
-constexpr int kQProjStages = 4;
 
 inline bool pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
 inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
@@ -100,25 +99,38 @@ int tmap_heads(CUtensorMap* tm, const void* base, long long N, int H, int bh, in
 // ---------------------------------------------------------------------------
 // Launch helpers
 // ---------------------------------------------------------------------------
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+inline int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return GQE_OK;
+  g_last_cuda_error = e;
+  return GQE_ERR_CUDA;
+}
+inline int launch_status() { return cuda_status(cudaGetLastError()); }
+
 template <typename K>
 int set_smem(K kernel, int bytes) {
   // cheap after the first call on a device; keeps multi-device use correct
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
-             ? GQE_OK
-             : GQE_ERR_CUDA;
+  return cuda_status(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
 }
 
-inline int launch_status() { return cudaGetLastError() == cudaSuccess ? GQE_OK : GQE_ERR_CUDA; }
 
-template <int BN, int AMODE>
-int launch_gemm(const GemmParams& p, long long grid, cudaStream_t st) {
-  constexpr int STAGES = AMODE == kATma ? kGemmStages : kQProjStages;
-  auto kern = gemm_bf16_kernel<BN, STAGES, AMODE>;
-  const int smem = GemmSmem<BN, STAGES>::kBytes;
+constexpr int kG2DenseBN = 256, kG2DenseStages = 4;
+constexpr int kG2GatherStages = 8;
+constexpr int kG2GatherMode = kAGatherLsu;
+
+int sm_count();
+
+template <int BN, int STAGES, int AMODE>
+int launch_gemm2(const GemmParams& p, long long tiles, cudaStream_t st) {
+  using C = G2Cfg<BN, STAGES, AMODE>;
+  auto kern = gemm2_kernel<BN, STAGES, AMODE>;
+  const int smem = C::kBytesBase + (AMODE != kATma ? (p.nsegs_q + 1) * 4 : 0);
   if (int e = set_smem(kern, smem)) return e;
-  if (grid <= 0) return GQE_OK;
-  if (grid > 0x7fffffffll) return GQE_ERR_UNSUPPORTED;
-  kern<<<(unsigned)grid, kGemmThreads, smem, st>>>(p);
+  if (tiles <= 0) return GQE_OK;
+  if (tiles > 0x7fffffffll) return GQE_ERR_UNSUPPORTED;
+  const int grid = (int)std::min<long long>(tiles, sm_count());
+  kern<<<grid, C::kThreads, smem, st>>>(p, (int)tiles);
   return launch_status();
 }
 
@@ -146,13 +158,13 @@ int gemm_dense(const void* A, long long rows, int K, const DenseSeg* segs, int n
     p.seg[s].ldc = segs[s].ldc;
     p.seg[s].C = static_cast<__nv_bfloat16*>(segs[s].C);
     p.seg[s].tile_start = nt;
-    nt += (int)cdiv(segs[s].n_cols, 128);
+    nt += (int)cdiv(segs[s].n_cols, kG2DenseBN);
   }
   p.nseg = nseg;
   p.ntn = nt;
   p.rows = (int)rows;
   p.K = K;
-  return launch_gemm<128, kATma>(p, cdiv(rows, kGemmBM) * nt, st);
+  return launch_gemm2<kG2DenseBN, kG2DenseStages, kATma>(p, cdiv(rows, kGemmBM) * nt, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -314,6 +326,7 @@ int do_qproj(const gqe_dims* d, const void* x, const void* Wq, const void* Wk, c
   GemmParams p;
   memset(&p, 0, sizeof(p));
   GQE_TRY(tmap_rows(&p.tmB[0], Wq, d->D, wq_cols, wq_cols, 64));
+  GQE_TRY(tmap_rows(&p.tmA, x, N, d->D, d->D, 1));  // one-row box: gathered 4 rows at a time
   p.K = d->D;
   p.x = static_cast<const __nv_bfloat16*>(x);
   p.seg_off = seg_off;
@@ -327,13 +340,20 @@ int do_qproj(const gqe_dims* d, const void* x, const void* Wq, const void* Wk, c
   p.Ha = Ha;
   p.ntok = (int)N;
   const long long tiles_max = cdiv(N * G * k, kGemmBM) + p.nsegs_q;
-  return launch_gemm<64, kAGather>(p, tiles_max, st);
+  return launch_gemm2<64, kG2GatherStages, kG2GatherMode>(p, tiles_max, st);
 }
 
-int do_attn(const gqe_dims* d, const void* Q, int Hq, const void* K, const void* V, void* O, bool dense,
-            cudaStream_t st) {
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// Persistent two-tile attention (attn2.cuh).
+int do_attn2(const gqe_dims* d, const void* Q, int Hq, const void* K, const void* V, void* O, bool dense,
+             cudaStream_t st) {
   const long long N = (long long)d->B * d->T;
-  AttnParams p;
+  Attn2Params p;
   memset(&p, 0, sizeof(p));
   const int rr = dense ? d->M : d->k;
   GQE_TRY(tmap_heads(&p.tmQ[0], Q, N, Hq, rr, 128 / rr));
@@ -348,13 +368,14 @@ int do_attn(const gqe_dims* d, const void* Q, int Hq, const void* K, const void*
   for (int g = 0; g < d->G; ++g) p.rs[nrs++] = AttnRowSet{g * rr, rr, g, 0};
   if (!dense) p.rs[nrs++] = AttnRowSet{d->G * d->k, 1, 0, 1};
   p.nrs = nrs;
-  p.nqt_max = (int)cdiv((long long)d->T * rr, 128);
+  p.npairs_max = (int)cdiv((long long)d->T * rr, 256);
+  const long long items = (long long)p.npairs_max * d->B * nrs;
+  if (items > 0x7fffffffll) return GQE_ERR_UNSUPPORTED;
+  p.total_items = (int)items;
   p.scale_log2 = 1.4426950408889634f / sqrtf(64.f);
-  GQE_TRY(set_smem(attn_fwd_kernel, AttnSmem::kBytes));
-  const long long gx = (long long)d->B * nrs;
-  if (gx > 0x7fffffffll || p.nqt_max > 65535) return GQE_ERR_UNSUPPORTED;
-  dim3 grid((unsigned)gx, (unsigned)p.nqt_max);
-  attn_fwd_kernel<<<grid, kAttnThreads, AttnSmem::kBytes, st>>>(p);
+  GQE_TRY(set_smem(attn2_fwd_kernel, A2Smem::kBytes));
+  const int grid = (int)std::min<long long>(items, sm_count());
+  attn2_fwd_kernel<<<grid, kA2Threads, A2Smem::kBytes, st>>>(p);
   return launch_status();
 }
 
@@ -441,7 +462,7 @@ int gqe_attn(const gqe_dims* d, const void* Q, const void* K, const void* V, voi
   GQE_TRY(check_dims(d));
   GQE_TRY(check_ptrs({Q, K, V, O}));
   GQE_TRY(check_device());
-  return do_attn(d, Q, d->G * d->k + 1, K, V, O, false, static_cast<cudaStream_t>(stream));
+  return do_attn2(d, Q, d->G * d->k + 1, K, V, O, false, static_cast<cudaStream_t>(stream));
 }
 
 int gqe_combine(const gqe_dims* d, const void* O, const float* w, const void* Wo, void* y, void* ws, size_t ws_bytes,
@@ -465,7 +486,7 @@ int gqe_forward(const gqe_dims* d, const void* x, const void* Wq, const void* Wk
   FwdWs f = carve_forward(c, d);
   GQE_TRY(do_route(d, x, Wr, br, f.sel, f.w, f.margin, f.seg_off, f.seg_tok, f.row_map, f.route, st));
   GQE_TRY(do_qproj(d, x, Wq, Wk, Wv, f.sel, f.seg_off, f.seg_tok, f.Q, f.K, f.V, st));
-  GQE_TRY(do_attn(d, f.Q, d->G * d->k + 1, f.K, f.V, f.O, false, st));
+  GQE_TRY(do_attn2(d, f.Q, d->G * d->k + 1, f.K, f.V, f.O, false, st));
   return do_combine(d, f.O, f.w, Wo, y, f.A, st);
 }
 
@@ -481,9 +502,9 @@ int gqe_forward_host(const gqe_dims* d, const void* x_host, const void* Wq, cons
   void* x_dev = c.take<__nv_bfloat16>((size_t)d->B * d->T * d->D);
   void* y_dev = c.take<__nv_bfloat16>((size_t)d->B * d->T * d->D);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemcpyAsync(x_dev, x_host, xbytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return GQE_ERR_CUDA;
+  GQE_TRY(cuda_status(cudaMemcpyAsync(x_dev, x_host, xbytes, cudaMemcpyHostToDevice, st)));
   GQE_TRY(gqe_forward(d, x_dev, Wq, Wk, Wv, Wr, br, Wo, y_dev, ws, ws_bytes, stream));
-  if (cudaMemcpyAsync(y_host, y_dev, xbytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return GQE_ERR_CUDA;
+  GQE_TRY(cuda_status(cudaMemcpyAsync(y_host, y_dev, xbytes, cudaMemcpyDeviceToHost, st)));
   return GQE_OK;
 }
 
@@ -505,15 +526,15 @@ int gqa_dense_forward(const gqe_dims* d, const void* x, const void* Wq, const vo
       {Wv, G * 64, 0, G * 64, w.V, (long long)G * 64, 0},
   };
   GQE_TRY(gemm_dense(x, N, d->D, segs, 3, st));
-  GQE_TRY(do_attn(d, w.Q, H, w.K, w.V, w.O, true, st));
+  GQE_TRY(do_attn2(d, w.Q, H, w.K, w.V, w.O, true, st));
   const DenseSeg so = {Wo_dense, d->D, 0, d->D, y, (long long)d->D, 0};
   return gemm_dense(w.O, N, H * 64, &so, 1, st);
 }
 
 int gqe_check_error(void* stream) {
-  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return GQE_ERR_CUDA;
+  GQE_TRY(cuda_status(cudaStreamSynchronize(static_cast<cudaStream_t>(stream))));
   int word = 0;
-  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(int)) != cudaSuccess) return GQE_ERR_CUDA;
+  GQE_TRY(cuda_status(cudaMemcpyFromSymbol(&word, g_error_word, sizeof(int))));
   if (word != 0) {
     const int zero = 0;
     cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int));
@@ -521,6 +542,8 @@ int gqe_check_error(void* stream) {
   }
   return GQE_OK;
 }
+
+const char* gqe_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_error); }
 
 const char* gqe_status_string(int status) {
   switch (status) {

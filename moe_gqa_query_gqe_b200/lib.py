@@ -22,7 +22,7 @@ OP_ROUTE, OP_QPROJ, OP_ATTN, OP_COMBINE, OP_FORWARD, OP_DENSE, OP_FORWARD_HOST =
 
 # every symbol include/gqe.h declares
 EXPORTS = ("gqe_workspace_bytes", "gqe_validate_dims", "gqe_route", "gqe_route_noalloc", "gqe_qproj", "gqe_attn", "gqe_combine",
-           "gqe_forward", "gqe_forward_host", "gqa_dense_forward", "gqe_check_error", "gqe_status_string",
+           "gqe_forward", "gqe_forward_host", "gqa_dense_forward", "gqe_check_error", "gqe_status_string", "gqe_last_cuda_error",
            "gqe_version")
 
 
@@ -31,8 +31,8 @@ class GqeDims(ctypes.Structure):
 
 
 class GqeError(RuntimeError):
-    def __init__(self, fn: str, code: int):
-        super().__init__(f"{fn} failed: {STATUS.get(code, code)} ({code})")
+    def __init__(self, fn: str, code: int, detail: str = ""):
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)} ({code}){': ' + detail if detail else ''}")
         self.code = code
 
 
@@ -62,6 +62,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "gqa_dense_forward": (ctypes.c_int, [dp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "gqe_check_error": (ctypes.c_int, [vp]),
         "gqe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "gqe_last_cuda_error": (ctypes.c_char_p, []),
         "gqe_version": (ctypes.c_int, []),
     }
     for name, (res, args) in sig.items():
@@ -98,7 +99,8 @@ def _stream(stream) -> int:
 def _call(name: str, *args) -> None:
     code = getattr(load(), name)(*args)
     if code != GQE_OK:
-        raise GqeError(name, code)
+        detail = load().gqe_last_cuda_error().decode() if code == -4 else ""
+        raise GqeError(name, code, detail)
 
 
 def workspace_bytes(dims, op: int) -> int:
