@@ -30,7 +30,7 @@
  *    recorded in a sticky per-device error word read by gqe_check_error().
  *
  * Supported shapes (others return GQE_ERR_UNSUPPORTED): dh == 64;
- * D % 64 == 0; 1 <= k <= M; G*M a power of two <= 64; k and M in {1,2,4,8}
+ * D % 64 == 0; 1 <= k <= M; G*M a power of two in [8, 64]; k and M in {1,2,4,8}
  * (128 must be a multiple of the rows each token contributes to one
  * attention tile); B*T < 2^31 / (G*k+1) / 64.
  */

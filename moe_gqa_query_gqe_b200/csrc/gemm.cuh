@@ -39,6 +39,15 @@ struct GemmParams {
   __nv_bfloat16* Q;        // [B*T, Ha, dh]
   int nsegs_q, G, M, k, Ha;
   int ntok;  // B*T: bound of every token index read from seg_tok
+  // routing epilogue (router logits x Wr on the tensor cores)
+  const float* r_br;   // [G*M] or null
+  int32_t* r_sel;      // [B*T, G, k]
+  float* r_w;          // [B*T, G, k]
+  float* r_margin;     // [B*T, G] or null
+  int32_t* r_counts;   // [B][nch][G*M]
+  int r_B, r_T, r_nch;
 };
+
+enum GemmEpilogue : int { kEpiStore = 0, kEpiRoute = 1 };
 
 }  // namespace gqe

@@ -34,9 +34,9 @@ int check_dims(const gqe_dims* d) {
   if (d->dh != 64) return GQE_ERR_UNSUPPORTED;
   if (d->D % 64 != 0) return GQE_ERR_UNSUPPORTED;
   const int GM = d->G * d->M;
-  if (GM < 2 || GM > 64 || !pow2(GM)) return GQE_ERR_UNSUPPORTED;
+  // 8 <= G*M: the router weight's rows must be a multiple of 16 bytes for TMA
+  if (GM < 8 || GM > 64 || !pow2(GM)) return GQE_ERR_UNSUPPORTED;
   if (!pow2(d->M) || d->M > 8 || !pow2(d->k) || d->k > 8) return GQE_ERR_UNSUPPORTED;
-  if ((long long)d->D * GM * 2 > kRouteMaxWrBytes) return GQE_ERR_UNSUPPORTED;
   if ((long long)d->B * GM > 8192) return GQE_ERR_UNSUPPORTED;
   const long long N = (long long)d->B * d->T;
   if (N * d->G * d->k >= (1ll << 31) || N * (d->G * d->M + 1) >= (1ll << 31)) return GQE_ERR_UNSUPPORTED;
@@ -116,16 +116,17 @@ int set_smem(K kernel, int bytes) {
 
 
 constexpr int kG2DenseBN = 256, kG2DenseStages = 4;
+constexpr int kRouteStages = 8;
 constexpr int kG2GatherStages = 8;
 constexpr int kG2GatherMode = kAGatherLsu;
 
 int sm_count();
 
-template <int BN, int STAGES, int AMODE>
+template <int BN, int STAGES, int AMODE, int EPI = kEpiStore>
 int launch_gemm2(const GemmParams& p, long long tiles, cudaStream_t st) {
   using C = G2Cfg<BN, STAGES, AMODE>;
-  auto kern = gemm2_kernel<BN, STAGES, AMODE>;
-  const int smem = C::kBytesBase + (AMODE != kATma ? (p.nsegs_q + 1) * 4 : 0);
+  auto kern = gemm2_kernel<BN, STAGES, AMODE, EPI>;
+  const int smem = C::kBytesBase + (AMODE != kATma ? (p.nsegs_q + 1) * 4 : 0) + (EPI == kEpiRoute ? 64 * 4 : 0);
   if (int e = set_smem(kern, smem)) return e;
   if (tiles <= 0) return GQE_OK;
   if (tiles > 0x7fffffffll) return GQE_ERR_UNSUPPORTED;
@@ -261,26 +262,10 @@ int check_device() {
 // ---------------------------------------------------------------------------
 // Stage implementations (arguments already validated)
 // ---------------------------------------------------------------------------
-template <int GM>
-int launch_route_select(const RouteParams& rp, long long grid, cudaStream_t st) {
-  constexpr int TPW = (64 / GM) < 1 ? 1 : ((64 / GM) > 16 ? 16 : (64 / GM));
-  constexpr int V = TPW * GM;
-  const int smem = rp.D * GM * 2 + kRouteWarps * V * 4 + GM * 4;
-  auto kern = route_select_kernel<GM>;
-  GQE_TRY(set_smem(kern, smem));
-  kern<<<(unsigned)grid, kRouteWarps * 32, smem, st>>>(rp);
-  return launch_status();
-}
-
 int do_route(const gqe_dims* d, const void* x, const void* Wr, const float* br, int32_t* sel, float* w,
              float* margin, int32_t* seg_off, int32_t* seg_tok, int32_t* row_map, RouteWs rw, cudaStream_t st) {
   RouteParams rp;
-  rp.x = static_cast<const __nv_bfloat16*>(x);
-  rp.Wr = static_cast<const __nv_bfloat16*>(Wr);
-  rp.br = br;
   rp.sel = sel;
-  rp.w = w;
-  rp.margin = margin;
   rp.counts = rw.counts;
   rp.chunk_base = rw.chunk_base;
   rp.seg_off = seg_off;
@@ -288,20 +273,34 @@ int do_route(const gqe_dims* d, const void* x, const void* Wr, const float* br, 
   rp.row_map = row_map;
   rp.B = d->B;
   rp.T = d->T;
-  rp.D = d->D;
   rp.G = d->G;
   rp.M = d->M;
   rp.k = d->k;
   rp.nch = (int)cdiv(d->T, kRouteChunk);
   const long long grid = (long long)d->B * rp.nch;
-  switch (d->G * d->M) {
-    case 2: GQE_TRY(launch_route_select<2>(rp, grid, st)); break;
-    case 4: GQE_TRY(launch_route_select<4>(rp, grid, st)); break;
-    case 8: GQE_TRY(launch_route_select<8>(rp, grid, st)); break;
-    case 16: GQE_TRY(launch_route_select<16>(rp, grid, st)); break;
-    case 32: GQE_TRY(launch_route_select<32>(rp, grid, st)); break;
-    case 64: GQE_TRY(launch_route_select<64>(rp, grid, st)); break;
-    default: return GQE_ERR_UNSUPPORTED;
+  {
+    // router logits on the tensor cores, routing decisions in the epilogue
+    GemmParams gp;
+    memset(&gp, 0, sizeof(gp));
+    const long long N = (long long)d->B * d->T;
+    const int GM = d->G * d->M;
+    GQE_TRY(tmap_rows(&gp.tmA, x, N, d->D, d->D, kGemmBM));
+    GQE_TRY(tmap_rows(&gp.tmB[0], Wr, d->D, GM, GM, 64));  // 64-wide box: columns past G*M read as zero
+    gp.nseg = 1;
+    gp.seg[0].n_cols = 64;
+    gp.K = d->D;
+    gp.G = d->G;
+    gp.M = d->M;
+    gp.k = d->k;
+    gp.r_br = br;
+    gp.r_sel = sel;
+    gp.r_w = w;
+    gp.r_margin = margin;
+    gp.r_counts = rw.counts;
+    gp.r_B = d->B;
+    gp.r_T = d->T;
+    gp.r_nch = rp.nch;
+    GQE_TRY((launch_gemm2<64, kRouteStages, kATma, kEpiRoute>(gp, grid, st)));
   }
   const int nseg = d->B * d->G * d->M;
   route_scan_kernel<<<1, 1024, nseg * 4, st>>>(rp);

@@ -53,7 +53,7 @@ def test_all_workloads_are_supported_and_sized():
 
 @pytest.mark.parametrize("bad,code", [
     (dict(dh=32), -2), (dict(D=1000), -2), (dict(k=3, M=2), -1), (dict(M=3, k=1), -2),
-    (dict(G=3, M=2), -2), (dict(T=0), -1), (dict(G=1, M=1), -2), (dict(k=0), -1),
+    (dict(G=3, M=2), -2), (dict(T=0), -1), (dict(G=1, M=1), -2), (dict(G=2, M=2), -2), (dict(k=0), -1),
 ])
 def test_unsupported_and_invalid_dims(bad, code):
     d = Dims(B=1, T=64, D=256, G=4, M=2, k=1).with_(**bad)
