@@ -134,6 +134,23 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(window), "scope": scope}
 
 
+def reduce_max(values, world: int, device) -> list:
+    """Element-wise max over ranks (timings: the slowest rank sets the job's
+    time). Works on any process group backend; identity for one rank."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job tokens/s: every rank processes its own batch (weak scaling)."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 def host_cores() -> int:
     try:
         return len(os.sched_getaffinity(0))
@@ -274,12 +291,9 @@ def main():
     attn_ms = sum(s[2] for s in stage_ms) / args.steps
     stage_avg = {n: sum(s[j] for s in stage_ms) / args.steps for j, n in
                  enumerate(("route", "qproj", "attention", "combine"))}
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_max([total_ms], world, dev)[0]
     ms_per_step = total_ms / args.steps
-    value = world * N / (ms_per_step / 1e3)
+    value = job_throughput(world, N, ms_per_step)
 
     # ---- dense GQA baseline of the same library (speedup denominator) -------
     ws_dense = gqe.workspace(d, gqe.OP_DENSE)
@@ -312,10 +326,7 @@ def main():
             e2e.append((e0, e1))
     torch.cuda.synchronize()
     e2e_ms = sum(a.elapsed_time(b) for a, b in e2e) / args.steps
-    if world > 1:
-        t = torch.tensor([e2e_ms, dense_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms, dense_ms = (float(v) for v in t.tolist())
+    e2e_ms, dense_ms = reduce_max([e2e_ms, dense_ms], world, dev)
     status = gqe.gqe_check_error()
     assert status == 0, gqe.gqe_status_string(status)
 
@@ -339,7 +350,7 @@ def main():
             "frac_bf16_peak": fl["gqe_total"] / (ms_per_step / 1e3) / 1e12 / peaks["bf16_tflops"],
             "dense_gqa_ms_per_step": dense_ms, "speedup_vs_dense": dense_ms / ms_per_step,
             "stage_ms": stage_avg, "roofline": roofline, "clocks": clocks,
-            "e2e": {"value": world * N / (e2e_ms / 1e3), "unit": "tokens/s",
+            "e2e": {"value": job_throughput(world, N, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": N * d.D * 2, "d2h_bytes_per_step": N * d.D * 2,
                     "entry": "gqe_forward_host"},
             "gpu_launches": launches_per_step * args.steps}
