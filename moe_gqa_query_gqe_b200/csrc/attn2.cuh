@@ -15,11 +15,12 @@
 // 128-row Q tiles (A, B) of one row set; items are visited heaviest first:
 //   warp 0      TMA producer: Q_A, Q_B once per item, K/V blocks of 128
 //               positions through a STAGES-deep ring
-//   warp 1      TMEM owner; lane 0 issues, per K/V block j,
+//   warps 1, 2  lane 0 issues the MMAs of tile A (warp 1, also the TMEM owner)
+//               or tile B (warp 2), per K/V block j:
 //                 S_t(j+1) = Q_t K_{j+1}^T  (SS MMA, M=128 N=128 K=64)
 //                 O_t     += P_t(j) V_j     (TS MMA: P read from TMEM, N=64)
-//               for t = A, B
-//   warps 2..3  idle (they only hand their registers to the softmax warps)
+//               so neither tile's pipeline waits on the other's barriers
+//   warp 3      idle (it only hands its registers to the softmax warps)
 //   warps 4..7  softmax of tile A, warps 8..11 softmax of tile B: one thread
 //               per row; S read from TMEM (then released at once so the next
 //               S can be computed under this block's softmax), lazily
@@ -203,11 +204,11 @@ __global__ void __launch_bounds__(kA2Threads, 1) attn2_fwd_kernel(const __grid_c
 
   if (tid == 0) {
     mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
+    mbar_init(q_empty, 2);  // one commit from each tile's MMA thread
     for (int s = 0; s < kA2Stages; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&kv_empty[s], 2);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
@@ -254,30 +255,29 @@ __global__ void __launch_bounds__(kA2Threads, 1) attn2_fwd_kernel(const __grid_c
         }
         ++n_items;
       }
-    } else if (warp == 1 && lane == 0) {
-      // ---- MMA issue -------------------------------------------------------------
+    } else if ((warp == 1 || warp == 2) && lane == 0) {
+      // ---- MMA issue: warp 1 drives tile A, warp 2 tile B --------------------------
+      const int t = warp - 1;
       constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false);  // Q, K both K-major
       constexpr uint32_t idesc_o = idesc_bf16(128, 64, false, true);    // P from TMEM, V MN-major
       uint32_t kv = 0, n_items = 0;
-      uint32_t s_cnt0 = 0, s_cnt1 = 0, pv_cnt0 = 0, pv_cnt1 = 0;  // issued so far, per tile
+      uint32_t s_cnt = 0, pv_cnt = 0;  // issued so far by this thread
       bool ok = true;
-      auto issue_s = [&](int t, uint32_t kvi) -> bool {
-        uint32_t& sc = t ? s_cnt1 : s_cnt0;
-        if (sc > 0 && !mbar_wait(&s_free[t], (sc - 1) & 1, abort_flag)) return false;
+      const uint32_t qa = sbase + L::kQ + t * 16384;
+      auto issue_s = [&](uint32_t kvi) -> bool {
+        if (s_cnt > 0 && !mbar_wait(&s_free[t], (s_cnt - 1) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t qa = sbase + L::kQ + t * 16384;
         const uint32_t ka = sbase + L::kK + (kvi % kA2Stages) * 16384;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           umma_ss(tmem_base + t * 128, sdesc_sw128(qa + kk * 32, 16, 1024), sdesc_sw128(ka + kk * 32, 16, 1024),
                   idesc_s, kk != 0);
         umma_commit(&s_full[t]);
-        ++sc;
+        ++s_cnt;
         return true;
       };
-      auto issue_pv = [&](int t, uint32_t kvi, bool acc) -> bool {
-        uint32_t& pc = t ? pv_cnt1 : pv_cnt0;
-        if (!mbar_wait(&p_full[t], pc & 1, abort_flag)) return false;
+      auto issue_pv = [&](uint32_t kvi, bool acc) -> bool {
+        if (!mbar_wait(&p_full[t], pv_cnt & 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t va = sbase + L::kV + (kvi % kA2Stages) * 16384;
 #pragma unroll
@@ -285,28 +285,30 @@ __global__ void __launch_bounds__(kA2Threads, 1) attn2_fwd_kernel(const __grid_c
           umma_ts(tmem_base + 256 + t * 64, tmem_base + 384 + t * 64 + kk * 8, sdesc_sw128(va + kk * 2048, 8192, 1024),
                   idesc_o, (acc || kk != 0) ? 1u : 0u);
         umma_commit(&pv_done[t]);
-        ++pc;
+        ++pv_cnt;
         return true;
       };
       for (int round = 0, item = a2_item_of(0); ok && item < p.total_items; item = a2_item_of(++round)) {
         const A2Item it = a2_decode(p, item);
         if (!it.valid) continue;
+        const int n = t == 0 ? it.nA : it.nB;
         if (!(ok = mbar_wait(q_full, n_items & 1, abort_flag))) break;
         const uint32_t kv0 = kv;
-        if (!(ok = mbar_wait(&k_full[kv0 % kA2Stages], (kv0 / kA2Stages) & 1, abort_flag))) break;
-        tc_fence_after();
-        ok = issue_s(0, kv0) && (it.nB == 0 || issue_s(1, kv0));
+        if (n > 0) {
+          if (!(ok = mbar_wait(&k_full[kv0 % kA2Stages], (kv0 / kA2Stages) & 1, abort_flag))) break;
+          if (!(ok = issue_s(kv0))) break;
+        }
         for (int j = 0; ok && j < it.nmax; ++j) {
           const uint32_t kvj = kv0 + j;
-          if (j + 1 < it.nmax) {
+          if (j + 1 < n) {
             if (!(ok = mbar_wait(&k_full[(kvj + 1) % kA2Stages], ((kvj + 1) / kA2Stages) & 1, abort_flag))) break;
-            if (j + 1 < it.nA && !(ok = issue_s(0, kvj + 1))) break;
-            if (j + 1 < it.nB && !(ok = issue_s(1, kvj + 1))) break;
+            if (!(ok = issue_s(kvj + 1))) break;
           }
-          if (!(ok = mbar_wait(&v_full[kvj % kA2Stages], (kvj / kA2Stages) & 1, abort_flag))) break;
-          if (j < it.nA && !(ok = issue_pv(0, kvj, j > 0))) break;
-          if (j < it.nB && !(ok = issue_pv(1, kvj, j > 0))) break;
-          umma_commit(&kv_empty[kvj % kA2Stages]);
+          if (j < n) {
+            if (!(ok = mbar_wait(&v_full[kvj % kA2Stages], (kvj / kA2Stages) & 1, abort_flag))) break;
+            if (!(ok = issue_pv(kvj, j > 0))) break;
+          }
+          umma_commit(&kv_empty[kvj % kA2Stages]);  // this thread is done with block j
         }
         umma_commit(q_empty);
         kv += it.nmax;
