@@ -334,7 +334,7 @@ def main():
     peaks = load_peaks()
     attn_flops = fl["gqe"]["attention"]
     attn_tflops = attn_flops / (attn_ms / 1e3) / 1e12
-    roofline = {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": attn_tflops,
+    roofline = {"bound": "tensor", "kernel": "attn2_fwd_kernel", "achieved": attn_tflops,
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16_tflops"],
                 "peak_source": f"{peaks['source']} bf16 burst",
                 "traffic": recorded_traffic(args.workload, "attn.cuh"),

@@ -28,12 +28,11 @@
 //               TMEM as bf16 pairs, final O / l stored as bf16.
 // TMEM columns: S_A [0,128) S_B [128,256) O_A [256,320) O_B [320,384)
 //               P_A [384,448) P_B [448,512).
-// Exponentials run on the MUFU ex2 unit. An FMA-pipe alternative for every
-// kA2PolyEvery-th column pair is kept (2^x = 2^j * p(x - j), j = round(x), p a
-// degree-3 minimax polynomial on [-1/2, 1/2], relative error 7.5e-5,
-// coefficients fitted by fit_exp2_poly.py in this directory); it is off
-// (kA2PolyEvery = 0) because every share tried measured slower here: the
-// softmax warps are latency-bound on the MMA round trips, not MUFU-bound.
+// Exponentials: MUFU ex2 delivers 16/clk/SM while each score needs 1/32 clk
+// of tensor time, so one column pair in kA2PolyEvery (= 8, the best share
+// measured) is evaluated on the FMA pipe instead: 2^x = 2^j * p(x - j),
+// j = round(x), p a degree-3 minimax polynomial on [-1/2, 1/2] (relative
+// error 7.5e-5; coefficients fitted by fit_exp2_poly.py in this directory).
 #pragma once
 
 #include "attn.cuh"
@@ -48,7 +47,7 @@ constexpr int kA2Threads = 384;
 // registers the block is launched with.
 constexpr int kA2RegsLow = 88;
 constexpr int kA2RegsHigh = 208;
-constexpr int kA2PolyEvery = 0;  // every n-th column pair uses the FMA-pipe exp2 (0: none)
+constexpr int kA2PolyEvery = 8;  // every n-th column pair uses the FMA-pipe exp2 (0: none)
 
 struct Attn2Params {
   CUtensorMap tmQ[2];  // [B*T, Ha, 64] boxes (64, rr, 128/rr)
