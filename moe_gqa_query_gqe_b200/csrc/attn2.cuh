@@ -13,8 +13,9 @@
 //
 // Per CTA (persistent, one per SM, 384 threads), work item = two adjacent
 // 128-row Q tiles (A, B) of one row set; items are visited heaviest first:
-//   warp 0      TMA producer: Q_A, Q_B once per item, K/V blocks of 128
-//               positions through a STAGES-deep ring
+//   warp 0      TMA producer: Q_A, Q_B once per item (two item buffers, so
+//               the next item's Q arrives while this one runs), K/V blocks of
+//               128 positions through a STAGES-deep ring
 //   warps 1, 2  lane 0 issues the MMAs of tile A (warp 1, also the TMEM owner)
 //               or tile B (warp 2), per K/V block j:
 //                 S_t(j+1) = Q_t K_{j+1}^T  (SS MMA, M=128 N=128 K=64)
@@ -60,8 +61,8 @@ struct Attn2Params {
 };
 
 struct A2Smem {
-  static constexpr int kQ = 0;  // Q_A, Q_B: 16 KB each
-  static constexpr int kK = 32768;
+  static constexpr int kQ = 0;  // two item buffers of [Q_A, Q_B], 16 KB each
+  static constexpr int kK = 65536;
   static constexpr int kV = kK + kA2Stages * 16384;
   static constexpr int kBar = kV + kA2Stages * 16384;
   static constexpr int kBytes = kBar + 512 + 1024;
@@ -187,9 +188,9 @@ __global__ void __launch_bounds__(kA2Threads, 1) attn2_fwd_kernel(const __grid_c
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  uint64_t* q_full = bars + 0;
-  uint64_t* q_empty = bars + 1;
-  uint64_t* k_full = bars + 2;                   // [STAGES]
+  uint64_t* q_full = bars + 0;                   // [2] item buffers
+  uint64_t* q_empty = bars + 2;                  // [2]
+  uint64_t* k_full = bars + 4;                   // [STAGES]
   uint64_t* v_full = k_full + kA2Stages;         // [STAGES]
   uint64_t* kv_empty = v_full + kA2Stages;       // [STAGES]
   uint64_t* s_full = kv_empty + kA2Stages;       // [2] (tile A, B)
@@ -202,8 +203,10 @@ __global__ void __launch_bounds__(kA2Threads, 1) attn2_fwd_kernel(const __grid_c
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 2);  // one commit from each tile's MMA thread
+    for (int qb = 0; qb < 2; ++qb) {
+      mbar_init(&q_full[qb], 1);
+      mbar_init(&q_empty[qb], 2);  // one commit from each tile's MMA thread
+    }
     for (int s = 0; s < kA2Stages; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
@@ -240,10 +243,12 @@ __global__ void __launch_bounds__(kA2Threads, 1) attn2_fwd_kernel(const __grid_c
         const A2Item it = a2_decode(p, item);
         if (!it.valid) continue;
         const int row0 = it.b * p.T;
-        if (!(ok = mbar_wait(q_empty, (n_items & 1) ^ 1, abort_flag))) break;
-        mbar_arrive_expect_tx(q_full, it.nB > 0 ? 32768 : 16384);
-        tma_load_3d(smem + L::kQ, &p.tmQ[it.rs.tm], q_full, 0, it.rs.h0, row0 + it.t0);
-        if (it.nB > 0) tma_load_3d(smem + L::kQ + 16384, &p.tmQ[it.rs.tm], q_full, 0, it.rs.h0, row0 + it.t0 + it.tpt);
+        const int qb = n_items & 1;
+        if (!(ok = mbar_wait(&q_empty[qb], ((n_items >> 1) & 1) ^ 1, abort_flag))) break;
+        uint8_t* qs = smem + L::kQ + qb * 32768;
+        mbar_arrive_expect_tx(&q_full[qb], it.nB > 0 ? 32768 : 16384);
+        tma_load_3d(qs, &p.tmQ[it.rs.tm], &q_full[qb], 0, it.rs.h0, row0 + it.t0);
+        if (it.nB > 0) tma_load_3d(qs + 16384, &p.tmQ[it.rs.tm], &q_full[qb], 0, it.rs.h0, row0 + it.t0 + it.tpt);
         for (int j = 0; j < it.nmax; ++j, ++kv) {
           const int s = kv % kA2Stages;
           if (!(ok = mbar_wait(&kv_empty[s], ((kv / kA2Stages) & 1) ^ 1, abort_flag))) break;
@@ -262,7 +267,7 @@ __global__ void __launch_bounds__(kA2Threads, 1) attn2_fwd_kernel(const __grid_c
       uint32_t kv = 0, n_items = 0;
       uint32_t s_cnt = 0, pv_cnt = 0;  // issued so far by this thread
       bool ok = true;
-      const uint32_t qa = sbase + L::kQ + t * 16384;
+      uint32_t qa = sbase + L::kQ + t * 16384;
       auto issue_s = [&](uint32_t kvi) -> bool {
         if (s_cnt > 0 && !mbar_wait(&s_free[t], (s_cnt - 1) & 1, abort_flag)) return false;
         tc_fence_after();
@@ -291,7 +296,9 @@ __global__ void __launch_bounds__(kA2Threads, 1) attn2_fwd_kernel(const __grid_c
         const A2Item it = a2_decode(p, item);
         if (!it.valid) continue;
         const int n = t == 0 ? it.nA : it.nB;
-        if (!(ok = mbar_wait(q_full, n_items & 1, abort_flag))) break;
+        const int qb = n_items & 1;
+        if (!(ok = mbar_wait(&q_full[qb], (n_items >> 1) & 1, abort_flag))) break;
+        qa = sbase + L::kQ + qb * 32768 + t * 16384;
         const uint32_t kv0 = kv;
         if (n > 0) {
           if (!(ok = mbar_wait(&k_full[kv0 % kA2Stages], (kv0 / kA2Stages) & 1, abort_flag))) break;
@@ -309,7 +316,7 @@ __global__ void __launch_bounds__(kA2Threads, 1) attn2_fwd_kernel(const __grid_c
           }
           umma_commit(&kv_empty[kvj % kA2Stages]);  // this thread is done with block j
         }
-        umma_commit(q_empty);
+        umma_commit(&q_empty[qb]);
         kv += it.nmax;
         ++n_items;
       }
