@@ -186,7 +186,10 @@ int gqe_attn(const gqe_dims* d, const void* Q, const void* K, const void* V,
  *   A[n] = [O[n,0..G*k-1] (concat) | sum_j w[n,g,j] O[n,g*k+j] for g (slot)
  *           | O[n,G*k] (shared)]           width (G*k + G + 1)*dh
  *   y    = A Wo,   Wo [(G*k+G+1)*dh, D] bf16, y [B*T, D] bf16.
- * ws: gqe_workspace_bytes(d, GQE_OP_COMBINE).
+ * For k == 1 every renormalised weight is exactly 1, so the slot of group g
+ * is O[n, g] and the projection reads all of A straight from O (no
+ * workspace). For k > 1 A is assembled in the workspace first.
+ * ws: gqe_workspace_bytes(d, GQE_OP_COMBINE) (0 when k == 1).
  */
 int gqe_combine(const gqe_dims* d, const void* O, const float* w,
                 const void* Wo, void* y, void* ws, size_t ws_bytes,

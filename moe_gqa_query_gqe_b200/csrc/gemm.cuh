@@ -46,6 +46,9 @@ struct GemmParams {
   float* r_margin;     // [B*T, G] or null
   int32_t* r_counts;   // [B][nch][G*M]
   int r_B, r_T, r_nch;
+  // A column remap for the k = 1 combine: A = [O_routed | O_routed | O_shared]
+  // read straight from O ([N, (G+1)*64]); 0 disables the remap
+  int amap_G;
 };
 
 enum GemmEpilogue : int { kEpiStore = 0, kEpiRoute = 1 };

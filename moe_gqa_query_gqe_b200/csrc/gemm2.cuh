@@ -199,7 +199,17 @@ __global__ void __launch_bounds__(G2Cfg<BN, STAGES, AMODE>::kThreads, 1)
         uint8_t* b_s = a_s + C::kABytes;
         if (lane == 0) {
           mbar_arrive_expect_tx(&full[s], (AMODE == kAGatherLsu ? 0 : C::kABytes) + nbox * 8192);
-          if constexpr (AMODE == kATma) tma_load_2d(a_s, &p.tmA, &full[s], kb * kGemmBK, t.m0);
+          if constexpr (AMODE == kATma) {
+            int a_col = kb * kGemmBK;
+            if (p.amap_G > 0) {
+              // k-block kb of A = [concat (G) | slot (G) | shared]: for k = 1 each
+              // slot equals its group's output (weight exactly 1), so both
+              // halves read O's routed columns and the last block its shared one
+              const int blk = kb < 2 * p.amap_G ? kb % p.amap_G : p.amap_G;
+              a_col = blk * kGemmBK;
+            }
+            tma_load_2d(a_s, &p.tmA, &full[s], a_col, t.m0);
+          }
           for (int nb = 0; nb < nbox; ++nb)
             tma_load_2d(b_s + nb * 8192, tmb, &full[s], b_col + nb * 64, kb * kGemmBK);
         }

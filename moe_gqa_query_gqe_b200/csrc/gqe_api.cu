@@ -216,11 +216,12 @@ FwdWs carve_forward(Carver& c, const gqe_dims* d) {
   f.K = c.take<__nv_bfloat16>(N * d->G * 64);
   f.V = c.take<__nv_bfloat16>(N * d->G * 64);
   f.O = c.take<__nv_bfloat16>(N * Ha * 64);
-  f.A = c.take<__nv_bfloat16>(N * (size_t)(d->G * d->k + d->G + 1) * 64);
+  f.A = c.take<__nv_bfloat16>(d->k == 1 ? 0 : N * (size_t)(d->G * d->k + d->G + 1) * 64);
   return f;
 }
 
 size_t combine_ws_bytes(const gqe_dims* d) {
+  if (d->k == 1) return 0;  // A is read straight from O (see do_combine)
   return align256((size_t)d->B * d->T * (d->G * d->k + d->G + 1) * 64 * 2);
 }
 
@@ -382,6 +383,22 @@ int do_combine(const gqe_dims* d, const void* O, const float* w, const void* Wo,
                cudaStream_t st) {
   const long long N = (long long)d->B * d->T;
   const int KA = (d->G * d->k + d->G + 1) * 64;
+  if (d->k == 1) {
+    // renormalised weights over one selected expert are exactly 1: the slot of
+    // group g is O[:, g] itself, so the projection reads A's blocks from O
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    const int Ha = d->G + 1;
+    GQE_TRY(tmap_rows(&p.tmA, O, N, Ha * 64, Ha * 64, kGemmBM));
+    GQE_TRY(tmap_rows(&p.tmB[0], Wo, KA, d->D, d->D, 64));
+    p.seg[0] = GemmSeg{d->D, 0, 0, 0, (long long)d->D, static_cast<__nv_bfloat16*>(y)};
+    p.nseg = 1;
+    p.ntn = (int)cdiv(d->D, kG2DenseBN);
+    p.rows = (int)N;
+    p.K = KA;
+    p.amap_G = d->G;
+    return launch_gemm2<kG2DenseBN, kG2DenseStages, kATma>(p, cdiv(N, kGemmBM) * p.ntn, st);
+  }
   CombineParams cp{static_cast<const __nv_bfloat16*>(O), w, A, N, d->G, d->k};
   const long long warps = N;
   const long long blocks = std::min<long long>(cdiv(warps * 32, 256), 148ll * 16);

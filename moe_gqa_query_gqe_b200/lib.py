@@ -193,7 +193,7 @@ def forward_views(dims, ws: torch.Tensor) -> dict:
             ("_counts", torch.int32, (d.B * nch * d.G * d.M,)), ("_chunk_base", torch.int32, (d.B * nch * d.G * d.M,)),
             ("Q", torch.bfloat16, (N, Ha, 64)), ("K", torch.bfloat16, (N, d.G, 64)),
             ("V", torch.bfloat16, (N, d.G, 64)), ("O", torch.bfloat16, (N, Ha, 64)),
-            ("A", torch.bfloat16, (N, (d.G * d.k + d.G + 1) * 64))]
+            ("A", torch.bfloat16, (N if d.k > 1 else 0, (d.G * d.k + d.G + 1) * 64))]
     out, off = {}, 0
     for name, dt, shape in spec:
         n = 1
