@@ -14,6 +14,7 @@
 #include "route.cuh"
 #include "gemm.cuh"
 #include "gemm2.cuh"
+#include "qgather.cuh"
 #include "attn.cuh"
 #include "attn2.cuh"
 #include "combine.cuh"
@@ -340,6 +341,14 @@ int do_qproj(const gqe_dims* d, const void* x, const void* Wq, const void* Wk, c
   p.Ha = Ha;
   p.ntok = (int)N;
   const long long tiles_max = cdiv(N * G * k, kGemmBM) + p.nsegs_q;
+  const int qg_smem = QgSmem::kBytesBase + (p.nsegs_q + 1) * 4;
+  if (d->D <= kQgMaxK && qg_smem <= 227 * 1024) {
+    // the head's weight slice stays resident in shared memory
+    GQE_TRY(set_smem(qgather_kernel, qg_smem));
+    const int grid = (int)std::min<long long>(tiles_max, sm_count());
+    qgather_kernel<<<grid, kQgThreads, qg_smem, st>>>(p);
+    return launch_status();
+  }
   return launch_gemm2<64, kG2GatherStages, kG2GatherMode>(p, tiles_max, st);
 }
 
