@@ -88,7 +88,8 @@ __device__ __forceinline__ G2Tile g2_decode(const GemmParams& p, int tile, const
   return t;
 }
 
-template <int BN, int STAGES, int AMODE, int EPI = kEpiStore>
+// RM: experts per group, compile-time in the routing epilogue (1, 2, 4 or 8)
+template <int BN, int STAGES, int AMODE, int EPI = kEpiStore, int RM = 1>
 __global__ void __launch_bounds__(G2Cfg<BN, STAGES, AMODE>::kThreads, 1)
     gemm2_kernel(const __grid_constant__ GemmParams p, int total_tiles) {
   using C = G2Cfg<BN, STAGES, AMODE>;
@@ -333,51 +334,58 @@ __global__ void __launch_bounds__(G2Cfg<BN, STAGES, AMODE>::kThreads, 1)
       const int tt = c * kGemmBM + row;
       if (tt < p.r_T) {
         const size_t n = (size_t)b * p.r_T + tt;
-        for (int g = 0; g < p.G; ++g) {
-          float l[8];
-          for (int e = 0; e < p.M; ++e) {
-            float v = 0.f;
+        // groups unrolled with static indices into lg (G*M <= 64)
 #pragma unroll
-            for (int i = 0; i < 64; ++i)
-              if (i == g * p.M + e) v = lg[i];
-            l[e] = p.r_br ? v + p.r_br[g * p.M + e] : v;
-          }
+        for (int g = 0; g < 64 / RM; ++g) {
+          if (g >= p.G) break;
+          float l[RM];
+#pragma unroll
+          for (int e = 0; e < RM; ++e) l[e] = p.r_br ? lg[g * RM + e] + p.r_br[g * RM + e] : lg[g * RM + e];
+          // top-k by logit, exact ties -> lower expert index
           uint32_t chosen = 0;
           float kth = 0.f;
           for (int j = 0; j < p.k; ++j) {
             int best = -1;
             float bv = 0.f;
-            for (int e = 0; e < p.M; ++e) {
-              if (chosen & (1u << e)) continue;
-              if (best < 0 || l[e] > bv) { best = e; bv = l[e]; }
+#pragma unroll
+            for (int e = 0; e < RM; ++e) {
+              const bool free_e = !(chosen & (1u << e));
+              if (free_e && (best < 0 || l[e] > bv)) { best = e; bv = l[e]; }
             }
             chosen |= 1u << best;
             kth = bv;
           }
           float mg = __int_as_float(0x7f800000);  // +inf when k == M
-          if (p.k < p.M) {
+          if (p.k < RM) {
             int best = -1;
             float bv = 0.f;
-            for (int e = 0; e < p.M; ++e) {
-              if (chosen & (1u << e)) continue;
-              if (best < 0 || l[e] > bv) { best = e; bv = l[e]; }
+#pragma unroll
+            for (int e = 0; e < RM; ++e) {
+              const bool free_e = !(chosen & (1u << e));
+              if (free_e && (best < 0 || l[e] > bv)) { best = e; bv = l[e]; }
             }
             mg = kth - bv;
           }
           float mx = -INFINITY;
-          for (int e = 0; e < p.M; ++e)
+#pragma unroll
+          for (int e = 0; e < RM; ++e)
             if (chosen & (1u << e)) mx = fmaxf(mx, l[e]);
+          float ex[RM];
           float den = 0.f;
-          for (int e = 0; e < p.M; ++e)
-            if (chosen & (1u << e)) den += expf(l[e] - mx);
+#pragma unroll
+          for (int e = 0; e < RM; ++e) {
+            ex[e] = (chosen & (1u << e)) ? expf(l[e] - mx) : 0.f;
+            den += ex[e];
+          }
           const float inv = 1.f / den;
           int j = 0;
-          for (int e = 0; e < p.M; ++e) {
+#pragma unroll
+          for (int e = 0; e < RM; ++e) {
             if (!(chosen & (1u << e))) continue;
             const size_t o = (n * p.G + g) * p.k + j;
             p.r_sel[o] = e;
-            p.r_w[o] = expf(l[e] - mx) * inv;
-            atomicAdd(&s_cnt[g * p.M + e], 1);
+            p.r_w[o] = ex[e] * inv;
+            atomicAdd(&s_cnt[g * RM + e], 1);
             ++j;
           }
           if (p.r_margin) p.r_margin[n * p.G + g] = mg;

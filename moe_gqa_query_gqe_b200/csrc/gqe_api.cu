@@ -123,10 +123,10 @@ constexpr int kG2GatherMode = kAGatherLsu;
 
 int sm_count();
 
-template <int BN, int STAGES, int AMODE, int EPI = kEpiStore>
+template <int BN, int STAGES, int AMODE, int EPI = kEpiStore, int RM = 1>
 int launch_gemm2(const GemmParams& p, long long tiles, cudaStream_t st) {
   using C = G2Cfg<BN, STAGES, AMODE>;
-  auto kern = gemm2_kernel<BN, STAGES, AMODE, EPI>;
+  auto kern = gemm2_kernel<BN, STAGES, AMODE, EPI, RM>;
   const int smem = C::kBytesBase + (AMODE != kATma ? (p.nsegs_q + 1) * 4 : 0) + (EPI == kEpiRoute ? 64 * 4 : 0);
   if (int e = set_smem(kern, smem)) return e;
   if (tiles <= 0) return GQE_OK;
@@ -302,7 +302,13 @@ int do_route(const gqe_dims* d, const void* x, const void* Wr, const float* br, 
     gp.r_B = d->B;
     gp.r_T = d->T;
     gp.r_nch = rp.nch;
-    GQE_TRY((launch_gemm2<64, kRouteStages, kATma, kEpiRoute>(gp, grid, st)));
+    switch (d->M) {
+      case 1: GQE_TRY((launch_gemm2<64, kRouteStages, kATma, kEpiRoute, 1>(gp, grid, st))); break;
+      case 2: GQE_TRY((launch_gemm2<64, kRouteStages, kATma, kEpiRoute, 2>(gp, grid, st))); break;
+      case 4: GQE_TRY((launch_gemm2<64, kRouteStages, kATma, kEpiRoute, 4>(gp, grid, st))); break;
+      case 8: GQE_TRY((launch_gemm2<64, kRouteStages, kATma, kEpiRoute, 8>(gp, grid, st))); break;
+      default: return GQE_ERR_UNSUPPORTED;
+    }
   }
   const int nseg = d->B * d->G * d->M;
   route_scan_kernel<<<1, 1024, nseg * 4, st>>>(rp);
