@@ -68,15 +68,20 @@ def kernel_source_hash(name: str) -> str:
 
 
 def recorded_traffic(workload: str, src: str) -> float | None:
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source."""
-    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    """DRAM bytes per launch of the kernel in csrc/<src>, from the committed
+    ncu summary profiles/traffic_<kernel source>_<workload>.md, but only if
+    that capture was taken on the current kernel source (its
+    `source_sha256_16:` line matches)."""
+    path = os.path.join(ROOT, "profiles", f"traffic_{src.split('.')[0]}_{workload}.md")
     try:
+        fields = {}
         with open(path) as fh:
-            rec = json.load(fh)
-        r = rec.get(workload, {}).get(src)
-        if r and r.get("source_hash") == kernel_source_hash(src):
-            return float(r["bytes_per_launch"])
+            for line in fh:
+                if ":" in line and not line.startswith("#"):
+                    key, val = line.split(":", 1)
+                    fields[key.strip("-* `")] = val.strip().strip("`")
+        if fields.get("source_sha256_16") == kernel_source_hash(src):
+            return float(fields["bytes_per_launch"])
     except Exception:
         pass
     return None
@@ -337,7 +342,7 @@ def main():
     roofline = {"bound": "tensor", "kernel": "attn2_fwd_kernel", "achieved": attn_tflops,
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16_tflops"],
                 "peak_source": f"{peaks['source']} bf16 burst",
-                "traffic": recorded_traffic(args.workload, "attn.cuh"),
+                "traffic": recorded_traffic(args.workload, "attn2.cuh"),
                 "algorithmic_flops_per_launch": attn_flops}
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
