@@ -28,6 +28,10 @@ SMALL = {
     "one_group_g1_m8_k2": Dims(B=2, T=200, D=192, G=1, M=8, k=2),
     "k_equals_m_t260": Dims(B=1, T=260, D=128, G=4, M=2, k=2),
     "pool8_k4_t136": Dims(B=2, T=136, D=256, G=8, M=8, k=4),
+    # +20 router bias on expert 0: every token picks it, the other experts'
+    # segments are empty
+    "empty_segments_bias20": Dims(B=2, T=160, D=256, G=4, M=4, k=1, bias0=20.0),
+    "one_token_b1_t1": Dims(B=1, T=1, D=128, G=4, M=2, k=1),
 }
 
 
@@ -107,6 +111,12 @@ def test_dense_gqa_baseline(cases, name):
     assert status == 0
     want = ref.gqa_dense_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wo_dense"], d)
     assert_close_bf16(y, want["y"], "dense GQA y vs oracle")
+
+
+def test_empty_segments_are_empty(cases):
+    d, inp, dev, st = cases["empty_segments_bias20"]
+    lens = np.diff(st["seg_off"].numpy()).reshape(d.B, d.G, d.M)
+    assert np.all(lens[:, :, 0] == d.T) and np.all(lens[:, :, 1:] == 0)
 
 
 def test_causality_bitwise_on_gpu(cases):
