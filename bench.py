@@ -254,66 +254,102 @@ def main():
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(ev=None):
-        if ev: ev[0].record(stream)
+    def stage_step(ev):
+        # the forward pass as four C-ABI calls, events between them (per-stage times)
+        ev[0].record(stream)
         gqe.gqe_route(d, inp["x"], inp["Wr"], inp["br"], sel, wts, margin, seg_off, seg_tok, row_map, ws_route)
-        if ev: ev[1].record(stream)
+        ev[1].record(stream)
         gqe.gqe_qproj(d, inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], sel, seg_off, seg_tok, Q, K, V)
-        if ev: ev[2].record(stream)
+        ev[2].record(stream)
         gqe.gqe_attn(d, Q, K, V, O)
-        if ev: ev[3].record(stream)
+        ev[3].record(stream)
         gqe.gqe_combine(d, O, wts, inp["Wo"], y, ws_comb)
-        if ev: ev[4].record(stream)
+        ev[4].record(stream)
 
-    launches_per_step = 3 + 2 + 1 + 2  # route 3, qproj 2, attention 1, combine 2
+    ws_fwd = gqe.workspace(d, gqe.OP_FORWARD)
+    ws_dense = gqe.workspace(d, gqe.OP_DENSE)
+    y_dense = torch.empty_like(y)
+
+    def gqe_step():
+        gqe.gqe_forward(d, inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"], inp["Wo"], y, ws_fwd)
+
+    def dense_step():
+        gqe.gqa_dense_forward(d, inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wo_dense"], y_dense, ws_dense)
+
+    def as_graph(fn):
+        # one step captured as a CUDA graph: the same kernels, no host enqueue
+        # inside the timed region
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            fn()
+        torch.cuda.synchronize()
+        return g
+
+    # kernels launched per forward step (k = 1: route 3, qproj 2, attention 1, Wo 1)
+    launches_per_step = 3 + 2 + 1 + (1 if d.k == 1 else 2)
 
     def barrier():
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
 
+    def timed(fn, n):
+        """n calls, L2 flushed before each outside the events; per-call ms."""
+        evs = []
+        for _ in range(n):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            evs.append((a, b))
+        return evs
+
+    g_gqe = as_graph(gqe_step)
+    g_dense = as_graph(dense_step)
+
     # ---- warm-up, then K timed steps (L2 flushed between steps) -----------
     sampler = ClockSampler(local_rank)
     sampler.wait_first()
-    for _ in range(args.warmup):
-        flush.fill_(1)
-        step()
+    timed(g_gqe.replay, args.warmup)
     assert gqe.gqe_check_error() == 0
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     barrier()
     t_begin = time.time()
-    for i in range(args.steps):
-        flush.fill_(1)
-        step(evs[i])
+    evs = timed(g_gqe.replay, args.steps)
     barrier()
     t_end = time.time()
     clocks = sampler.stop(t_begin, t_end)
     status = gqe.gqe_check_error()
     assert status == 0, gqe.gqe_status_string(status)
-    stage_ms = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)]
-    step_ms = [sum(s) for s in stage_ms]
-    total_ms = sum(step_ms)
-    attn_ms = sum(s[2] for s in stage_ms) / args.steps
-    stage_avg = {n: sum(s[j] for s in stage_ms) / args.steps for j, n in
-                 enumerate(("route", "qproj", "attention", "combine"))}
+    total_ms = sum(a.elapsed_time(b) for a, b in evs)
     total_ms = reduce_max([total_ms], world, dev)[0]
     ms_per_step = total_ms / args.steps
     value = job_throughput(world, N, ms_per_step)
 
-    # ---- dense GQA baseline of the same library (speedup denominator) -------
-    ws_dense = gqe.workspace(d, gqe.OP_DENSE)
-    y_dense = torch.empty_like(y)
-    dense_ms = []
+    # ---- per-stage times (the same kernels through the four stage calls) -----
+    sevs = []
     for i in range(args.warmup + args.steps):
         flush.fill_(1)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        gqe.gqa_dense_forward(d, inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wo_dense"], y_dense, ws_dense)
-        e1.record(stream)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        stage_step(ev)
         if i >= args.warmup:
-            dense_ms.append((e0, e1))
+            sevs.append(ev)
     torch.cuda.synchronize()
-    dense_ms = sum(a.elapsed_time(b) for a, b in dense_ms) / args.steps
+    stage_ms = [[ev[j].elapsed_time(ev[j + 1]) for j in range(4)] for ev in sevs]
+    attn_ms = sum(s[2] for s in stage_ms) / len(stage_ms)
+    stage_avg = {n: sum(s[j] for s in stage_ms) / len(stage_ms) for j, n in
+                 enumerate(("route", "qproj", "attention", "combine"))}
+
+    # ---- dense GQA baseline of the same library (speedup denominator) -------
+    timed(g_dense.replay, args.warmup)
+    devs = timed(g_dense.replay, args.steps)
+    torch.cuda.synchronize()
+    dense_ms = sum(a.elapsed_time(b) for a, b in devs) / args.steps
 
     # ---- end to end through the host-buffer entry point ---------------------
     x_host = inp["x"].cpu().pin_memory()
@@ -358,7 +394,8 @@ def main():
             "e2e": {"value": job_throughput(world, N, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": N * d.D * 2, "d2h_bytes_per_step": N * d.D * 2,
                     "entry": "gqe_forward_host"},
-            "gpu_launches": launches_per_step * args.steps}
+            "gpu_launches": launches_per_step * args.steps,
+            "timing": "each step one CUDA-graph replay of gqe_forward; stage_ms from the four stage calls"}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tokens, times = oracle_sample(d, args.cpu_budget)

@@ -1,5 +1,8 @@
-// gemm2.cuh -- persistent tcgen05 GEMM for the GQE projections:
-// C = A * B, bf16 in, fp32 accumulate in TMEM, bf16 out.
+// gemm2.cuh -- persistent single-CTA tcgen05 GEMM: C = A * B, bf16 in, fp32
+// accumulate in TMEM. Used for the router logits (with the routing epilogue)
+// and for the selected-expert query projection when the head's weight slice
+// is too large to stay resident (D > 1024); the dense projections run on CTA
+// pairs (gemm2sm.cuh).
 //
 //   A [rows, K] row-major (K-major operand): TMA tiles (dense rows), or rows
 //     gathered by a segment's token list with TMA tile::gather4 (the

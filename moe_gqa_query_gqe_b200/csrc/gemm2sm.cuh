@@ -1,0 +1,233 @@
+// gemm2sm.cuh -- dense projection GEMM on CTA pairs (tcgen05 .cta_group::2):
+// C = A * B, bf16 in, fp32 accumulate in TMEM, bf16 out. Used for the K/V (and
+// shared-head Q) projection, the output projection Wo and the dense GQA
+// baseline's projections.
+//
+//   A [rows, K] row-major (K-major operand), B [K, N] row-major weight
+//   (MN-major operand), both by TMA with 128-byte swizzle; up to three output
+//   segments (weights) per launch, as in gemm2.cuh.
+//
+// Why pairs: a 128 x 256 tile on one SM needs 48 KB of operands per 64-deep
+// k-block for 512 tensor-core cycles, more than one SM pulls from L2. A pair
+// of SMs computes a 256 x 256 tile: each SM loads its 128 rows of A and half
+// (128 columns) of B, 32 KB per k-block for the same 512 cycles, and the MMA
+// issued by the even CTA reads both CTAs' shared memory.
+//
+// Per pair tile (256 rows x up to 256 columns; narrow segment tails are
+// rounded up to 128 columns so both halves of B are whole 64-column boxes):
+//   warp 0 (both CTAs)   TMA producer: A rows [m0 + 128*rank, +128) and B
+//                        columns [n0 + rank*N/2, +N/2); the bytes of both CTAs
+//                        are counted on the even CTA's stage barrier
+//   warp 1 (even CTA)    TMEM owner + MMA issue (M=256, N, K=16 per MMA);
+//                        its commits release the stage in both CTAs and mark
+//                        the accumulator full in both
+//   warps 2..5 (both)    epilogue: this CTA's 128 rows from its own TMEM,
+//                        then one arrival per warp on the even CTA's
+//                        accumulator-empty barrier
+// TMEM: two 256-column accumulators per CTA (double buffer), so the epilogue
+// of one tile overlaps the main loop of the next.
+#pragma once
+
+#include "gemm.cuh"
+#include "sm100.cuh"
+
+namespace gqe {
+
+constexpr int kPairBM = 256;  // rows per pair tile (128 per CTA)
+constexpr int kPairBN = 256;  // columns per pair tile (B: 128 per CTA)
+constexpr int kPairStages = 6;
+constexpr int kPairThreads = 192;
+
+struct PairSmem {
+  static constexpr int kABytes = 128 * kGemmBK * 2;  // 16 KB
+  static constexpr int kBBytes = 128 * kGemmBK * 2;  // two 64-column boxes of 8 KB
+  static constexpr int kStage = kABytes + kBBytes;
+  static constexpr int kBar = kPairStages * kStage;
+  static constexpr int kBytes = kBar + 256 + 1024;  // barriers + alignment slack
+};
+
+struct PairTile {
+  int m0;      // first row of the pair tile
+  int seg;     // output segment
+  int n0;      // first column within the segment
+  int nvalid;  // MMA N: multiple of 128, <= 256
+};
+
+__device__ __forceinline__ PairTile pair_decode(const GemmParams& p, int tile) {
+  PairTile t;
+  const int mt = tile / p.ntn, nt = tile % p.ntn;
+  t.m0 = mt * kPairBM;
+  t.seg = 0;
+  for (int s = 1; s < p.nseg; ++s)
+    if (nt >= p.seg[s].tile_start) t.seg = s;
+  t.n0 = (nt - p.seg[t.seg].tile_start) * kPairBN;
+  const int rem = p.seg[t.seg].n_cols - t.n0;
+  t.nvalid = rem >= kPairBN ? kPairBN : ((rem + 127) / 128) * 128;
+  return t;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ GemmParams p, int total_tiles) {
+  using L = PairSmem;
+  extern __shared__ uint8_t smem_raw[];
+  // same offset in both CTAs: the MMA addresses the peer's operands by it
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);  // [stages], used in the even CTA
+  uint64_t* empty = full + kPairStages;                           // [stages]
+  uint64_t* acc_full = empty + kPairStages;                       // [2]
+  uint64_t* acc_empty = acc_full + 2;                             // [2], used in the even CTA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int nk = (p.K + kGemmBK - 1) / kGemmBK;
+
+  if (tid == 0) {
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(&full[s], 1);   // the even producer's arrive.expect_tx
+      mbar_init(&empty[s], 1);  // the MMA commit
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 8);  // 4 epilogue warps x 2 CTAs
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_slot, 2 * kPairBN);
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tmA);
+    for (int s = 0; s < p.nseg; ++s) tma_prefetch_desc(&p.tmB[s]);
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t smem_base = smem_u32(smem);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---- TMA producer (both CTAs) --------------------------------------------
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < total_tiles; tile += npairs) {
+        const PairTile t = pair_decode(p, tile);
+        const int half = t.nvalid / 2;  // columns of B this CTA holds
+        const int nbox = half / 64;
+        const int b_col = p.seg[t.seg].b_col0 + t.n0 + (int)rank * half;
+        const CUtensorMap* tmb = &p.tmB[t.seg];
+        const int a_row = t.m0 + (int)rank * 128;
+        // pair tiles running at the same time start at different k-blocks
+        const int rot = tile % nk;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % kPairStages;
+          if (!(ok = mbar_wait(&empty[s], ((it / kPairStages) & 1) ^ 1, abort_flag))) break;
+          const uint32_t fb = mapa_shared(smem_u32(&full[s]), 0);
+          // the even CTA announces both CTAs' bytes; the odd CTA's copies may
+          // land first (the count then dips below zero until the announcement)
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * (L::kABytes + nbox * 8192));
+          const int kq = kb + rot < nk ? kb + rot : kb + rot - nk;
+          int a_col = kq * kGemmBK;
+          if (p.amap_G > 0) {
+            // k = 1 combine: A = [concat (G) | slot (G) | shared] read from O,
+            // the slot of group g being O's block g itself (weight exactly 1)
+            const int blk = kq < 2 * p.amap_G ? kq % p.amap_G : p.amap_G;
+            a_col = blk * kGemmBK;
+          }
+          uint8_t* a_s = smem + s * L::kStage;
+          uint8_t* b_s = a_s + L::kABytes;
+          tma_load_2d_pair(a_s, &p.tmA, fb, a_col, a_row);
+          for (int nb = 0; nb < nbox; ++nb) tma_load_2d_pair(b_s + nb * 8192, tmb, fb, b_col + nb * 64, kq * kGemmBK);
+        }
+      }
+      // wait until the MMA has released every stage in flight, so no commit
+      // arrival can reach this CTA after it has left
+      for (uint32_t i = it; ok && i < it + kPairStages; ++i)
+        ok = mbar_wait(&empty[i % kPairStages], ((i / kPairStages) & 1) ^ 1, abort_flag);
+    }
+  } else if (warp == 1) {
+    if (leader && lane == 0) {
+      // ---- MMA issue (even CTA) -------------------------------------------------
+      // cluster addresses of the stage-empty and accumulator-full barriers of
+      // both CTAs (a CTA's shared memory is contiguous in the cluster window)
+      const uint32_t empty_c0 = mapa_shared(smem_u32(empty), 0), empty_c1 = mapa_shared(smem_u32(empty), 1);
+      const uint32_t accf_c0 = mapa_shared(smem_u32(acc_full), 0), accf_c1 = mapa_shared(smem_u32(acc_full), 1);
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < total_tiles; tile += npairs, ++tcount) {
+        const PairTile t = pair_decode(p, tile);
+        const uint32_t a = tcount & 1;
+        if (!(ok = mbar_wait(&acc_empty[a], ((tcount >> 1) & 1) ^ 1, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + a * kPairBN;
+        const uint32_t idesc = idesc_bf16(kPairBM, t.nvalid, false, true);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % kPairStages;
+          if (!(ok = mbar_wait(&full[s], (it / kPairStages) & 1, abort_flag))) break;
+          tc_fence_after();
+          const uint32_t a_addr = smem_base + s * L::kStage;
+          const uint32_t b_addr = a_addr + L::kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kGemmBK / 16; ++kk)
+            umma_ss_pair(d_tmem, sdesc_sw128(a_addr + kk * 32, 16, 1024), sdesc_sw128(b_addr + kk * 2048, 8192, 1024),
+                         idesc, (kb | kk) != 0);
+          umma_commit_pair(empty_c0 + 8 * s);
+          umma_commit_pair(empty_c1 + 8 * s);
+        }
+        if (!ok) break;
+        umma_commit_pair(accf_c0 + 8 * a);
+        umma_commit_pair(accf_c1 + 8 * a);
+      }
+    }
+  } else {
+    // ---- epilogue (both CTAs): this CTA's 128 rows ----------------------------------
+    const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
+    const int row = q * 32 + lane;
+    const uint32_t acce_c = mapa_shared(smem_u32(acc_empty), 0);
+    uint32_t tcount = 0;
+    for (int tile = pair; tile < total_tiles; tile += npairs, ++tcount) {
+      const PairTile t = pair_decode(p, tile);
+      const uint32_t a = tcount & 1;
+      const bool ok = mbar_wait(&acc_full[a], (tcount >> 1) & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const GemmSeg& sg = p.seg[t.seg];
+      const int grow = t.m0 + (int)rank * 128 + row;
+      __nv_bfloat16* dst_row = grow < p.rows ? sg.C + (size_t)grow * sg.ldc + sg.c_col0 + t.n0 : nullptr;
+      const int ncols = min(t.nvalid, sg.n_cols - t.n0);
+      const uint32_t tm = tmem_base + a * kPairBN + (static_cast<uint32_t>(q * 32) << 16);
+      for (int cc = 0; cc < t.nvalid / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tm + cc * 32, r);
+        if (dst_row != nullptr && cc * 32 < ncols) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+          __nv_bfloat16* d = dst_row + cc * 32;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) st_global_v4(d + i * 8, pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acce_c + 8 * a);
+    }
+  }
+
+  tc_fence_before();
+  if (*abort_flag) {
+    // copies of either CTA may still be landing on this CTA's buffers
+    const unsigned long long t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 100000ull) {}
+  }
+  cluster_sync();  // no CTA leaves while its peer's MMAs or arrivals may still reach it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, 2 * kPairBN);
+  }
+}
+
+}  // namespace gqe

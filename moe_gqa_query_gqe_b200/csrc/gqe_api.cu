@@ -14,6 +14,7 @@
 #include "route.cuh"
 #include "gemm.cuh"
 #include "gemm2.cuh"
+#include "gemm2sm.cuh"
 #include "qgather.cuh"
 #include "attn.cuh"
 #include "attn2.cuh"
@@ -116,7 +117,7 @@ int set_smem(K kernel, int bytes) {
 }
 
 
-constexpr int kG2DenseBN = 256, kG2DenseStages = 4;
+constexpr int kG2DenseBN = kPairBN;
 constexpr int kRouteStages = 8;
 constexpr int kG2GatherStages = 8;
 constexpr int kG2GatherMode = kAGatherLsu;
@@ -133,6 +134,57 @@ int launch_gemm2(const GemmParams& p, long long tiles, cudaStream_t st) {
   if (tiles > 0x7fffffffll) return GQE_ERR_UNSUPPORTED;
   const int grid = (int)std::min<long long>(tiles, sm_count());
   kern<<<grid, C::kThreads, smem, st>>>(p, (int)tiles);
+  return launch_status();
+}
+
+// Clusters of two CTAs that can be resident at once for a kernel launched with
+// `threads` threads and `smem` bytes of dynamic shared memory (a pair needs two
+// free SMs of one GPC, so this can be below half the SM count). Kernels with a
+// blocked work split must not launch more pairs than this, or the surplus
+// would run as a second wave.
+template <typename K>
+int max_resident_pairs(K kernel, int threads, int smem) {
+  struct Entry {
+    const void* fn;
+    int dev, threads, smem, pairs;
+  };
+  static std::mutex mu;
+  static Entry cache[32];
+  static int ncache = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return sm_count() / 2;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < ncache; ++i)
+    if (cache[i].fn == (const void*)kernel && cache[i].dev == dev && cache[i].threads == threads &&
+        cache[i].smem == smem)
+      return cache[i].pairs;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(2 * 1024, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 2;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = sm_count() / 2;
+  }
+  if (ncache < 32) cache[ncache++] = Entry{(const void*)kernel, dev, threads, smem, n};
+  return n;
+}
+
+int launch_gemm_pair(const GemmParams& p, long long tiles, cudaStream_t st) {
+  if (int e = set_smem(gemm_pair_kernel, PairSmem::kBytes)) return e;
+  if (tiles <= 0) return GQE_OK;
+  if (tiles > 0x7fffffffll) return GQE_ERR_UNSUPPORTED;
+  const int pairs = (int)std::min<long long>(tiles, max_resident_pairs(gemm_pair_kernel, kPairThreads, PairSmem::kBytes));
+  gemm_pair_kernel<<<2 * pairs, kPairThreads, PairSmem::kBytes, st>>>(p, (int)tiles);
   return launch_status();
 }
 
@@ -166,7 +218,7 @@ int gemm_dense(const void* A, long long rows, int K, const DenseSeg* segs, int n
   p.ntn = nt;
   p.rows = (int)rows;
   p.K = K;
-  return launch_gemm2<kG2DenseBN, kG2DenseStages, kATma>(p, cdiv(rows, kGemmBM) * nt, st);
+  return launch_gemm_pair(p, cdiv(rows, kPairBM) * nt, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -412,7 +464,7 @@ int do_combine(const gqe_dims* d, const void* O, const float* w, const void* Wo,
     p.rows = (int)N;
     p.K = KA;
     p.amap_G = d->G;
-    return launch_gemm2<kG2DenseBN, kG2DenseStages, kATma>(p, cdiv(N, kGemmBM) * p.ntn, st);
+    return launch_gemm_pair(p, cdiv(N, kPairBM) * p.ntn, st);
   }
   CombineParams cp{static_cast<const __nv_bfloat16*>(O), w, A, N, d->G, d->k};
   const long long warps = N;
