@@ -290,8 +290,10 @@ def main():
         torch.cuda.synchronize()
         return g
 
-    # kernels launched per forward step (k = 1: route 3, qproj 2, attention 1, Wo 1)
-    launches_per_step = 3 + 2 + 1 + (1 if d.k == 1 else 2)
+    # kernels launched per forward step: K/V + shared-query + router pair GEMM,
+    # scan, compaction, selected-query gather, attention, Wo (+ the combine
+    # build when k > 1)
+    launches_per_step = 6 + (0 if d.k == 1 else 1)
 
     def barrier():
         if world > 1:

@@ -184,6 +184,8 @@ __device__ __forceinline__ int a2_item_of(int round) {
 }
 
 __global__ void __launch_bounds__(kA2Threads, 1) attn2_fwd_kernel(const __grid_constant__ Attn2Params p) {
+  pdl_wait();
+  pdl_trigger();
   using L = A2Smem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));

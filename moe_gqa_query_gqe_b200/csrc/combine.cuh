@@ -27,6 +27,8 @@ struct CombineParams {
 };
 
 __global__ void __launch_bounds__(256) combine_build_kernel(const CombineParams p) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;

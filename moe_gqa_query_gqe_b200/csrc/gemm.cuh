@@ -39,9 +39,14 @@ struct GemmParams {
   __nv_bfloat16* Q;        // [B*T, Ha, dh]
   int nsegs_q, G, M, k, Ha;
   int ntok;  // B*T: bound of every token index read from seg_tok
-  // routing epilogue (router logits x Wr on the tensor cores)
+  // routing tiles of the CTA-pair GEMM (router logits x Wr on the tensor
+  // cores, decisions in the epilogue): pair tiles r_tile0 .. r_tile0 +
+  // r_B*r_nblk - 1, tile (b, blk) covering tokens [blk*256, blk*256 + 256) of
+  // sequence b; r_tile0 = total tile count when there are none
+  CUtensorMap tmR;     // Wr [D, G*M], 64 x 64 boxes (columns past G*M read as zero)
+  int r_tile0, r_nblk;
   const float* r_br;   // [G*M] or null
-  int32_t* r_sel;      // [B*T, G, k]
+  int32_t* r_sel;      // [B*T, G, k]: expert | rank in the chunk << 8 (see route.cuh)
   float* r_w;          // [B*T, G, k]
   float* r_margin;     // [B*T, G] or null
   int32_t* r_counts;   // [B][nch][G*M]
@@ -51,6 +56,5 @@ struct GemmParams {
   int amap_G;
 };
 
-enum GemmEpilogue : int { kEpiStore = 0, kEpiRoute = 1 };
 
 }  // namespace gqe

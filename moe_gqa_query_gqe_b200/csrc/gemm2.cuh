@@ -48,21 +48,9 @@ struct G2Tile {
   int row0, row_end;  // gather: compacted row range of the tile
 };
 
-template <int BN, int EPI = kEpiStore>
+template <int BN>
 __device__ __forceinline__ G2Tile g2_decode(const GemmParams& p, int tile, const int* s_prefix) {
   G2Tile t;
-  if constexpr (EPI == kEpiRoute) {
-    // one tile per (batch, chunk of 128 tokens); rows past the sequence end are
-    // loaded (next sequence or zero fill) but never used
-    const int b = tile / p.r_nch, c = tile % p.r_nch;
-    t.m0 = b * p.r_T + c * kGemmBM;
-    t.seg = 0;
-    t.n0 = 0;
-    t.nvalid = 64;
-    t.row0 = b;        // batch
-    t.row_end = c;     // chunk
-    return t;
-  }
   if (s_prefix == nullptr) {
     const int mt = tile / p.ntn, nt = tile % p.ntn;
     t.m0 = mt * kGemmBM;
@@ -91,10 +79,11 @@ __device__ __forceinline__ G2Tile g2_decode(const GemmParams& p, int tile, const
   return t;
 }
 
-// RM: experts per group, compile-time in the routing epilogue (1, 2, 4 or 8)
-template <int BN, int STAGES, int AMODE, int EPI = kEpiStore, int RM = 1>
+template <int BN, int STAGES, int AMODE>
 __global__ void __launch_bounds__(G2Cfg<BN, STAGES, AMODE>::kThreads, 1)
     gemm2_kernel(const __grid_constant__ GemmParams p, int total_tiles) {
+  pdl_wait();
+  pdl_trigger();
   using C = G2Cfg<BN, STAGES, AMODE>;
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
   extern __shared__ uint8_t smem_raw[];
@@ -161,7 +150,7 @@ __global__ void __launch_bounds__(G2Cfg<BN, STAGES, AMODE>::kThreads, 1)
     uint32_t it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
-      const G2Tile t = g2_decode<BN, EPI>(p, tile, prefix);
+      const G2Tile t = g2_decode<BN>(p, tile, prefix);
       int b_col;
       const CUtensorMap* tmb;
       int tk0 = 0, tk1 = 0, tk2 = 0, tk3 = 0;
@@ -229,7 +218,7 @@ __global__ void __launch_bounds__(G2Cfg<BN, STAGES, AMODE>::kThreads, 1)
       uint32_t it = 0, tcount = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++tcount) {
-        const G2Tile t = g2_decode<BN, EPI>(p, tile, prefix);
+        const G2Tile t = g2_decode<BN>(p, tile, prefix);
         const uint32_t a = tcount & 1;
         if (!(ok = mbar_wait(&acc_empty[a], ((tcount >> 1) & 1) ^ 1, abort_flag))) break;
         tc_fence_after();
@@ -262,7 +251,7 @@ __global__ void __launch_bounds__(G2Cfg<BN, STAGES, AMODE>::kThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       auto fetch_rows = [&](int tile, int (&tk)[4]) {
-        const G2Tile t = g2_decode<BN, EPI>(p, tile, prefix);
+        const G2Tile t = g2_decode<BN>(p, tile, prefix);
         const int first = p.seg_tok[t.row0];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -300,114 +289,13 @@ __global__ void __launch_bounds__(G2Cfg<BN, STAGES, AMODE>::kThreads, 1)
       }
       asm volatile("cp.async.wait_all;" ::: "memory");  // nothing may be in flight when the CTA exits
     }
-  } else if constexpr (EPI == kEpiRoute) {
-    // ---- routing epilogue: one thread per token row ------------------------------
-    // logits[e'] = (x Wr)[row, e'] + br[e'] for e' = g*M + e; per group: top-k by
-    // logit (exact ties -> lower expert), weights renormalised over the
-    // selected set, margin k-th minus (k+1)-th logit; per-chunk expert counts.
-    const int q = warp & 3;
-    const int row = q * 32 + lane;
-    const int GM = p.G * p.M;
-    int* s_cnt = s_prefix;  // [G*M] per-tile expert counts (shared memory)
-    for (int i = tid - 64; i < GM; i += 128) s_cnt[i] = 0;
-    named_barrier_sync(1, 128);
-    uint32_t tcount = 0;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tcount) {
-      const G2Tile t = g2_decode<BN, EPI>(p, tile, prefix);
-      const uint32_t a = tcount & 1;
-      const bool ok = mbar_wait(&acc_full[a], (tcount >> 1) & 1, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      float lg[64];
-      const uint32_t tm = tmem_base + a * BN + (static_cast<uint32_t>(q * 32) << 16);
-      {
-        uint32_t r[32];
-        tmem_ld32(tm, r);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) lg[i] = __uint_as_float(r[i]);
-        if (GM > 32) {
-          tmem_ld32(tm + 32, r);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) lg[32 + i] = __uint_as_float(r[i]);
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&acc_empty[a]);
-      const int b = t.row0, c = t.row_end;
-      const int tt = c * kGemmBM + row;
-      if (tt < p.r_T) {
-        const size_t n = (size_t)b * p.r_T + tt;
-        // groups unrolled with static indices into lg (G*M <= 64)
-#pragma unroll
-        for (int g = 0; g < 64 / RM; ++g) {
-          if (g >= p.G) break;
-          float l[RM];
-#pragma unroll
-          for (int e = 0; e < RM; ++e) l[e] = p.r_br ? lg[g * RM + e] + p.r_br[g * RM + e] : lg[g * RM + e];
-          // top-k by logit, exact ties -> lower expert index
-          uint32_t chosen = 0;
-          float kth = 0.f;
-          for (int j = 0; j < p.k; ++j) {
-            int best = -1;
-            float bv = 0.f;
-#pragma unroll
-            for (int e = 0; e < RM; ++e) {
-              const bool free_e = !(chosen & (1u << e));
-              if (free_e && (best < 0 || l[e] > bv)) { best = e; bv = l[e]; }
-            }
-            chosen |= 1u << best;
-            kth = bv;
-          }
-          float mg = __int_as_float(0x7f800000);  // +inf when k == M
-          if (p.k < RM) {
-            int best = -1;
-            float bv = 0.f;
-#pragma unroll
-            for (int e = 0; e < RM; ++e) {
-              const bool free_e = !(chosen & (1u << e));
-              if (free_e && (best < 0 || l[e] > bv)) { best = e; bv = l[e]; }
-            }
-            mg = kth - bv;
-          }
-          float mx = -INFINITY;
-#pragma unroll
-          for (int e = 0; e < RM; ++e)
-            if (chosen & (1u << e)) mx = fmaxf(mx, l[e]);
-          float ex[RM];
-          float den = 0.f;
-#pragma unroll
-          for (int e = 0; e < RM; ++e) {
-            ex[e] = (chosen & (1u << e)) ? expf(l[e] - mx) : 0.f;
-            den += ex[e];
-          }
-          const float inv = 1.f / den;
-          int j = 0;
-#pragma unroll
-          for (int e = 0; e < RM; ++e) {
-            if (!(chosen & (1u << e))) continue;
-            const size_t o = (n * p.G + g) * p.k + j;
-            p.r_sel[o] = e;
-            p.r_w[o] = ex[e] * inv;
-            atomicAdd(&s_cnt[g * RM + e], 1);
-            ++j;
-          }
-          if (p.r_margin) p.r_margin[n * p.G + g] = mg;
-        }
-      }
-      named_barrier_sync(1, 128);
-      for (int i = tid - 64; i < GM; i += 128) {
-        p.r_counts[((size_t)b * p.r_nch + c) * GM + i] = s_cnt[i];
-        s_cnt[i] = 0;
-      }
-      named_barrier_sync(1, 128);
-    }
   } else {
     // ---- epilogue ---------------------------------------------------------------
     const int q = warp & 3;
     const int row = q * 32 + lane;
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tcount) {
-      const G2Tile t = g2_decode<BN, EPI>(p, tile, prefix);
+      const G2Tile t = g2_decode<BN>(p, tile, prefix);
       const uint32_t a = tcount & 1;
       const bool ok = mbar_wait(&acc_full[a], (tcount >> 1) & 1, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;

@@ -29,6 +29,7 @@
 #pragma once
 
 #include "gemm.cuh"
+#include "route.cuh"
 #include "sm100.cuh"
 
 namespace gqe {
@@ -43,18 +44,29 @@ struct PairSmem {
   static constexpr int kBBytes = 128 * kGemmBK * 2;  // two 64-column boxes of 8 KB
   static constexpr int kStage = kABytes + kBBytes;
   static constexpr int kBar = kPairStages * kStage;
-  static constexpr int kBytes = kBar + 256 + 1024;  // barriers + alignment slack
+  static constexpr int kTot = kBar + 256;             // routing epilogue: 8 groups x 4 warps of u64
+  static constexpr int kBytes = kTot + 256 + 1024;    // + alignment slack
 };
 
 struct PairTile {
   int m0;      // first row of the pair tile
-  int seg;     // output segment
-  int n0;      // first column within the segment
+  int seg;     // output segment; -1: routing tile
+  int n0;      // first column within the segment; routing tile: block of 256 tokens
   int nvalid;  // MMA N: multiple of 128, <= 256
+  int rb;      // routing tile: sequence
 };
 
 __device__ __forceinline__ PairTile pair_decode(const GemmParams& p, int tile) {
   PairTile t;
+  if (tile >= p.r_tile0) {
+    const int rt = tile - p.r_tile0;
+    t.rb = rt / p.r_nblk;
+    t.n0 = rt % p.r_nblk;
+    t.m0 = t.rb * p.r_T + t.n0 * kPairBM;
+    t.seg = -1;
+    t.nvalid = 128;  // G*M <= 64 logits in the even CTA's half; the odd half reads zeros
+    return t;
+  }
   const int mt = tile / p.ntn, nt = tile % p.ntn;
   t.m0 = mt * kPairBM;
   t.seg = 0;
@@ -63,11 +75,105 @@ __device__ __forceinline__ PairTile pair_decode(const GemmParams& p, int tile) {
   t.n0 = (nt - p.seg[t.seg].tile_start) * kPairBN;
   const int rem = p.seg[t.seg].n_cols - t.n0;
   t.nvalid = rem >= kPairBN ? kPairBN : ((rem + 127) / 128) * 128;
+  t.rb = 0;
   return t;
+}
+
+// RM (1, 2, 4 or 8) consecutive fp32 TMEM columns of this warp's 32 lanes.
+template <int RM>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&f)[RM]) {
+  if constexpr (RM == 1) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n\ttcgen05.wait::ld.sync.aligned;"
+                 : "=f"(f[0]) : "r"(taddr) : "memory");
+  } else if constexpr (RM == 2) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];\n\ttcgen05.wait::ld.sync.aligned;"
+                 : "=f"(f[0]), "=f"(f[1]) : "r"(taddr) : "memory");
+  } else if constexpr (RM == 4) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];\n\ttcgen05.wait::ld.sync.aligned;"
+                 : "=f"(f[0]), "=f"(f[1]), "=f"(f[2]), "=f"(f[3]) : "r"(taddr) : "memory");
+  } else {
+    static_assert(RM == 8, "RM");
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\ttcgen05.wait::ld.sync.aligned;"
+        : "=f"(f[0]), "=f"(f[1]), "=f"(f[2]), "=f"(f[3]), "=f"(f[4]), "=f"(f[5]), "=f"(f[6]), "=f"(f[7])
+        : "r"(taddr)
+        : "memory");
+  }
+}
+
+// Routing epilogue of one CTA of a routing pair tile: its 128 rows are chunk c
+// of sequence b (one thread per token). Per group: logits from TMEM (+ br),
+// the decision (route.cuh), then a block scan over the chunk of packed 8-bit
+// per-expert flags gives each token its rank in its experts' lists and the
+// chunk's per-expert counts. Groups go eight at a time through s_tot.
+template <int RM>
+__device__ void pair_route_epilogue(const GemmParams& p, uint32_t tm, int b, int c, int q, int lane,
+                                    unsigned long long* s_tot) {
+  const int row = q * 32 + lane;
+  const int t = c * kRouteChunk + row;
+  const bool valid = t < p.r_T;
+  const size_t n = (size_t)b * p.r_T + (valid ? t : 0);
+  const int G = p.G, k = p.k, GM = G * RM;
+  for (int g0 = 0; g0 < G; g0 += 8) {
+    const int gn = min(8, G - g0);
+    unsigned long long mine[8], incl[8];
+    uint32_t chosen[8];
+#pragma unroll
+    for (int gi = 0; gi < 8; ++gi) {
+      mine[gi] = 0;
+      chosen[gi] = 0;
+      if (gi < gn) {
+        const int g = g0 + gi;
+        float l[RM];
+        tmem_ld_cols<RM>(tm + g * RM, l);
+#pragma unroll
+        for (int e = 0; e < RM; ++e) l[e] += p.r_br ? p.r_br[g * RM + e] : 0.f;
+        const size_t o = (n * G + g) * k;
+        chosen[gi] = route_decide<RM>(l, k, valid, p.r_sel + o, p.r_w + o, p.r_margin ? p.r_margin + n * G + g : nullptr);
+        if (valid)
+#pragma unroll
+          for (int e = 0; e < RM; ++e)
+            if (chosen[gi] & (1u << e)) mine[gi] += 1ull << (8 * e);
+      }
+      incl[gi] = mine[gi];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long u = __shfl_up_sync(0xffffffffu, incl[gi], o);
+        if (lane >= o) incl[gi] += u;
+      }
+      if (lane == 31) s_tot[gi * 4 + q] = incl[gi];
+    }
+    named_barrier_sync(1, 128);
+#pragma unroll
+    for (int gi = 0; gi < 8; ++gi) {
+      if (gi >= gn) break;
+      const int g = g0 + gi;
+      unsigned long long base = 0, total = 0;
+      for (int w = 0; w < 4; ++w) {
+        if (w < q) base += s_tot[gi * 4 + w];
+        total += s_tot[gi * 4 + w];
+      }
+      const unsigned long long excl = base + incl[gi] - mine[gi];
+      if (valid) {
+        int j = 0;
+#pragma unroll
+        for (int e = 0; e < RM; ++e) {
+          if (!(chosen[gi] & (1u << e))) continue;
+          const int rank = static_cast<int>((excl >> (8 * e)) & 0xFFull);
+          p.r_sel[(n * G + g) * k + j] = e | (rank << 8);
+          ++j;
+        }
+      }
+      if (row < RM) p.r_counts[((size_t)b * p.r_nch + c) * GM + g * RM + row] = static_cast<int>((total >> (8 * row)) & 0xFFull);
+    }
+    named_barrier_sync(1, 128);
+  }
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     gemm_pair_kernel(const __grid_constant__ GemmParams p, int total_tiles) {
+  pdl_wait();
+  pdl_trigger();
   using L = PairSmem;
   extern __shared__ uint8_t smem_raw[];
   // same offset in both CTAs: the MMA addresses the peer's operands by it
@@ -78,6 +184,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   uint64_t* acc_empty = acc_full + 2;                             // [2], used in the even CTA
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  unsigned long long* s_tot = reinterpret_cast<unsigned long long*>(smem + L::kTot);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
@@ -101,6 +208,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&p.tmA);
     for (int s = 0; s < p.nseg; ++s) tma_prefetch_desc(&p.tmB[s]);
+    if (p.r_tile0 < total_tiles) tma_prefetch_desc(&p.tmR);
   }
   tc_fence_before();
   cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
@@ -117,11 +225,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const PairTile t = pair_decode(p, tile);
         const int half = t.nvalid / 2;  // columns of B this CTA holds
         const int nbox = half / 64;
-        const int b_col = p.seg[t.seg].b_col0 + t.n0 + (int)rank * half;
-        const CUtensorMap* tmb = &p.tmB[t.seg];
+        const bool rt = t.seg < 0;
+        const int b_col = rt ? (int)rank * half : p.seg[t.seg].b_col0 + t.n0 + (int)rank * half;
+        const CUtensorMap* tmb = rt ? &p.tmR : &p.tmB[t.seg];
         const int a_row = t.m0 + (int)rank * 128;
-        // pair tiles running at the same time start at different k-blocks
-        const int rot = tile % nk;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % kPairStages;
           if (!(ok = mbar_wait(&empty[s], ((it / kPairStages) & 1) ^ 1, abort_flag))) break;
@@ -129,18 +236,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           // the even CTA announces both CTAs' bytes; the odd CTA's copies may
           // land first (the count then dips below zero until the announcement)
           if (leader) mbar_arrive_expect_tx(&full[s], 2 * (L::kABytes + nbox * 8192));
-          const int kq = kb + rot < nk ? kb + rot : kb + rot - nk;
-          int a_col = kq * kGemmBK;
+          int a_col = kb * kGemmBK;
           if (p.amap_G > 0) {
             // k = 1 combine: A = [concat (G) | slot (G) | shared] read from O,
             // the slot of group g being O's block g itself (weight exactly 1)
-            const int blk = kq < 2 * p.amap_G ? kq % p.amap_G : p.amap_G;
+            const int blk = kb < 2 * p.amap_G ? kb % p.amap_G : p.amap_G;
             a_col = blk * kGemmBK;
           }
           uint8_t* a_s = smem + s * L::kStage;
           uint8_t* b_s = a_s + L::kABytes;
           tma_load_2d_pair(a_s, &p.tmA, fb, a_col, a_row);
-          for (int nb = 0; nb < nbox; ++nb) tma_load_2d_pair(b_s + nb * 8192, tmb, fb, b_col + nb * 64, kq * kGemmBK);
+          for (int nb = 0; nb < nbox; ++nb) tma_load_2d_pair(b_s + nb * 8192, tmb, fb, b_col + nb * 64, kb * kGemmBK);
         }
       }
       // wait until the MMA has released every stage in flight, so no commit
@@ -194,6 +300,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       const bool ok = mbar_wait(&acc_full[a], (tcount >> 1) & 1, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
+      if (t.seg < 0) {
+        const uint32_t tm = tmem_base + a * kPairBN + (static_cast<uint32_t>(q * 32) << 16);
+        const int c = t.n0 * 2 + (int)rank;  // this CTA's chunk of 128 tokens
+        if (c < p.r_nch) {
+          switch (p.M) {
+            case 1: pair_route_epilogue<1>(p, tm, t.rb, c, q, lane, s_tot); break;
+            case 2: pair_route_epilogue<2>(p, tm, t.rb, c, q, lane, s_tot); break;
+            case 4: pair_route_epilogue<4>(p, tm, t.rb, c, q, lane, s_tot); break;
+            default: pair_route_epilogue<8>(p, tm, t.rb, c, q, lane, s_tot); break;
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acce_c + 8 * a);
+        continue;
+      }
       const GemmSeg& sg = p.seg[t.seg];
       const int grow = t.m0 + (int)rank * 128 + row;
       __nv_bfloat16* dst_row = grow < p.rows ? sg.C + (size_t)grow * sg.ldc + sg.c_col0 + t.n0 : nullptr;

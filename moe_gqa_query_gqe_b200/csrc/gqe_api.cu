@@ -8,6 +8,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "gqe.h"
 #include "sm100.cuh"
@@ -110,6 +111,25 @@ inline int cuda_status(cudaError_t e) {
 }
 inline int launch_status() { return cuda_status(cudaGetLastError()); }
 
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel in the stream is still finishing (every kernel of
+// the library waits on it with griddepcontrol.wait before touching memory).
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, int smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...));
+}
+
 template <typename K>
 int set_smem(K kernel, int bytes) {
   // cheap after the first call on a device; keeps multi-device use correct
@@ -118,23 +138,21 @@ int set_smem(K kernel, int bytes) {
 
 
 constexpr int kG2DenseBN = kPairBN;
-constexpr int kRouteStages = 8;
 constexpr int kG2GatherStages = 8;
 constexpr int kG2GatherMode = kAGatherLsu;
 
 int sm_count();
 
-template <int BN, int STAGES, int AMODE, int EPI = kEpiStore, int RM = 1>
+template <int BN, int STAGES, int AMODE>
 int launch_gemm2(const GemmParams& p, long long tiles, cudaStream_t st) {
   using C = G2Cfg<BN, STAGES, AMODE>;
-  auto kern = gemm2_kernel<BN, STAGES, AMODE, EPI, RM>;
-  const int smem = C::kBytesBase + (AMODE != kATma ? (p.nsegs_q + 1) * 4 : 0) + (EPI == kEpiRoute ? 64 * 4 : 0);
+  auto kern = gemm2_kernel<BN, STAGES, AMODE>;
+  const int smem = C::kBytesBase + (AMODE != kATma ? (p.nsegs_q + 1) * 4 : 0);
   if (int e = set_smem(kern, smem)) return e;
   if (tiles <= 0) return GQE_OK;
   if (tiles > 0x7fffffffll) return GQE_ERR_UNSUPPORTED;
   const int grid = (int)std::min<long long>(tiles, sm_count());
-  kern<<<grid, C::kThreads, smem, st>>>(p, (int)tiles);
-  return launch_status();
+  return launch_pdl(kern, dim3(grid), dim3(C::kThreads), smem, st, p, (int)tiles);
 }
 
 // Clusters of two CTAs that can be resident at once for a kernel launched with
@@ -184,8 +202,7 @@ int launch_gemm_pair(const GemmParams& p, long long tiles, cudaStream_t st) {
   if (tiles <= 0) return GQE_OK;
   if (tiles > 0x7fffffffll) return GQE_ERR_UNSUPPORTED;
   const int pairs = (int)std::min<long long>(tiles, max_resident_pairs(gemm_pair_kernel, kPairThreads, PairSmem::kBytes));
-  gemm_pair_kernel<<<2 * pairs, kPairThreads, PairSmem::kBytes, st>>>(p, (int)tiles);
-  return launch_status();
+  return launch_pdl(gemm_pair_kernel, dim3(2 * pairs), dim3(kPairThreads), PairSmem::kBytes, st, p, (int)tiles);
 }
 
 // Dense multi-segment projection: A [rows, K] times up to three weights.
@@ -199,8 +216,9 @@ struct DenseSeg {
   int c_col0;
 };
 
-int gemm_dense(const void* A, long long rows, int K, const DenseSeg* segs, int nseg, cudaStream_t st) {
-  GemmParams p;
+// Pair-GEMM parameters of a dense multi-segment projection; returns the
+// number of pair tiles (no routing tiles yet).
+int dense_params(GemmParams& p, const void* A, long long rows, int K, const DenseSeg* segs, int nseg, long long* tiles) {
   memset(&p, 0, sizeof(p));
   if (int e = tmap_rows(&p.tmA, A, rows, K, K, kGemmBM)) return e;
   int nt = 0;
@@ -218,7 +236,16 @@ int gemm_dense(const void* A, long long rows, int K, const DenseSeg* segs, int n
   p.ntn = nt;
   p.rows = (int)rows;
   p.K = K;
-  return launch_gemm_pair(p, cdiv(rows, kPairBM) * nt, st);
+  *tiles = nt > 0 ? cdiv(rows, kPairBM) * nt : 0;
+  p.r_tile0 = 0x7fffffff;
+  return GQE_OK;
+}
+
+int gemm_dense(const void* A, long long rows, int K, const DenseSeg* segs, int nseg, cudaStream_t st) {
+  GemmParams p;
+  long long tiles = 0;
+  if (int e = dense_params(p, A, rows, K, segs, nseg, &tiles)) return e;
+  return launch_gemm_pair(p, tiles, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -316,8 +343,34 @@ int check_device() {
 // ---------------------------------------------------------------------------
 // Stage implementations (arguments already validated)
 // ---------------------------------------------------------------------------
-int do_route(const gqe_dims* d, const void* x, const void* Wr, const float* br, int32_t* sel, float* w,
-             float* margin, int32_t* seg_off, int32_t* seg_tok, int32_t* row_map, RouteWs rw, cudaStream_t st) {
+// Routing tiles (router logits and decisions, gemm2sm.cuh) appended to the
+// pair-GEMM launch `p` over x, starting at pair tile `tile0`; returns in
+// *tiles the number added. p.tmA must already map x with 128-row boxes.
+int add_route_tiles(GemmParams& p, const gqe_dims* d, const void* Wr, const float* br, int32_t* sel, float* w,
+                    float* margin, RouteWs rw, long long tile0, long long* tiles) {
+  const int GM = d->G * d->M;
+  GQE_TRY(tmap_rows(&p.tmR, Wr, d->D, GM, GM, 64));  // 64-wide box: columns past G*M read as zero
+  p.K = d->D;
+  p.G = d->G;
+  p.M = d->M;
+  p.k = d->k;
+  p.r_br = br;
+  p.r_sel = sel;
+  p.r_w = w;
+  p.r_margin = margin;
+  p.r_counts = rw.counts;
+  p.r_B = d->B;
+  p.r_T = d->T;
+  p.r_nch = (int)cdiv(d->T, kRouteChunk);
+  p.r_nblk = (int)cdiv(d->T, kPairBM);
+  p.r_tile0 = (int)tile0;
+  *tiles = (long long)d->B * p.r_nblk;
+  return tile0 + *tiles > 0x7fffffffll ? GQE_ERR_UNSUPPORTED : GQE_OK;
+}
+
+// After the routing tiles: segment offsets, chunk bases, compacted lists.
+int route_finish(const gqe_dims* d, int32_t* sel, int32_t* seg_off, int32_t* seg_tok, int32_t* row_map, RouteWs rw,
+                 cudaStream_t st) {
   RouteParams rp;
   rp.sel = sel;
   rp.counts = rw.counts;
@@ -331,57 +384,43 @@ int do_route(const gqe_dims* d, const void* x, const void* Wr, const float* br, 
   rp.M = d->M;
   rp.k = d->k;
   rp.nch = (int)cdiv(d->T, kRouteChunk);
-  const long long grid = (long long)d->B * rp.nch;
-  {
-    // router logits on the tensor cores, routing decisions in the epilogue
-    GemmParams gp;
-    memset(&gp, 0, sizeof(gp));
-    const long long N = (long long)d->B * d->T;
-    const int GM = d->G * d->M;
-    GQE_TRY(tmap_rows(&gp.tmA, x, N, d->D, d->D, kGemmBM));
-    GQE_TRY(tmap_rows(&gp.tmB[0], Wr, d->D, GM, GM, 64));  // 64-wide box: columns past G*M read as zero
-    gp.nseg = 1;
-    gp.seg[0].n_cols = 64;
-    gp.K = d->D;
-    gp.G = d->G;
-    gp.M = d->M;
-    gp.k = d->k;
-    gp.r_br = br;
-    gp.r_sel = sel;
-    gp.r_w = w;
-    gp.r_margin = margin;
-    gp.r_counts = rw.counts;
-    gp.r_B = d->B;
-    gp.r_T = d->T;
-    gp.r_nch = rp.nch;
-    switch (d->M) {
-      case 1: GQE_TRY((launch_gemm2<64, kRouteStages, kATma, kEpiRoute, 1>(gp, grid, st))); break;
-      case 2: GQE_TRY((launch_gemm2<64, kRouteStages, kATma, kEpiRoute, 2>(gp, grid, st))); break;
-      case 4: GQE_TRY((launch_gemm2<64, kRouteStages, kATma, kEpiRoute, 4>(gp, grid, st))); break;
-      case 8: GQE_TRY((launch_gemm2<64, kRouteStages, kATma, kEpiRoute, 8>(gp, grid, st))); break;
-      default: return GQE_ERR_UNSUPPORTED;
-    }
-  }
   const int nseg = d->B * d->G * d->M;
-  route_scan_kernel<<<1, 1024, nseg * 4, st>>>(rp);
-  GQE_TRY(launch_status());
-  route_scatter_kernel<<<(unsigned)grid, kRouteChunk, 0, st>>>(rp);
-  return launch_status();
+  GQE_TRY(launch_pdl(route_scan_kernel, dim3(1), dim3(1024), nseg * 4, st, rp));
+  const long long rows = (long long)d->B * d->T * d->G * d->k;
+  const long long blocks = std::min<long long>(cdiv(rows, 256), (long long)sm_count() * 8);
+  return launch_pdl(route_finalize_kernel, dim3((unsigned)std::max<long long>(blocks, 1)), dim3(256), 0, st, rp);
 }
 
-int do_qproj(const gqe_dims* d, const void* x, const void* Wq, const void* Wk, const void* Wv, const int32_t* sel,
-             const int32_t* seg_off, const int32_t* seg_tok, void* Q, void* K, void* V, cudaStream_t st) {
+int do_route(const gqe_dims* d, const void* x, const void* Wr, const float* br, int32_t* sel, float* w,
+             float* margin, int32_t* seg_off, int32_t* seg_tok, int32_t* row_map, RouteWs rw, cudaStream_t st) {
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  const long long N = (long long)d->B * d->T;
+  GQE_TRY(tmap_rows(&p.tmA, x, N, d->D, d->D, kGemmBM));
+  p.rows = (int)N;
+  long long tiles = 0;
+  GQE_TRY(add_route_tiles(p, d, Wr, br, sel, w, margin, rw, 0, &tiles));
+  GQE_TRY(launch_gemm_pair(p, tiles, st));
+  return route_finish(d, sel, seg_off, seg_tok, row_map, rw, st);
+}
+
+// The dense part of the query/key/value projections, one launch over x: K,
+// V and the shared head's query.
+void kv_segments(const gqe_dims* d, const void* Wq, const void* Wk, const void* Wv, void* Q, void* K, void* V,
+                 DenseSeg (&segs)[3]) {
+  const int G = d->G, M = d->M, k = d->k, Ha = G * k + 1;
+  const int wq_cols = (G * M + 1) * 64;
+  segs[0] = DenseSeg{Wk, G * 64, 0, G * 64, K, (long long)G * 64, 0};
+  segs[1] = DenseSeg{Wv, G * 64, 0, G * 64, V, (long long)G * 64, 0};
+  segs[2] = DenseSeg{Wq, wq_cols, G * M * 64, 64, Q, (long long)Ha * 64, G * k * 64};
+}
+
+// Selected experts: one segment per (b, g, e), rows gathered by seg_tok.
+int do_qgather(const gqe_dims* d, const void* x, const void* Wq, const int32_t* sel, const int32_t* seg_off,
+               const int32_t* seg_tok, void* Q, cudaStream_t st) {
   const long long N = (long long)d->B * d->T;
   const int G = d->G, M = d->M, k = d->k, Ha = G * k + 1;
   const int wq_cols = (G * M + 1) * 64;
-  // dense part: K, V and the shared head's query, one launch over x
-  const DenseSeg segs[3] = {
-      {Wk, G * 64, 0, G * 64, K, (long long)G * 64, 0},
-      {Wv, G * 64, 0, G * 64, V, (long long)G * 64, 0},
-      {Wq, wq_cols, G * M * 64, 64, Q, (long long)Ha * 64, G * k * 64},
-  };
-  GQE_TRY(gemm_dense(x, N, d->D, segs, 3, st));
-  // selected experts: one segment per (b, g, e), rows gathered by seg_tok
   GemmParams p;
   memset(&p, 0, sizeof(p));
   GQE_TRY(tmap_rows(&p.tmB[0], Wq, d->D, wq_cols, wq_cols, 64));
@@ -399,15 +438,24 @@ int do_qproj(const gqe_dims* d, const void* x, const void* Wq, const void* Wk, c
   p.Ha = Ha;
   p.ntok = (int)N;
   const long long tiles_max = cdiv(N * G * k, kGemmBM) + p.nsegs_q;
-  const int qg_smem = QgSmem::kBytesBase + (p.nsegs_q + 1) * 4;
-  if (d->D <= kQgMaxK && qg_smem <= 227 * 1024) {
+  const int nk = d->D / kGemmBK;
+  const int qg_stages = std::min(kQgMaxStages, (232448 - QgLayout{0, nk}.bytes(p.nsegs_q)) / 16384);
+  if (d->D <= kQgMaxK && d->D % kGemmBK == 0 && qg_stages >= kQgMinStages) {
     // the head's weight slice stays resident in shared memory
+    const int qg_smem = QgLayout{qg_stages, nk}.bytes(p.nsegs_q);
     GQE_TRY(set_smem(qgather_kernel, qg_smem));
     const int grid = (int)std::min<long long>(tiles_max, sm_count());
-    qgather_kernel<<<grid, kQgThreads, qg_smem, st>>>(p);
-    return launch_status();
+    return launch_pdl(qgather_kernel, dim3(grid), dim3(kQgThreads), qg_smem, st, p, qg_stages);
   }
   return launch_gemm2<64, kG2GatherStages, kG2GatherMode>(p, tiles_max, st);
+}
+
+int do_qproj(const gqe_dims* d, const void* x, const void* Wq, const void* Wk, const void* Wv, const int32_t* sel,
+             const int32_t* seg_off, const int32_t* seg_tok, void* Q, void* K, void* V, cudaStream_t st) {
+  DenseSeg segs[3];
+  kv_segments(d, Wq, Wk, Wv, Q, K, V, segs);
+  GQE_TRY(gemm_dense(x, (long long)d->B * d->T, d->D, segs, 3, st));
+  return do_qgather(d, x, Wq, sel, seg_off, seg_tok, Q, st);
 }
 
 int sm_count() {
@@ -442,8 +490,7 @@ int do_attn2(const gqe_dims* d, const void* Q, int Hq, const void* K, const void
   p.scale_log2 = 1.4426950408889634f / sqrtf(64.f);
   GQE_TRY(set_smem(attn2_fwd_kernel, A2Smem::kBytes));
   const int grid = (int)std::min<long long>(items, sm_count());
-  attn2_fwd_kernel<<<grid, kA2Threads, A2Smem::kBytes, st>>>(p);
-  return launch_status();
+  return launch_pdl(attn2_fwd_kernel, dim3(grid), dim3(kA2Threads), A2Smem::kBytes, st, p);
 }
 
 int do_combine(const gqe_dims* d, const void* O, const float* w, const void* Wo, void* y, __nv_bfloat16* A,
@@ -464,13 +511,13 @@ int do_combine(const gqe_dims* d, const void* O, const float* w, const void* Wo,
     p.rows = (int)N;
     p.K = KA;
     p.amap_G = d->G;
+    p.r_tile0 = 0x7fffffff;
     return launch_gemm_pair(p, cdiv(N, kPairBM) * p.ntn, st);
   }
   CombineParams cp{static_cast<const __nv_bfloat16*>(O), w, A, N, d->G, d->k};
   const long long warps = N;
   const long long blocks = std::min<long long>(cdiv(warps * 32, 256), 148ll * 16);
-  combine_build_kernel<<<(unsigned)blocks, 256, 0, st>>>(cp);
-  GQE_TRY(launch_status());
+  GQE_TRY(launch_pdl(combine_build_kernel, dim3((unsigned)blocks), dim3(256), 0, st, cp));
   const DenseSeg seg = {Wo, d->D, 0, d->D, y, (long long)d->D, 0};
   return gemm_dense(A, N, KA, &seg, 1, st);
 }
@@ -567,8 +614,17 @@ int gqe_forward(const gqe_dims* d, const void* x, const void* Wq, const void* Wk
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Carver c{static_cast<uint8_t*>(ws)};
   FwdWs f = carve_forward(c, d);
-  GQE_TRY(do_route(d, x, Wr, br, f.sel, f.w, f.margin, f.seg_off, f.seg_tok, f.row_map, f.route, st));
-  GQE_TRY(do_qproj(d, x, Wq, Wk, Wv, f.sel, f.seg_off, f.seg_tok, f.Q, f.K, f.V, st));
+  // one pair-GEMM launch over x: K, V, the shared head's query and the router
+  // (logits and decisions), then the compaction and the selected queries
+  DenseSeg segs[3];
+  kv_segments(d, Wq, Wk, Wv, f.Q, f.K, f.V, segs);
+  GemmParams p;
+  long long dense_tiles = 0, route_tiles = 0;
+  GQE_TRY(dense_params(p, x, (long long)d->B * d->T, d->D, segs, 3, &dense_tiles));
+  GQE_TRY(add_route_tiles(p, d, Wr, br, f.sel, f.w, f.margin, f.route, dense_tiles, &route_tiles));
+  GQE_TRY(launch_gemm_pair(p, dense_tiles + route_tiles, st));
+  GQE_TRY(route_finish(d, f.sel, f.seg_off, f.seg_tok, f.row_map, f.route, st));
+  GQE_TRY(do_qgather(d, x, Wq, f.sel, f.seg_off, f.seg_tok, f.Q, st));
   GQE_TRY(do_attn2(d, f.Q, d->G * d->k + 1, f.K, f.V, f.O, false, st));
   return do_combine(d, f.O, f.w, Wo, y, f.A, st);
 }

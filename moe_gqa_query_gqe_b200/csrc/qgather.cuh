@@ -27,34 +27,42 @@
 
 namespace gqe {
 
-constexpr int kQgStages = 5;
+constexpr int kQgMaxStages = 12;
+constexpr int kQgMinStages = 4;
 constexpr int kQgThreads = 448;
 constexpr int kQgMaxK = 1024;  // resident weight slice: K x 64 bf16 <= 128 KB
+constexpr int kQgBarBytes = 512;
 
-struct QgSmem {
-  static constexpr int kA = 0;                              // kQgStages x 16 KB
-  static constexpr int kB = kQgStages * 16384;              // kQgMaxK/64 boxes of 8 KB
-  static constexpr int kBar = kB + (kQgMaxK / 64) * 8192;
-  static constexpr int kPrefix = kBar + 256;
-  static constexpr int kBytesBase = kPrefix + 1024;         // + (nsegs + 1) * 4
+// Shared memory: `stages` A stages of 16 KB, the resident weight slice (nk
+// boxes of 8 KB), barriers, the tile prefix over the segments. As many
+// stages as fit (the gather is bound by the bytes in flight).
+struct QgLayout {
+  int stages, nk;
+  __host__ __device__ int a_off(int s) const { return s * 16384; }
+  __host__ __device__ int b_off() const { return stages * 16384; }
+  __host__ __device__ int bar_off() const { return b_off() + nk * 8192; }
+  __host__ __device__ int prefix_off() const { return bar_off() + kQgBarBytes; }
+  __host__ __device__ int bytes(int nsegs) const { return prefix_off() + (nsegs + 1) * 4 + 1024; }
 };
 
-__global__ void __launch_bounds__(kQgThreads, 1) qgather_kernel(const __grid_constant__ GemmParams p) {
-  using L = QgSmem;
+__global__ void __launch_bounds__(kQgThreads, 1) qgather_kernel(const __grid_constant__ GemmParams p, int stages) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);  // [stages]
-  uint64_t* empty = full + kQgStages;                             // [stages]
-  uint64_t* acc_full = empty + kQgStages;                         // [2]
+  const int nk = p.K / kGemmBK;
+  const QgLayout L{stages, nk};
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off());  // [stages]
+  uint64_t* empty = full + kQgMaxStages;                              // [stages]
+  uint64_t* acc_full = empty + kQgMaxStages;                          // [2]
   uint64_t* acc_empty = acc_full + 2;                             // [2]
   uint64_t* b_full = acc_empty + 2;
   uint64_t* b_empty = b_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(b_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* s_prefix = reinterpret_cast<int*>(smem + L::kPrefix);
+  int* s_prefix = reinterpret_cast<int*>(smem + L.prefix_off());
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nk = p.K / kGemmBK;
   const int GM = p.G * p.M;
 
   if (warp == 0) {
@@ -76,7 +84,7 @@ __global__ void __launch_bounds__(kQgThreads, 1) qgather_kernel(const __grid_con
     if (lane == 0) s_prefix[p.nsegs_q] = before;
   }
   if (tid == 0) {
-    for (int s = 0; s < kQgStages; ++s) {
+    for (int s = 0; s < stages; ++s) {
       mbar_init(&full[s], 256);  // one cp.async-tracked arrival per copier thread
       mbar_init(&empty[s], 1);
     }
@@ -121,7 +129,7 @@ __global__ void __launch_bounds__(kQgThreads, 1) qgather_kernel(const __grid_con
         if (loads > 0 && !mbar_wait(b_empty, (loads - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(b_full, nk * 8192);
         for (int kb = 0; kb < nk; ++kb)
-          tma_load_2d(smem + L::kB + kb * 8192, &p.tmB[0], b_full, head * 64, kb * kGemmBK);
+          tma_load_2d(smem + L.b_off() + kb * 8192, &p.tmB[0], b_full, head * 64, kb * kGemmBK);
         cur_head = head;
         ++loads;
       }
@@ -131,7 +139,9 @@ __global__ void __launch_bounds__(kQgThreads, 1) qgather_kernel(const __grid_con
       // ---- MMA issue ------------------------------------------------------------
       constexpr uint32_t idesc = idesc_bf16(kGemmBM, 64, false, true);
       int cur_head = -1;
-      uint32_t loads = 0, it = 0, tcount = 0;
+      uint32_t loads = 0, tcount = 0;
+      int s = 0;
+      uint32_t ph = 0;  // stage s and the parity of its current use (no division in the loop)
       bool ok = true;
       for (int tile = first; ok && tile < last; ++tile, ++tcount) {
         const int head = seg_of(tile) % GM;
@@ -144,18 +154,21 @@ __global__ void __launch_bounds__(kQgThreads, 1) qgather_kernel(const __grid_con
         if (!(ok = mbar_wait(&acc_empty[a], ((tcount >> 1) & 1) ^ 1, abort_flag))) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + a * 64;
-        for (int kb = 0; kb < nk; ++kb, ++it) {
-          const int s = it % kQgStages;
-          if (!(ok = mbar_wait(&full[s], (it / kQgStages) & 1, abort_flag))) break;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!(ok = mbar_wait(&full[s], ph, abort_flag))) break;
           fence_proxy_async_smem();  // rows copied by cp.async (generic proxy) feed the MMA (async proxy)
           tc_fence_after();
-          const uint32_t a_addr = smem_base + L::kA + s * 16384;
-          const uint32_t b_addr = smem_base + L::kB + kb * 8192;
+          const uint32_t a_addr = smem_base + L.a_off(s);
+          const uint32_t b_addr = smem_base + L.b_off() + kb * 8192;
 #pragma unroll
           for (int kk = 0; kk < kGemmBK / 16; ++kk)
             umma_ss(d_tmem, sdesc_sw128(a_addr + kk * 32, 16, 1024), sdesc_sw128(b_addr + kk * 2048, 8192, 1024),
                     idesc, (kb | kk) != 0);
           umma_commit(&empty[s]);
+          if (++s == stages) {
+            s = 0;
+            ph ^= 1;
+          }
         }
         umma_commit(&acc_full[a]);
         // the weight slice may be replaced once this run's last tile is issued
@@ -211,17 +224,21 @@ __global__ void __launch_bounds__(kQgThreads, 1) qgather_kernel(const __grid_con
     // ---- copiers (warps 6..13): 16-byte chunk c of rows r = i*32 + ct/8 ---------------
     const int ct = tid - 192;  // 0..255
     const int c = ct & 7;
-    uint32_t it = 0;
+    int s = 0;
+    uint32_t ph = 0;
     bool ok = true;
+    // The next tile's token rows are loaded while this tile's copies run. Rows
+    // past the segment re-read its first row (their results are never
+    // stored); the row index is clamped before the load and nothing reads the
+    // loaded values until the tile boundary, so the loads do not stall here.
     auto fetch_rows = [&](int tile, int (&tk)[4]) {
       const int seg = seg_of(tile);
       const int row0 = p.seg_off[seg] + (tile - s_prefix[seg]) * kGemmBM;
       const int row_end = min(p.seg_off[seg + 1], p.seg_off[p.nsegs_q]);
-      const int first_tok = p.seg_tok[row0];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int r = i * 32 + (ct >> 3);
-        tk[i] = (row0 + r < row_end) ? p.seg_tok[row0 + r] : first_tok;
+        tk[i] = p.seg_tok[row0 + r < row_end ? row0 + r : row0];
       }
     };
     int tk_cur[4] = {0, 0, 0, 0}, tk_next[4] = {0, 0, 0, 0};
@@ -241,13 +258,16 @@ __global__ void __launch_bounds__(kQgThreads, 1) qgather_kernel(const __grid_con
         src[i] = p.x + (size_t)v * p.K + c * 8;
         dst_off[i] = r * 128 + ((c ^ (r & 7)) << 4);
       }
-      for (int kb = 0; kb < nk; ++kb, ++it) {
-        const int s = it % kQgStages;
-        if (!(ok = mbar_wait(&empty[s], ((it / kQgStages) & 1) ^ 1, abort_flag))) break;
-        const uint32_t a_addr = smem_base + L::kA + s * 16384;
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!(ok = mbar_wait(&empty[s], ph ^ 1, abort_flag))) break;
+        const uint32_t a_addr = smem_base + L.a_off(s);
 #pragma unroll
         for (int i = 0; i < 4; ++i) cp_async_16_full(a_addr + dst_off[i], src[i] + kb * kGemmBK);
         cp_async_mbar_arrive_noinc(&full[s]);  // arrives when these copies land
+        if (++s == stages) {
+          s = 0;
+          ph ^= 1;
+        }
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) tk_cur[i] = tk_next[i];

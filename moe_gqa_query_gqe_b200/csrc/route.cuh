@@ -7,22 +7,26 @@
 // probabilities); animattoys.com article, section 4 (a light router scores the
 // experts of each group and activates the k best).
 //
-// Three launches, no host synchronisation between them:
-//   router logits + decisions: x Wr on the tensor cores (gemm2.cuh, routing
-//                         epilogue): logits + br (fp32), in-group top-k,
-//                         renormalised weights, margins, per-chunk counts of
-//                         every (group, expert)
+// Three steps, no host synchronisation between them:
+//   router logits + decisions: x Wr on the tensor cores as 256-row tiles of
+//                         the CTA-pair GEMM (gemm2sm.cuh; alone, or next to the
+//                         K/V projection tiles over the same x). Each CTA's
+//                         epilogue holds one chunk of 128 tokens of one
+//                         sequence: logits + br (fp32), in-group top-k,
+//                         renormalised weights, margins, every token's rank in
+//                         its experts' lists within the chunk (kept in sel's
+//                         upper bits until the last step), per-chunk counts
 //   route_scan_kernel   : exclusive scans of the counts -> segment offsets and
 //                         per-chunk bases inside each segment
-//   route_scatter_kernel: block-scan of packed per-expert flags -> the
-//                         compacted token list of every segment and row_map
+//   route_finalize_kernel: segment offset + chunk base + rank -> the compacted
+//                         token list of every segment and row_map
 #pragma once
 
 #include "sm100.cuh"
 
 namespace gqe {
 
-constexpr int kRouteChunk = 128;      // tokens per chunk (= one routing GEMM tile, one scatter CTA)
+constexpr int kRouteChunk = 128;  // tokens per chunk (= the rows of one CTA of a routing pair tile)
 
 struct RouteParams {
   int32_t* sel;
@@ -34,8 +38,75 @@ struct RouteParams {
   int B, T, G, M, k, nch;
 };
 
+// Decision of one group for one token from its RM logits (br included): top-k
+// by logit, exact ties to the lower expert; weights = softmax over the
+// selected logits only (the in-group softmax renormalised over the selected
+// set); margin = k-th largest minus (k+1)-th largest logit (+inf when k == M).
+// Returns the selected experts as a bit mask; when `out` is true writes
+// sel[.., j] (ascending expert order), w[.., j] and the margin.
+template <int RM>
+__device__ __forceinline__ uint32_t route_decide(const float (&l)[RM], int k, bool out, int32_t* sel, float* w,
+                                                 float* margin) {
+  uint32_t chosen = 0;
+  float kth = 0.f;
+  for (int j = 0; j < k; ++j) {
+    int best = -1;
+    float bv = 0.f;
+#pragma unroll
+    for (int e = 0; e < RM; ++e) {
+      const bool free_e = !(chosen & (1u << e));
+      if (free_e && (best < 0 || l[e] > bv)) {
+        best = e;
+        bv = l[e];
+      }
+    }
+    chosen |= 1u << best;
+    kth = bv;
+  }
+  float mg = __int_as_float(0x7f800000);  // +inf when k == M
+  if (k < RM) {
+    int best = -1;
+    float bv = 0.f;
+#pragma unroll
+    for (int e = 0; e < RM; ++e) {
+      const bool free_e = !(chosen & (1u << e));
+      if (free_e && (best < 0 || l[e] > bv)) {
+        best = e;
+        bv = l[e];
+      }
+    }
+    mg = kth - bv;
+  }
+  if (out) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < RM; ++e)
+      if (chosen & (1u << e)) mx = fmaxf(mx, l[e]);
+    float ex[RM];
+    float den = 0.f;
+#pragma unroll
+    for (int e = 0; e < RM; ++e) {
+      ex[e] = (chosen & (1u << e)) ? expf(l[e] - mx) : 0.f;
+      den += ex[e];
+    }
+    const float inv = 1.f / den;
+    int j = 0;
+#pragma unroll
+    for (int e = 0; e < RM; ++e) {
+      if (!(chosen & (1u << e))) continue;
+      sel[j] = e;
+      w[j] = ex[e] * inv;
+      ++j;
+    }
+    if (margin) *margin = mg;
+  }
+  return chosen;
+}
+
 // One CTA. Segment s = b*GM + g*M + e (= (b*G + g)*M + e).
 __global__ void __launch_bounds__(1024) route_scan_kernel(const RouteParams p) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int s_tot[];  // [nseg]
   const int GM = p.G * p.M;
   const int nseg = p.B * GM;
@@ -77,48 +148,36 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const RouteParams p) {
   }
 }
 
-// One CTA per chunk of kRouteChunk tokens, one thread per token. For every
-// group, each thread packs one 8-bit count per expert (M <= 8, counts <= 128)
-// into a 64-bit word; a block-wide exclusive scan of the words gives every
-// token its rank inside each expert's list for this chunk.
-__global__ void __launch_bounds__(kRouteChunk) route_scatter_kernel(const RouteParams p) {
-  __shared__ unsigned long long s_warp[kRouteChunk / 32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int b = blockIdx.x / p.nch, c = blockIdx.x % p.nch;
-  const int t = c * kRouteChunk + tid;
-  const bool valid = t < p.T;
-  const size_t n = (size_t)b * p.T + (valid ? t : 0);
-  const int GM = p.G * p.M;
-  for (int g = 0; g < p.G; ++g) {
-    int es[8];
-    unsigned long long mine = 0;
-    for (int j = 0; j < p.k; ++j) {
-      es[j] = valid ? p.sel[(n * p.G + g) * p.k + j] : 0;
-      if (valid) mine += 1ull << (8 * es[j]);
+// One thread per (token, group, selection). The routing epilogue leaves
+// sel = e | rank << 8, rank being the token's place in expert e's list within
+// its chunk; here it becomes the row of the compacted list and sel goes back
+// to the expert index.
+__global__ void __launch_bounds__(256) route_finalize_kernel(const RouteParams p) {
+  pdl_wait();
+  pdl_trigger();
+  const int GM = p.G * p.M, Gk = p.G * p.k;
+  const long long total = (long long)p.B * p.T * Gk;
+  const long long rows = total;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long n = i / Gk;
+    const int g = (int)(i % Gk) / p.k;
+    const int b = (int)(n / p.T), c = (int)(n % p.T) / kRouteChunk;
+    const int packed = p.sel[i];
+    const int e = packed & 0xFF, rank = packed >> 8;
+    p.sel[i] = e;
+    if (e >= p.M || rank < 0 || rank >= kRouteChunk) {
+      flag_bounds_error();
+      continue;
     }
-    unsigned long long incl = mine;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned long long u = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += u;
+    const int ge = g * p.M + e;
+    const long long dst = (long long)p.seg_off[b * GM + ge] + p.chunk_base[((size_t)b * p.nch + c) * GM + ge] + rank;
+    if (dst < 0 || dst >= rows) {
+      flag_bounds_error();
+      continue;
     }
-    if (lane == 31) s_warp[warp] = incl;
-    __syncthreads();
-    unsigned long long base = 0;
-    for (int w2 = 0; w2 < warp; ++w2) base += s_warp[w2];
-    const unsigned long long excl = base + incl - mine;
-    if (valid) {
-      for (int j = 0; j < p.k; ++j) {
-        const int e = es[j];
-        const int rank = static_cast<int>((excl >> (8 * e)) & 0xFFull);
-        const int ge = g * p.M + e;
-        const long long dst = (long long)p.seg_off[b * GM + ge] + p.chunk_base[((size_t)b * p.nch + c) * GM + ge] + rank;
-        if (dst < 0 || dst >= (long long)p.B * p.T * p.G * p.k) { flag_bounds_error(); continue; }
-        p.seg_tok[dst] = static_cast<int32_t>(n);
-        if (p.row_map) p.row_map[(n * p.G + g) * p.k + j] = static_cast<int32_t>(dst);
-      }
-    }
-    __syncthreads();
+    p.seg_tok[dst] = static_cast<int32_t>(n);
+    if (p.row_map) p.row_map[i] = static_cast<int32_t>(dst);
   }
 }
 

@@ -356,6 +356,18 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar_cluster) {
                : "memory");
 }
 
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch. Every kernel of the library is launched so
+// that it may start while the previous kernel in the stream is finishing; it
+// calls pdl_wait() before its first access to global memory, which returns
+// once that kernel has completed and its writes are visible (immediately when
+// launched without the attribute), then pdl_trigger() so the next kernel can
+// be scheduled early. The next grid only launches once every CTA of this one
+// has triggered or exited, so an early trigger cannot starve this grid.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Named barrier over a subset of the CTA's warps (ids 1..15; 0 is __syncthreads).
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
