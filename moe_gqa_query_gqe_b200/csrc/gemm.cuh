@@ -26,6 +26,7 @@ struct GemmSeg {
 struct GemmParams {
   CUtensorMap tmA;
   CUtensorMap tmB[kMaxGemmSegs];
+  CUtensorMap tmC[kMaxGemmSegs];  // CTA-pair GEMM: output of segment s, box 64 cols x 32 rows (TMA stores)
   GemmSeg seg[kMaxGemmSegs];
   int nseg;
   int ntn;   // n-tiles over all segments

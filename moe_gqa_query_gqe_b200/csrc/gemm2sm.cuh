@@ -22,8 +22,10 @@
 //                        its commits release the stage in both CTAs and mark
 //                        the accumulator full in both
 //   warps 2..5 (both)    epilogue: this CTA's 128 rows from its own TMEM,
-//                        then one arrival per warp on the even CTA's
-//                        accumulator-empty barrier
+//                        converted to bf16 into swizzled shared-memory rows
+//                        (one row per lane) and written by TMA stores of 32
+//                        rows x 64 columns, then one arrival per warp on the
+//                        even CTA's accumulator-empty barrier
 // TMEM: two 256-column accumulators per CTA (double buffer), so the epilogue
 // of one tile overlaps the main loop of the next.
 #pragma once
@@ -43,8 +45,11 @@ struct PairSmem {
   static constexpr int kABytes = 128 * kGemmBK * 2;  // 16 KB
   static constexpr int kBBytes = 128 * kGemmBK * 2;  // two 64-column boxes of 8 KB
   static constexpr int kStage = kABytes + kBBytes;
-  static constexpr int kBar = kPairStages * kStage;
-  static constexpr int kTot = kBar + 256;             // routing epilogue: 8 groups x 4 warps of u64
+  static constexpr int kBar = kPairStages * kStage;  // (end of the stages)
+  static constexpr int kStageOut = kBar;               // epilogue staging: 4 warps x 2 x (32 rows x 128 B)
+  static constexpr int kOutBytes = 4096;
+  static constexpr int kBarOff = kStageOut + 4 * 2 * kOutBytes;
+  static constexpr int kTot = kBarOff + 256;          // routing epilogue: 8 groups x 4 warps of u64
   static constexpr int kBytes = kTot + 256 + 1024;    // + alignment slack
 };
 
@@ -178,7 +183,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   // same offset in both CTAs: the MMA addresses the peer's operands by it
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);  // [stages], used in the even CTA
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);  // [stages], used in the even CTA
   uint64_t* empty = full + kPairStages;                           // [stages]
   uint64_t* acc_full = empty + kPairStages;                       // [2]
   uint64_t* acc_empty = acc_full + 2;                             // [2], used in the even CTA
@@ -293,6 +298,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
     const int row = q * 32 + lane;
     const uint32_t acce_c = mapa_shared(smem_u32(acc_empty), 0);
+    uint8_t* stage_out = smem + L::kStageOut + q * 2 * L::kOutBytes;  // this warp's two staging buffers
+    uint32_t nstore = 0;                                               // chunks staged by this warp
     uint32_t tcount = 0;
     for (int tile = pair; tile < total_tiles; tile += npairs, ++tcount) {
       const PairTile t = pair_decode(p, tile);
@@ -316,22 +323,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         if (lane == 0) mbar_arrive_cluster(acce_c + 8 * a);
         continue;
       }
+      // 64-column chunks: TMEM -> registers -> bf16 -> swizzled staging rows (one
+      // row per lane, conflict-free) -> one TMA store of 32 rows x 64 columns
       const GemmSeg& sg = p.seg[t.seg];
-      const int grow = t.m0 + (int)rank * 128 + row;
-      __nv_bfloat16* dst_row = grow < p.rows ? sg.C + (size_t)grow * sg.ldc + sg.c_col0 + t.n0 : nullptr;
+      const int wrow0 = t.m0 + (int)rank * 128 + q * 32;  // first row of this warp
       const int ncols = min(t.nvalid, sg.n_cols - t.n0);
       const uint32_t tm = tmem_base + a * kPairBN + (static_cast<uint32_t>(q * 32) << 16);
-      for (int cc = 0; cc < t.nvalid / 32; ++cc) {
-        uint32_t r[32];
-        tmem_ld32(tm + cc * 32, r);
-        if (dst_row != nullptr && cc * 32 < ncols) {
-          uint32_t pk[16];
+      for (int ch = 0; ch < t.nvalid / 64; ++ch) {
+        uint32_t r[64];
+        tmem_ld64(tm + ch * 64, r);
+        if (ch * 64 >= ncols || wrow0 >= p.rows) continue;  // warp-uniform
+        uint8_t* sb = stage_out + (nstore & 1) * L::kOutBytes;
+        // the store issued two chunks ago from this buffer must have read it
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+        const uint32_t rb = smem_u32(sb) + lane * 128;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-          __nv_bfloat16* d = dst_row + cc * 32;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) st_global_v4(d + i * 8, pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(rb + ((c ^ (lane & 7)) << 4), pack_bf16x2(__uint_as_float(r[8 * c]), __uint_as_float(r[8 * c + 1])),
+                       pack_bf16x2(__uint_as_float(r[8 * c + 2]), __uint_as_float(r[8 * c + 3])),
+                       pack_bf16x2(__uint_as_float(r[8 * c + 4]), __uint_as_float(r[8 * c + 5])),
+                       pack_bf16x2(__uint_as_float(r[8 * c + 6]), __uint_as_float(r[8 * c + 7])));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&p.tmC[t.seg], sb, sg.c_col0 + t.n0 + ch * 64, wrow0);
+          bulk_commit();
         }
+        ++nstore;
       }
       tc_fence_before();
       __syncwarp();
@@ -339,6 +358,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     }
   }
 
+  if (warp >= 2 && lane == 0) bulk_wait_all();  // this warp's output stores have landed
   tc_fence_before();
   if (*abort_flag) {
     // copies of either CTA may still be landing on this CTA's buffers

@@ -224,6 +224,7 @@ int dense_params(GemmParams& p, const void* A, long long rows, int K, const Dens
   int nt = 0;
   for (int s = 0; s < nseg; ++s) {
     if (int e = tmap_rows(&p.tmB[s], segs[s].W, K, segs[s].w_cols, segs[s].w_cols, 64)) return e;
+    if (int e = tmap_rows(&p.tmC[s], segs[s].C, rows, segs[s].ldc, segs[s].ldc, 32)) return e;
     p.seg[s].n_cols = segs[s].n_cols;
     p.seg[s].b_col0 = segs[s].b_col0;
     p.seg[s].c_col0 = segs[s].c_col0;
@@ -506,6 +507,7 @@ int do_combine(const gqe_dims* d, const void* O, const float* w, const void* Wo,
     GQE_TRY(tmap_rows(&p.tmA, O, N, Ha * 64, Ha * 64, kGemmBM));
     GQE_TRY(tmap_rows(&p.tmB[0], Wo, KA, d->D, d->D, 64));
     p.seg[0] = GemmSeg{d->D, 0, 0, 0, (long long)d->D, static_cast<__nv_bfloat16*>(y)};
+    GQE_TRY(tmap_rows(&p.tmC[0], y, N, d->D, d->D, 32));
     p.nseg = 1;
     p.ntn = (int)cdiv(d->D, kG2DenseBN);
     p.rows = (int)N;
