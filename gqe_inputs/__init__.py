@@ -111,3 +111,24 @@ def make_x(dims: Dims, seed: int, device: str = "cpu") -> torch.Tensor:
     gen = torch.Generator(device=device)
     gen.manual_seed(seed)
     return _normal(gen, (dims.B * dims.T, dims.D), 1.0, device)
+
+
+def make_decode_inputs(dims: Dims, cache_len, seed: int = 0, device: str = "cpu") -> dict:
+    """One decode step of the layer: weights as ``make_inputs`` (dims.T is the
+    cache capacity), the new tokens x_new [B, D] ~ N(0, 1), and K/V caches
+    [B, T, G, dh] ~ N(0, (0.02*sqrt(D))^2) -- the spread of x Wk for x ~ N(0, 1)
+    and weights ~ N(0, 0.02^2) -- with the rows at and past cache_len[b]
+    zeroed. cache_len ([B] ints, each < T) is returned as an int32 tensor."""
+    d = dims
+    out = make_inputs(Dims(B=d.B, T=1, D=d.D, G=d.G, M=d.M, k=d.k, dh=d.dh, bias0=d.bias0), seed, device)
+    out["x_new"] = out.pop("x")
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed + 7919)
+    std = 0.02 * d.D ** 0.5
+    lens = torch.as_tensor(list(cache_len), dtype=torch.int32)
+    keep = (torch.arange(d.T)[None, :] < lens[:, None]).to(device)[:, :, None, None]
+    for key in ("K_cache", "V_cache"):
+        c = torch.randn((d.B, d.T, d.G, d.dh), generator=gen, device=device, dtype=torch.float32) * std
+        out[key] = (c * keep).to(torch.bfloat16)
+    out["cache_len"] = lens.to(device)
+    return out

@@ -29,7 +29,10 @@ design notes of this repository):
   * one weighted slot per group;
   * shared head attends KV head 0;
   * scale 1/sqrt(dh), causal mask s <= t, no positional encoding or biases;
-  * Wo rows: [concat (g-major, slot j) | slot g | shared].
+  * Wo rows: [concat (g-major, slot j) | slot g | shared];
+  * decode step: the new token of sequence b sits at position cache_len[b],
+    its K/V row is appended there and its queries attend positions
+    0..cache_len[b] (the pages describe no decode procedure).
 
 Layout conventions (match the ones ``gqe_inputs`` draws): x [B*T, D],
 Wq [D, (G*M+1)*dh] with routed head h = g*M + e and the shared head last,
@@ -173,6 +176,28 @@ def _project_kv(X, Wk, Wv, B, T, G, dh):
     return K, V
 
 
+def _project_q_selected(Xr, Wq, sel, dims) -> np.ndarray:
+    """Query rows of the selected experts only ([GS] "query-side sparsity";
+    [AT] section 4: every expert has its own query projection), plus the
+    shared head: Q[r, g*k + j] = x_r Wq[:, head g*M + sel[r, g, j]],
+    Q[r, G*k] = x_r Wq[:, shared]."""
+    G, M, k, dh = dims.G, dims.M, dims.k, dims.dh
+    WQ = _f64(Wq)
+    nr = Xr.shape[0]
+    Q = np.zeros((nr, G * k + 1, dh))
+    for g in range(G):
+        for j in range(k):
+            e_col = sel[:, g, j]
+            for e in range(M):
+                m = e_col == e
+                if not m.any():
+                    continue
+                h = g * M + e
+                Q[m, g * k + j] = Xr[m] @ WQ[:, h * dh:(h + 1) * dh]
+    Q[:, G * k] = Xr @ WQ[:, G * M * dh:(G * M + 1) * dh]
+    return Q
+
+
 def attend_selected(Q, rows, K, V, dims) -> np.ndarray:
     """Attention step of the GQE layer for query rows ``rows`` (flat n).
 
@@ -237,28 +262,55 @@ def gqe_forward(x, Wq, Wk, Wv, Wr, br, Wo, dims, rows=None, forced_sel=None) -> 
     sel, w = R["sel"], R["w"]
 
     K, V = _project_kv(X, Wk, Wv, B, T, G, dh)
-    WQ = _f64(Wq)
-    Xr = X[rows]
-    nr = len(rows)
-    Ha = G * k + 1
-    Q = np.zeros((nr, Ha, dh))
-
-    for g in range(G):
-        for j in range(k):
-            e_col = sel[:, g, j]
-            for e in range(M):
-                m = e_col == e
-                if not m.any():
-                    continue
-                h = g * M + e
-                Q[m, g * k + j] = Xr[m] @ WQ[:, h * dh:(h + 1) * dh]
-    Q[:, G * k] = Xr @ WQ[:, G * M * dh:(G * M + 1) * dh]
+    Q = _project_q_selected(X[rows], Wq, sel, dims)
 
     O = attend_selected(Q, rows, K, V, dims)
     A = combine(O, w, dims)
     y = A @ _f64(Wo)
     return {"rows": rows, "sel": sel, "w": w, "margin": R["margin"], "logits": R["logits"],
             "p": R["p"], "K": K, "V": V, "Q": Q, "O": O, "A": A, "y": y}
+
+
+# ---------------------------------------------------------------------------
+# One generation step with a key/value cache. [WK], "from the inference
+# angle": a decoder caches the key/value heads and reads them back at every
+# step, which is where sharing K/V heads pays. Reading (the pages describe no
+# decode procedure): the new token of sequence b sits at position L_b =
+# cache_len[b]; its K/V row is appended there and each of its query rows
+# attends positions 0..L_b; routing, projections and the output construction
+# are those of the layer above applied to that one token.
+# ---------------------------------------------------------------------------
+def gqe_decode(x_new, Wq, Wk, Wv, Wr, br, Wo, K_cache, V_cache, cache_len, dims, forced_sel=None) -> dict:
+    """x_new [B, D]: the token at position cache_len[b] of sequence b.
+    K_cache, V_cache [B, Tmax, G, dh]: rows < cache_len[b] of sequence b are
+    its keys/values; the rest is ignored. Returns y [B, D], the new token's
+    K/V rows K_new, V_new [B, G, dh] (the rows the step appends), and the
+    routing and intermediate values (float64)."""
+    B, D, G, M, k, dh = dims.B, dims.D, dims.G, dims.M, dims.k, dims.dh
+    X = _f64(x_new).reshape(B, D)
+    lens = np.asarray(cache_len, dtype=np.int64).reshape(B)
+    R = route(X, Wr, br, G, M, k, forced_sel=forced_sel)
+    sel, w = R["sel"], R["w"]
+    K_new = (X @ _f64(Wk)).reshape(B, G, dh)
+    V_new = (X @ _f64(Wv)).reshape(B, G, dh)
+    Q = _project_q_selected(X, Wq, sel, dims)
+    Kc = _f64(K_cache).reshape(B, -1, G, dh)
+    Vc = _f64(V_cache).reshape(B, -1, G, dh)
+    scale = 1.0 / math.sqrt(dh)
+    O = np.zeros(Q.shape)
+    for b in range(B):
+        L = int(lens[b])
+        for g in range(G):
+            Kb = np.concatenate([Kc[b, :L, g], K_new[b, g][None]], axis=0)
+            Vb = np.concatenate([Vc[b, :L, g], V_new[b, g][None]], axis=0)
+            pos = np.full(k, L)
+            O[b, g * k:(g + 1) * k] = causal_attention(Q[b, g * k:(g + 1) * k], pos, Kb, Vb, scale)
+        Kb = np.concatenate([Kc[b, :L, 0], K_new[b, 0][None]], axis=0)
+        Vb = np.concatenate([Vc[b, :L, 0], V_new[b, 0][None]], axis=0)
+        O[b, G * k] = causal_attention(Q[b, G * k][None], np.array([L]), Kb, Vb, scale)[0]
+    A = combine(O, w, dims)
+    y = A @ _f64(Wo)
+    return {"sel": sel, "w": w, "margin": R["margin"], "K_new": K_new, "V_new": V_new, "Q": Q, "O": O, "A": A, "y": y}
 
 
 def gqa_dense_forward(x, Wq, Wk, Wv, Wo_dense, dims, rows=None) -> dict:

@@ -371,3 +371,71 @@ def test_planted_wrong_softmax_scale_is_caught():
         *(torch.from_numpy(a)[None, None] for a in (Q, K, V)), is_causal=True)[0, 0].numpy()
     np.testing.assert_allclose(good, Ot, atol=1e-12)
     assert not np.allclose(bad, Ot, atol=1e-6)
+
+
+# ---------------------------------------------------------------------------
+# Decode step with a key/value cache
+# ---------------------------------------------------------------------------
+def _decode_from_forward(d, inp, lens, garbage_seed=None):
+    """Inputs of one decode step built from a full forward run: the cache of
+    sequence b holds the forward's K/V at positions < lens[b] (garbage past
+    them when garbage_seed is given) and the new token is x at lens[b]."""
+    full = _fwd(d, inp)
+    X = inp["x"].reshape(d.B, d.T, d.D)
+    x_new = torch.stack([X[b, lens[b]] for b in range(d.B)])
+    K = full["K"].copy()
+    V = full["V"].copy()
+    if garbage_seed is not None:
+        rng = np.random.default_rng(garbage_seed)
+        for b in range(d.B):
+            K[b, lens[b]:] = rng.normal(size=K[b, lens[b]:].shape) * 5
+            V[b, lens[b]:] = rng.normal(size=V[b, lens[b]:].shape) * 5
+    return full, x_new, K, V
+
+
+def _dec(d, inp, x_new, K, V, lens, **kw):
+    return ref.gqe_decode(x_new, inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"], inp["Wo"], K, V, lens, d, **kw)
+
+
+@pytest.mark.parametrize("G,M,k", [(2, 2, 1), (2, 3, 2), (1, 4, 4)])
+def test_decode_equals_forward_at_the_last_position(G, M, k):
+    d, inp = _small(B=3, T=40, G=G, M=M, k=k)
+    lens = [39, 17, 0]
+    full, x_new, K, V = _decode_from_forward(d, inp, lens, garbage_seed=5)
+    out = _dec(d, inp, x_new, K, V, lens)
+    rows = np.array([b * d.T + lens[b] for b in range(d.B)])
+    np.testing.assert_allclose(out["y"], full["y"][rows], rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(out["sel"], full["sel"][rows])
+    np.testing.assert_allclose(out["w"], full["w"][rows], rtol=0, atol=1e-14)
+    for b in range(d.B):
+        np.testing.assert_allclose(out["K_new"][b], full["K"][b, lens[b]], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(out["V_new"][b], full["V"][b, lens[b]], rtol=0, atol=1e-13)
+
+
+def test_decode_with_an_empty_cache_returns_the_new_value():
+    d, inp = _small(B=2, T=4, G=2, M=2, k=1)
+    X = inp["x"].double().numpy()[:d.B]
+    K = np.zeros((d.B, d.T, d.G, d.dh))
+    out = _dec(d, inp, inp["x"][:d.B], K, K, [0, 0])
+    Vn = (X @ inp["Wv"].double().numpy()).reshape(d.B, d.G, d.dh)
+    for b in range(d.B):
+        for g in range(d.G):
+            np.testing.assert_allclose(out["O"][b, g], Vn[b, g], rtol=0, atol=1e-14)
+        np.testing.assert_allclose(out["O"][b, d.G], Vn[b, 0], rtol=0, atol=1e-14)
+    A = np.concatenate([Vn.reshape(d.B, -1), Vn.reshape(d.B, -1), Vn[:, 0]], axis=1)
+    np.testing.assert_allclose(out["y"], A @ inp["Wo"].double().numpy(), rtol=0, atol=1e-13)
+
+
+def test_decode_reads_exactly_the_first_cache_len_rows():
+    d, inp = _small(B=2, T=30, G=2, M=3, k=2)
+    lens = [12, 29]
+    _, x_new, K, V = _decode_from_forward(d, inp, lens)
+    base = _dec(d, inp, x_new, K, V, lens)["y"]
+    K2, V2 = K.copy(), V.copy()
+    K2[0, 12:] += 3.0
+    V2[0, 12:] -= 3.0
+    np.testing.assert_array_equal(_dec(d, inp, x_new, K2, V2, lens)["y"], base)
+    K3 = K.copy()
+    K3[0, 11, 0] += 1.0
+    assert not np.allclose(_dec(d, inp, x_new, K3, V, lens)["y"][0], base[0])
+    np.testing.assert_array_equal(_dec(d, inp, x_new, K3, V, lens)["y"][1], base[1])
