@@ -71,7 +71,8 @@ enum gqe_op {
   GQE_OP_COMBINE = 4,
   GQE_OP_FORWARD = 5,
   GQE_OP_DENSE = 6,
-  GQE_OP_FORWARD_HOST = 7
+  GQE_OP_FORWARD_HOST = 7,
+  GQE_OP_DECODE = 8
 };
 
 /* Workspace bytes the operation needs for these dims (0 if none); returns 0
@@ -216,6 +217,38 @@ int gqe_forward_host(const gqe_dims* d, const void* x_host, const void* Wq,
                      const void* Wk, const void* Wv, const void* Wr,
                      const float* br, const void* Wo, void* y_host, void* ws,
                      size_t ws_bytes, void* stream);
+
+/*
+ * gqe_decode -- one generation step of the layer against a key/value cache.
+ * Method: the layer of gqe_forward applied to one new token per sequence
+ * (gist.science summary, "Architecture and routing"; animattoys.com
+ * article, section 4); aiboss88.com wiki on grouped-query attention,
+ * inference section: a decoder caches the key/value heads and reads them
+ * back at every step. The pages give no decode procedure; this library's
+ * reading: the new token of sequence b sits at position L_b = cache_len[b],
+ * its K/V row is written there, and each of its query rows (the k selected
+ * experts of every group, the shared head on KV head 0) attends positions
+ * 0..L_b.
+ *
+ * d->B sequences, d->T = cache capacity (positions per sequence).
+ * In : cache_len [B] int32 (device), 0 <= L_b < T; x_new [B, D] bf16;
+ *      Wq, Wk, Wv, Wr, br, Wo as gqe_forward.
+ * In/out: K_cache, V_cache [B, T, G, dh] bf16: rows < L_b are read; row L_b
+ *      of each sequence is overwritten with the new token's K/V; rows past
+ *      L_b are neither read nor written.
+ * Out: y [B, D] bf16; sel [B, G, k] int32 and w [B, G, k] fp32 (the routing
+ *      of the new tokens, as gqe_route).
+ * ws : gqe_workspace_bytes(d, GQE_OP_DECODE).
+ * A cache_len outside [0, T) skips that sequence's cache access and sets the
+ * device check word (gqe_check_error returns GQE_ERR_DEVICE_CHECK). All
+ * pointers are device pointers except d; B <= 65535. Asynchronous on
+ * `stream`; capturable in a CUDA graph (no host synchronisation).
+ */
+int gqe_decode(const gqe_dims* d, const int32_t* cache_len, const void* x_new,
+               const void* Wq, const void* Wk, const void* Wv, const void* Wr,
+               const float* br, const void* Wo, void* K_cache, void* V_cache,
+               void* y, int32_t* sel, float* w, void* ws, size_t ws_bytes,
+               void* stream);
 
 /*
  * gqa_dense_forward -- the all-heads GQA baseline the method is compared with

@@ -312,10 +312,12 @@ __global__ void __launch_bounds__(kA2Threads, 1) attn2_fwd_kernel(const __grid_c
             if (!(ok = mbar_wait(&k_full[(kvj + 1) % kA2Stages], ((kvj + 1) / kA2Stages) & 1, abort_flag))) break;
             if (!(ok = issue_s(kvj + 1))) break;
           }
-          if (j < n) {
-            if (!(ok = mbar_wait(&v_full[kvj % kA2Stages], (kvj / kA2Stages) & 1, abort_flag))) break;
-            if (!(ok = issue_pv(kvj, j > 0))) break;
-          }
+          // A block this tile does not use (j >= n) is released only after it
+          // has arrived: an earlier release could complete the stage's previous
+          // phase (the other tile still reading the block before it) and let
+          // the producer overwrite that block.
+          if (!(ok = mbar_wait(&v_full[kvj % kA2Stages], (kvj / kA2Stages) & 1, abort_flag))) break;
+          if (j < n && !(ok = issue_pv(kvj, j > 0))) break;
           umma_commit(&kv_empty[kvj % kA2Stages]);  // this thread is done with block j
         }
         umma_commit(&q_empty[qb]);

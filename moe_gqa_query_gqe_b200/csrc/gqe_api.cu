@@ -20,6 +20,7 @@
 #include "attn.cuh"
 #include "attn2.cuh"
 #include "combine.cuh"
+#include "decode.cuh"
 
 using namespace gqe;
 
@@ -541,6 +542,45 @@ int gqe_version(void) { return 100; }
 
 int gqe_validate_dims(const gqe_dims* d) { return check_dims(d); }
 
+// Decode step: the B new tokens as one sequence of B tokens for the prefill
+// kernels (routing, projections, output projection).
+gqe_dims decode_token_dims(const gqe_dims* d) {
+  gqe_dims t = *d;
+  t.B = 1;
+  t.T = d->B;
+  return t;
+}
+
+struct DecodeWs {
+  RouteWs route;
+  float* margin;
+  int32_t *seg_off, *seg_tok;
+  __nv_bfloat16 *Kn, *Vn, *Q, *O, *A;
+  float *part_ml, *part_o;
+  int nsplit, rmax;
+};
+DecodeWs carve_decode(Carver& c, const gqe_dims* d) {
+  const gqe_dims t = decode_token_dims(d);
+  const size_t B = d->B;
+  const int Ha = d->G * d->k + 1;
+  DecodeWs f;
+  f.route = carve_route(c, &t);
+  f.margin = c.take<float>(B * d->G);
+  f.seg_off = c.take<int32_t>((size_t)d->G * d->M + 1);
+  f.seg_tok = c.take<int32_t>(B * d->G * d->k);
+  f.Kn = c.take<__nv_bfloat16>(B * d->G * 64);
+  f.Vn = c.take<__nv_bfloat16>(B * d->G * 64);
+  f.Q = c.take<__nv_bfloat16>(B * Ha * 64);
+  f.O = c.take<__nv_bfloat16>(B * Ha * 64);
+  f.A = d->k == 1 ? nullptr : c.take<__nv_bfloat16>(B * (size_t)(d->G * d->k + d->G + 1) * 64);
+  f.nsplit = (int)cdiv(d->T, kDecChunk);
+  f.rmax = d->k + 1;
+  const size_t parts = B * d->G * f.rmax * (size_t)f.nsplit;
+  f.part_ml = c.take<float>(parts * 2);
+  f.part_o = c.take<float>(parts * 64);
+  return f;
+}
+
 size_t gqe_workspace_bytes(const gqe_dims* d, int op) {
   if (check_dims(d) != GQE_OK) return 0;
   Carver c{nullptr};
@@ -557,6 +597,7 @@ size_t gqe_workspace_bytes(const gqe_dims* d, int op) {
       return c.off;
     }
     case GQE_OP_DENSE: carve_dense(c, d); return c.off;
+    case GQE_OP_DECODE: carve_decode(c, d); return c.off;
     default: return 0;
   }
 }
@@ -647,6 +688,60 @@ int gqe_forward_host(const gqe_dims* d, const void* x_host, const void* Wq, cons
   GQE_TRY(gqe_forward(d, x_dev, Wq, Wk, Wv, Wr, br, Wo, y_dev, ws, ws_bytes, stream));
   GQE_TRY(cuda_status(cudaMemcpyAsync(y_host, y_dev, xbytes, cudaMemcpyDeviceToHost, st)));
   return GQE_OK;
+}
+
+int gqe_decode(const gqe_dims* d, const int32_t* cache_len, const void* x_new, const void* Wq, const void* Wk,
+               const void* Wv, const void* Wr, const float* br, const void* Wo, void* K_cache, void* V_cache, void* y,
+               int32_t* sel, float* w, void* ws, size_t ws_bytes, void* stream) {
+  GQE_TRY(check_dims(d));
+  GQE_TRY(check_ptrs({cache_len, x_new, Wq, Wk, Wv, Wr, Wo, K_cache, V_cache, y, sel, w}));
+  if (br && !aligned16(br)) return GQE_ERR_INVALID_ARG;
+  if (d->B > 65535) return GQE_ERR_UNSUPPORTED;
+  GQE_TRY(check_ws(ws, ws_bytes, gqe_workspace_bytes(d, GQE_OP_DECODE)));
+  GQE_TRY(check_device());
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Carver c{static_cast<uint8_t*>(ws)};
+  DecodeWs f = carve_decode(c, d);
+  const gqe_dims t = decode_token_dims(d);
+  // one pair-GEMM launch over the new tokens: K, V, the shared query and the
+  // router, then the compaction and the selected queries (prefill kernels)
+  DenseSeg segs[3];
+  kv_segments(&t, Wq, Wk, Wv, f.Q, f.Kn, f.Vn, segs);
+  GemmParams p;
+  long long dense_tiles = 0, route_tiles = 0;
+  GQE_TRY(dense_params(p, x_new, d->B, d->D, segs, 3, &dense_tiles));
+  GQE_TRY(add_route_tiles(p, &t, Wr, br, sel, w, f.margin, f.route, dense_tiles, &route_tiles));
+  GQE_TRY(launch_gemm_pair(p, dense_tiles + route_tiles, st));
+  GQE_TRY(route_finish(&t, sel, f.seg_off, f.seg_tok, nullptr, f.route, st));
+  GQE_TRY(do_qgather(&t, x_new, Wq, sel, f.seg_off, f.seg_tok, f.Q, st));
+  // the cache side: append, split-K attention, merge
+  DecodeParams dp;
+  dp.Q = f.Q;
+  dp.Kn = f.Kn;
+  dp.Vn = f.Vn;
+  dp.Kc = static_cast<__nv_bfloat16*>(K_cache);
+  dp.Vc = static_cast<__nv_bfloat16*>(V_cache);
+  dp.cache_len = cache_len;
+  dp.part_ml = f.part_ml;
+  dp.part_o = f.part_o;
+  dp.O = f.O;
+  dp.B = d->B;
+  dp.T = d->T;
+  dp.G = d->G;
+  dp.k = d->k;
+  dp.Ha = d->G * d->k + 1;
+  dp.rmax = f.rmax;
+  dp.nsplit = f.nsplit;
+  dp.scale_log2 = 1.4426950408889634f / sqrtf(64.f);
+  const long long pieces = (long long)d->B * d->G * 64 / 8 * 2;
+  GQE_TRY(launch_pdl(decode_append_kernel, dim3((unsigned)std::min<long long>(cdiv(pieces, 256), 4096)), dim3(256), 0,
+                     st, dp));
+  const int attn_smem = f.rmax * (64 + kDecChunk + 4 * 64) * 4;
+  GQE_TRY(set_smem(decode_attn_kernel, attn_smem));
+  GQE_TRY(launch_pdl(decode_attn_kernel, dim3(f.nsplit, d->G, d->B), dim3(kDecThreads), attn_smem, st, dp));
+  const long long warps = (long long)d->B * dp.Ha;
+  GQE_TRY(launch_pdl(decode_merge_kernel, dim3((unsigned)cdiv(warps * 32, 256)), dim3(256), 0, st, dp));
+  return do_combine(&t, f.O, w, Wo, y, f.A, st);
 }
 
 int gqa_dense_forward(const gqe_dims* d, const void* x, const void* Wq, const void* Wk, const void* Wv,

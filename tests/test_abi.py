@@ -49,6 +49,14 @@ def test_all_workloads_are_supported_and_sized():
         assert gqe.workspace_bytes(d, gqe.OP_FORWARD_HOST) > gqe.workspace_bytes(d, gqe.OP_FORWARD)
         assert gqe.workspace_bytes(d, gqe.OP_DENSE) > 0
         assert gqe.workspace_bytes(d, gqe.OP_QPROJ) == 0
+        assert gqe.workspace_bytes(d, gqe.OP_DECODE) > 0
+
+
+def test_decode_workspace_grows_with_the_cache_capacity():
+    d = Dims(B=4, T=1024, D=256, G=4, M=2, k=1)
+    small = gqe.workspace_bytes(d, gqe.OP_DECODE)
+    assert gqe.workspace_bytes(d.with_(T=32 * 1024), gqe.OP_DECODE) > small
+    assert gqe.workspace_bytes(d.with_(k=2), gqe.OP_DECODE) > small
 
 
 @pytest.mark.parametrize("bad,code", [
@@ -77,6 +85,11 @@ def test_null_and_misaligned_pointers_are_rejected_before_any_launch():
     assert _raw("gqe_route", dp, P, P, None, P, P, None, P, P, None, P, small, None) == -3
     assert _raw("gqe_route", dp, P, P, None, P, P, None, P, P, None, P + 16, 1 << 30, None) == -3  # ws misaligned
     assert _raw("gqa_dense_forward", dp, P, P, P, P, P, None, P, 1 << 30, None) == -1
+    # gqe_decode: null cache_len, misaligned x_new, missing workspace
+    args = [P, P, P, P, P, P, None, P, P, P, P, P, P]
+    assert _raw("gqe_decode", dp, None, *args[1:], P, 1 << 30, None) == -1
+    assert _raw("gqe_decode", dp, P, P + 2, *args[2:], P, 1 << 30, None) == -1
+    assert _raw("gqe_decode", dp, *args, None, 0, None) == -3
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device answer")

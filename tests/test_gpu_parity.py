@@ -142,6 +142,32 @@ def test_repeat_calls_are_deterministic(cases):
     assert torch.equal(y1, y2)
 
 
+def test_repeat_calls_are_bitwise_identical_at_the_main_shape():
+    """Twenty forwards of the main workload (each with a freshly filled
+    workspace) give bit-identical attention outputs and y. This caught a
+    release-order race of the attention's K/V ring: in an item whose two
+    tiles use different numbers of K/V blocks, the shorter tile released a
+    block it never waited for, which could complete the stage's previous
+    phase and let the producer overwrite a block the other tile still read
+    (about one run in six went wrong)."""
+    import moe_gqa_query_gqe_b200 as gqe
+    d = CONFIGS["main_b8_t2048"]
+    dev = to_dev(make_inputs(d, seed=0))
+    first = None
+    for rep in range(20):
+        ws = gqe.workspace(d, gqe.OP_FORWARD)
+        ws.fill_(0x5A if rep % 2 else 0x21)
+        y = torch.empty(d.B * d.T, d.D, dtype=torch.bfloat16, device="cuda")
+        gqe.gqe_forward(d, dev["x"], dev["Wq"], dev["Wk"], dev["Wv"], dev["Wr"], dev["br"], dev["Wo"], y, ws)
+        assert gqe.gqe_check_error() == 0
+        cur = (gqe.forward_views(d, ws)["O"].clone(), y)
+        if first is None:
+            first = cur
+            continue
+        assert torch.equal(cur[0], first[0]), f"attention output differs on repeat {rep}"
+        assert torch.equal(cur[1], first[1]), f"y differs on repeat {rep}"
+
+
 # ---- the workloads at full size: sampled query rows against the oracle ----
 
 def _sampled_parity(d, n_uniform, seed=0, dense=True):
