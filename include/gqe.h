@@ -72,7 +72,17 @@ enum gqe_op {
   GQE_OP_FORWARD = 5,
   GQE_OP_DENSE = 6,
   GQE_OP_FORWARD_HOST = 7,
-  GQE_OP_DECODE = 8
+  GQE_OP_DECODE = 8,
+  GQE_OP_FORWARD_VARIANT = 9
+};
+
+/* Output construction of gqe_forward_variant. */
+enum gqe_combine_mode {
+  GQE_COMBINE_SLOT = 0,     /* GQE: [hard concat | renormalised slot per group | shared] */
+  GQE_COMBINE_HARD = 1,     /* ablation: [hard concat | shared], no slot                 */
+  GQE_COMBINE_WEIGHTED = 2  /* ablation: [concat, each selected output scaled by its
+                               expert's in-group probability (not renormalised) |
+                               shared], no slot                                           */
 };
 
 /* Workspace bytes the operation needs for these dims (0 if none); returns 0
@@ -217,6 +227,27 @@ int gqe_forward_host(const gqe_dims* d, const void* x_host, const void* Wq,
                      const void* Wk, const void* Wv, const void* Wr,
                      const float* br, const void* Wo, void* y_host, void* ws,
                      size_t ws_bytes, void* stream);
+
+/*
+ * gqe_forward_variant -- gqe_forward with the output construction chosen by
+ * `mode` (enum gqe_combine_mode). Method: animattoys.com article, section 6:
+ * besides the full design (hard concatenation, a renormalised weighted slot
+ * and the always-on shared head) the ablation trains a pure hard
+ * concatenation and a concatenation weighted directly by the router's scores
+ * without the renormalised slot. This library's reading: both variants keep
+ * the shared head (the page does not say they drop it), and the "router's
+ * scores" are the in-group softmax probabilities of the selected experts.
+ *
+ * Wo: [(G*k + G + 1)*dh, D] for GQE_COMBINE_SLOT (identical to gqe_forward),
+ *     [(G*k + 1)*dh, D] for the two variants (rows: concat g-major, slot j;
+ *     then the shared head).
+ * ws: gqe_workspace_bytes(d, GQE_OP_FORWARD_VARIANT). An unknown mode returns
+ * GQE_ERR_INVALID_ARG. Everything else as gqe_forward.
+ */
+int gqe_forward_variant(const gqe_dims* d, int mode, const void* x, const void* Wq,
+                        const void* Wk, const void* Wv, const void* Wr,
+                        const float* br, const void* Wo, void* y, void* ws,
+                        size_t ws_bytes, void* stream);
 
 /*
  * gqe_decode -- one generation step of the layer against a key/value cache.

@@ -20,10 +20,11 @@ namespace gqe {
 
 struct CombineParams {
   const __nv_bfloat16* O;  // [N, Ha, 64]
-  const float* w;          // [N, G, k]
-  __nv_bfloat16* A;        // [N, (G*k + G + 1) * 64]
+  const float* w;          // [N, G, k]: renormalised weights (slot) or in-group probabilities (weighted)
+  __nv_bfloat16* A;        // [N, (G*k + G + 1) * 64] (slot) or [N, (G*k + 1) * 64] (weighted)
   long long N;
   int G, k;
+  int weighted;            // 1: A = [w-scaled concat | shared], no slot
 };
 
 __global__ void __launch_bounds__(256) combine_build_kernel(const CombineParams p) {
@@ -33,16 +34,25 @@ __global__ void __launch_bounds__(256) combine_build_kernel(const CombineParams 
   const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
   const int Ha = p.G * p.k + 1;
-  const int KA = (p.G * p.k + p.G + 1) * 64;
+  const int KA = (p.G * p.k + (p.weighted ? 0 : p.G) + 1) * 64;
   const int n_concat = p.G * p.k * 8;  // 16-byte chunks
-  const int n_slot = p.G * 8;
+  const int n_slot = p.weighted ? 0 : p.G * 8;
   const int n_all = KA / 8;
   for (long long n = warp0; n < p.N; n += nwarps) {
     const uint4* orow = reinterpret_cast<const uint4*>(p.O + (size_t)n * Ha * 64);
     uint4* arow = reinterpret_cast<uint4*>(p.A + (size_t)n * KA);
     for (int c = lane; c < n_all; c += 32) {
       uint4 v;
-      if (c < n_concat) {
+      if (c < n_concat && p.weighted) {
+        // weighted concatenation: slot (g, j) scaled by its in-group probability
+        const float wj = p.w[(size_t)n * p.G * p.k + (c >> 3)];
+        const uint4 o = orow[c];
+        const uint32_t ou[4] = {o.x, o.y, o.z, o.w};
+        uint32_t r4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) r4[i] = pack_bf16x2(wj * bf16lo_to_f32(ou[i]), wj * bf16hi_to_f32(ou[i]));
+        v = make_uint4(r4[0], r4[1], r4[2], r4[3]);
+      } else if (c < n_concat) {
         v = orow[c];
       } else if (c < n_concat + n_slot) {
         const int g = (c - n_concat) >> 3, d8 = (c - n_concat) & 7;

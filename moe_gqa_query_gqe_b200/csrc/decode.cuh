@@ -101,31 +101,46 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecodePa
   }
   __syncthreads();
 
-  // scores: one key per thread per pass
+  // scores: each thread takes two keys per pass (both rows' loads in flight
+  // before the math), kDecThreads * 2 keys per pass over the chunk
   float mloc[9];
 #pragma unroll
   for (int r = 0; r < 9; ++r) mloc[r] = -INFINITY;
-  for (int i = k0 + tid; i < k1; i += kDecThreads) {
-    const uint4* kp = reinterpret_cast<const uint4*>(p.Kc + (((size_t)b * p.T + i) * p.G + g) * 64);
-    float kv[64];
+  for (int i0 = k0 + tid; i0 < k1; i0 += 2 * kDecThreads) {
+    const int i1 = i0 + kDecThreads;
+    uint4 u[2][8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const uint4 u = kp[c];
-      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+    for (int h = 0; h < 2; ++h) {
+      const int i = h ? i1 : i0;
+      if (i < k1) {
+        const uint4* kp = reinterpret_cast<const uint4*>(p.Kc + (((size_t)b * p.T + i) * p.G + g) * 64);
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        kv[c * 8 + 2 * h] = bf16lo_to_f32(w4[h]);
-        kv[c * 8 + 2 * h + 1] = bf16hi_to_f32(w4[h]);
+        for (int c = 0; c < 8; ++c) u[h][c] = kp[c];
       }
     }
 #pragma unroll
-    for (int r = 0; r < 9; ++r) {
-      if (r >= R) break;
-      float acc = 0.f;
+    for (int h = 0; h < 2; ++h) {
+      const int i = h ? i1 : i0;
+      if (i >= k1) break;
+      float kv[64];
 #pragma unroll
-      for (int d = 0; d < 64; ++d) acc = fmaf(q[r * 64 + d], kv[d], acc);
-      sc[r * kDecChunk + (i - k0)] = acc;
-      mloc[r] = fmaxf(mloc[r], acc);
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t w4[4] = {u[h][c].x, u[h][c].y, u[h][c].z, u[h][c].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          kv[c * 8 + 2 * e] = bf16lo_to_f32(w4[e]);
+          kv[c * 8 + 2 * e + 1] = bf16hi_to_f32(w4[e]);
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < 9; ++r) {
+        if (r >= R) break;
+        float acc = 0.f;
+#pragma unroll
+        for (int d = 0; d < 64; ++d) acc = fmaf(q[r * 64 + d], kv[d], acc);
+        sc[r * kDecChunk + (i - k0)] = acc;
+        mloc[r] = fmaxf(mloc[r], acc);
+      }
     }
   }
   // chunk max per row
@@ -178,15 +193,25 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecodePa
   float o0[9], o1[9];
 #pragma unroll
   for (int r = 0; r < 9; ++r) o0[r] = o1[r] = 0.f;
-  for (int i = k0 + warp; i < k1; i += 4) {
-    const uint32_t v2 = reinterpret_cast<const uint32_t*>(p.Vc + (((size_t)b * p.T + i) * p.G + g) * 64)[lane];
-    const float v0 = bf16lo_to_f32(v2), v1 = bf16hi_to_f32(v2);
+  for (int i0 = k0 + warp; i0 < k1; i0 += 4 * 8) {
+    uint32_t v2[8];
 #pragma unroll
-    for (int r = 0; r < 9; ++r) {
-      if (r >= R) break;
-      const float pr = sc[r * kDecChunk + (i - k0)];
-      o0[r] = fmaf(pr, v0, o0[r]);
-      o1[r] = fmaf(pr, v1, o1[r]);
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + 4 * u;
+      v2[u] = i < k1 ? reinterpret_cast<const uint32_t*>(p.Vc + (((size_t)b * p.T + i) * p.G + g) * 64)[lane] : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + 4 * u;
+      if (i >= k1) break;
+      const float v0 = bf16lo_to_f32(v2[u]), v1 = bf16hi_to_f32(v2[u]);
+#pragma unroll
+      for (int r = 0; r < 9; ++r) {
+        if (r >= R) break;
+        const float pr = sc[r * kDecChunk + (i - k0)];
+        o0[r] = fmaf(pr, v0, o0[r]);
+        o1[r] = fmaf(pr, v1, o1[r]);
+      }
     }
   }
 #pragma unroll

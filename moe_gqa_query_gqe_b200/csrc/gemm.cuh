@@ -50,6 +50,7 @@ struct GemmParams {
   int32_t* r_sel;      // [B*T, G, k]: expert | rank in the chunk << 8 (see route.cuh)
   float* r_w;          // [B*T, G, k]
   float* r_margin;     // [B*T, G] or null
+  float* r_p;          // [B*T, G, k] in-group probabilities of the selected experts, or null
   int32_t* r_counts;   // [B][nch][G*M]
   int r_B, r_T, r_nch;
   // A column remap for the k = 1 combine: A = [O_routed | O_routed | O_shared]

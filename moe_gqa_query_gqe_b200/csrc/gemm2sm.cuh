@@ -134,7 +134,8 @@ __device__ void pair_route_epilogue(const GemmParams& p, uint32_t tm, int b, int
 #pragma unroll
         for (int e = 0; e < RM; ++e) l[e] += p.r_br ? p.r_br[g * RM + e] : 0.f;
         const size_t o = (n * G + g) * k;
-        chosen[gi] = route_decide<RM>(l, k, valid, p.r_sel + o, p.r_w + o, p.r_margin ? p.r_margin + n * G + g : nullptr);
+        chosen[gi] = route_decide<RM>(l, k, valid, p.r_sel + o, p.r_w + o, p.r_margin ? p.r_margin + n * G + g : nullptr,
+                                      p.r_p ? p.r_p + o : nullptr);
         if (valid)
 #pragma unroll
           for (int e = 0; e < RM; ++e)

@@ -517,11 +517,27 @@ int do_combine(const gqe_dims* d, const void* O, const float* w, const void* Wo,
     p.r_tile0 = 0x7fffffff;
     return launch_gemm_pair(p, cdiv(N, kPairBM) * p.ntn, st);
   }
-  CombineParams cp{static_cast<const __nv_bfloat16*>(O), w, A, N, d->G, d->k};
+  CombineParams cp{static_cast<const __nv_bfloat16*>(O), w, A, N, d->G, d->k, 0};
   const long long warps = N;
   const long long blocks = std::min<long long>(cdiv(warps * 32, 256), 148ll * 16);
   GQE_TRY(launch_pdl(combine_build_kernel, dim3((unsigned)blocks), dim3(256), 0, st, cp));
   const DenseSeg seg = {Wo, d->D, 0, d->D, y, (long long)d->D, 0};
+  return gemm_dense(A, N, KA, &seg, 1, st);
+}
+
+// Output construction of the ablation variants (no slot): A = [concat |
+// shared] with the concatenated outputs as they are (hard) or each scaled by
+// its expert's in-group probability (weighted); y = A Wo with Wo of
+// (G*k + 1)*64 rows. The hard variant's A is O itself.
+int do_combine_variant(const gqe_dims* d, int mode, const void* O, const float* p_sel, const void* Wo, void* y,
+                       __nv_bfloat16* A, cudaStream_t st) {
+  const long long N = (long long)d->B * d->T;
+  const int KA = (d->G * d->k + 1) * 64;
+  const DenseSeg seg = {Wo, d->D, 0, d->D, y, (long long)d->D, 0};
+  if (mode == GQE_COMBINE_HARD) return gemm_dense(O, N, KA, &seg, 1, st);
+  CombineParams cp{static_cast<const __nv_bfloat16*>(O), p_sel, A, N, d->G, d->k, 1};
+  const long long blocks = std::min<long long>(cdiv(N * 32, 256), 148ll * 16);
+  GQE_TRY(launch_pdl(combine_build_kernel, dim3((unsigned)blocks), dim3(256), 0, st, cp));
   return gemm_dense(A, N, KA, &seg, 1, st);
 }
 
@@ -598,6 +614,13 @@ size_t gqe_workspace_bytes(const gqe_dims* d, int op) {
     }
     case GQE_OP_DENSE: carve_dense(c, d); return c.off;
     case GQE_OP_DECODE: carve_decode(c, d); return c.off;
+    case GQE_OP_FORWARD_VARIANT: {
+      carve_forward(c, d);
+      const size_t N = (size_t)d->B * d->T;
+      c.take<float>(N * d->G * d->k);                                      // probabilities
+      c.take<__nv_bfloat16>(N * (size_t)(d->G * d->k + 1) * 64);            // variant A
+      return c.off;
+    }
     default: return 0;
   }
 }
@@ -647,16 +670,19 @@ int gqe_combine(const gqe_dims* d, const void* O, const float* w, const void* Wo
   return do_combine(d, O, w, Wo, y, static_cast<__nv_bfloat16*>(ws), static_cast<cudaStream_t>(stream));
 }
 
-int gqe_forward(const gqe_dims* d, const void* x, const void* Wq, const void* Wk, const void* Wv, const void* Wr,
-                const float* br, const void* Wo, void* y, void* ws, size_t ws_bytes, void* stream) {
-  GQE_TRY(check_dims(d));
-  GQE_TRY(check_ptrs({x, Wq, Wk, Wv, Wr, Wo, y}));
-  if (br && !aligned16(br)) return GQE_ERR_INVALID_ARG;
-  GQE_TRY(check_ws(ws, ws_bytes, gqe_workspace_bytes(d, GQE_OP_FORWARD)));
-  GQE_TRY(check_device());
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+// The layer: mode GQE_COMBINE_SLOT is the GQE output construction; the other
+// modes are the ablation variants (see gqe_forward_variant).
+int do_forward(const gqe_dims* d, int mode, const void* x, const void* Wq, const void* Wk, const void* Wv,
+               const void* Wr, const float* br, const void* Wo, void* y, void* ws, cudaStream_t st) {
   Carver c{static_cast<uint8_t*>(ws)};
   FwdWs f = carve_forward(c, d);
+  const size_t N = (size_t)d->B * d->T;
+  float* p_sel = nullptr;
+  __nv_bfloat16* A2 = nullptr;
+  if (mode != GQE_COMBINE_SLOT) {
+    p_sel = c.take<float>(N * d->G * d->k);
+    A2 = c.take<__nv_bfloat16>(N * (size_t)(d->G * d->k + 1) * 64);
+  }
   // one pair-GEMM launch over x: K, V, the shared head's query and the router
   // (logits and decisions), then the compaction and the selected queries
   DenseSeg segs[3];
@@ -665,11 +691,36 @@ int gqe_forward(const gqe_dims* d, const void* x, const void* Wq, const void* Wk
   long long dense_tiles = 0, route_tiles = 0;
   GQE_TRY(dense_params(p, x, (long long)d->B * d->T, d->D, segs, 3, &dense_tiles));
   GQE_TRY(add_route_tiles(p, d, Wr, br, f.sel, f.w, f.margin, f.route, dense_tiles, &route_tiles));
+  p.r_p = mode == GQE_COMBINE_WEIGHTED ? p_sel : nullptr;
   GQE_TRY(launch_gemm_pair(p, dense_tiles + route_tiles, st));
   GQE_TRY(route_finish(d, f.sel, f.seg_off, f.seg_tok, f.row_map, f.route, st));
   GQE_TRY(do_qgather(d, x, Wq, f.sel, f.seg_off, f.seg_tok, f.Q, st));
   GQE_TRY(do_attn2(d, f.Q, d->G * d->k + 1, f.K, f.V, f.O, false, st));
-  return do_combine(d, f.O, f.w, Wo, y, f.A, st);
+  if (mode == GQE_COMBINE_SLOT) return do_combine(d, f.O, f.w, Wo, y, f.A, st);
+  return do_combine_variant(d, mode, f.O, p_sel, Wo, y, A2, st);
+}
+
+int gqe_forward(const gqe_dims* d, const void* x, const void* Wq, const void* Wk, const void* Wv, const void* Wr,
+                const float* br, const void* Wo, void* y, void* ws, size_t ws_bytes, void* stream) {
+  GQE_TRY(check_dims(d));
+  GQE_TRY(check_ptrs({x, Wq, Wk, Wv, Wr, Wo, y}));
+  if (br && !aligned16(br)) return GQE_ERR_INVALID_ARG;
+  GQE_TRY(check_ws(ws, ws_bytes, gqe_workspace_bytes(d, GQE_OP_FORWARD)));
+  GQE_TRY(check_device());
+  return do_forward(d, GQE_COMBINE_SLOT, x, Wq, Wk, Wv, Wr, br, Wo, y, ws, static_cast<cudaStream_t>(stream));
+}
+
+int gqe_forward_variant(const gqe_dims* d, int mode, const void* x, const void* Wq, const void* Wk, const void* Wv,
+                        const void* Wr, const float* br, const void* Wo, void* y, void* ws, size_t ws_bytes,
+                        void* stream) {
+  GQE_TRY(check_dims(d));
+  if (mode != GQE_COMBINE_SLOT && mode != GQE_COMBINE_HARD && mode != GQE_COMBINE_WEIGHTED)
+    return GQE_ERR_INVALID_ARG;
+  GQE_TRY(check_ptrs({x, Wq, Wk, Wv, Wr, Wo, y}));
+  if (br && !aligned16(br)) return GQE_ERR_INVALID_ARG;
+  GQE_TRY(check_ws(ws, ws_bytes, gqe_workspace_bytes(d, GQE_OP_FORWARD_VARIANT)));
+  GQE_TRY(check_device());
+  return do_forward(d, mode, x, Wq, Wk, Wv, Wr, br, Wo, y, ws, static_cast<cudaStream_t>(stream));
 }
 
 int gqe_forward_host(const gqe_dims* d, const void* x_host, const void* Wq, const void* Wk, const void* Wv,

@@ -18,11 +18,13 @@ GQE_OK = 0
 STATUS = {0: "GQE_OK", -1: "GQE_ERR_INVALID_ARG", -2: "GQE_ERR_UNSUPPORTED", -3: "GQE_ERR_WORKSPACE",
           -4: "GQE_ERR_CUDA", -5: "GQE_ERR_TIMEOUT", -6: "GQE_ERR_NO_DEVICE",
           -7: "GQE_ERR_DEVICE_CHECK"}
-OP_ROUTE, OP_QPROJ, OP_ATTN, OP_COMBINE, OP_FORWARD, OP_DENSE, OP_FORWARD_HOST, OP_DECODE = 1, 2, 3, 4, 5, 6, 7, 8
+OP_ROUTE, OP_QPROJ, OP_ATTN, OP_COMBINE, OP_FORWARD, OP_DENSE, OP_FORWARD_HOST, OP_DECODE, OP_FORWARD_VARIANT = \
+    1, 2, 3, 4, 5, 6, 7, 8, 9
+COMBINE_SLOT, COMBINE_HARD, COMBINE_WEIGHTED = 0, 1, 2
 
 # every symbol include/gqe.h declares
 EXPORTS = ("gqe_workspace_bytes", "gqe_validate_dims", "gqe_route", "gqe_route_noalloc", "gqe_qproj", "gqe_attn", "gqe_combine",
-           "gqe_forward", "gqe_forward_host", "gqe_decode", "gqa_dense_forward", "gqe_check_error", "gqe_status_string", "gqe_last_cuda_error",
+           "gqe_forward", "gqe_forward_variant", "gqe_forward_host", "gqe_decode", "gqa_dense_forward", "gqe_check_error", "gqe_status_string", "gqe_last_cuda_error",
            "gqe_version")
 
 
@@ -59,6 +61,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "gqe_combine": (ctypes.c_int, [dp, vp, f32p, vp, vp, vp, sz, vp]),
         "gqe_forward": (ctypes.c_int, [dp, vp, vp, vp, vp, vp, f32p, vp, vp, vp, sz, vp]),
         "gqe_decode": (ctypes.c_int, [dp, i32p, vp, vp, vp, vp, vp, f32p, vp, vp, vp, vp, i32p, f32p, vp, sz, vp]),
+        "gqe_forward_variant": (ctypes.c_int, [dp, ctypes.c_int, vp, vp, vp, vp, vp, f32p, vp, vp, vp, sz, vp]),
         "gqe_forward_host": (ctypes.c_int, [dp, vp, vp, vp, vp, vp, f32p, vp, vp, vp, sz, vp]),
         "gqa_dense_forward": (ctypes.c_int, [dp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "gqe_check_error": (ctypes.c_int, [vp]),
@@ -150,6 +153,13 @@ def gqe_combine(dims, O, w, Wo, y, ws, stream=None) -> None:
 def gqe_forward(dims, x, Wq, Wk, Wv, Wr, br, Wo, y, ws, stream=None) -> None:
     _call("gqe_forward", ctypes.byref(dims_struct(dims)), _ptr(x), _ptr(Wq), _ptr(Wk), _ptr(Wv), _ptr(Wr),
           _ptr(br), _ptr(Wo), _ptr(y), _ptr(ws), ws.numel(), _stream(stream))
+
+
+def gqe_forward_variant(dims, mode, x, Wq, Wk, Wv, Wr, br, Wo, y, ws, stream=None) -> None:
+    """gqe_forward with the output construction `mode` (COMBINE_SLOT, _HARD,
+    _WEIGHTED); the variants' Wo has (G*k + 1)*64 rows."""
+    _call("gqe_forward_variant", ctypes.byref(dims_struct(dims)), int(mode), _ptr(x), _ptr(Wq), _ptr(Wk), _ptr(Wv),
+          _ptr(Wr), _ptr(br), _ptr(Wo), _ptr(y), _ptr(ws), ws.numel(), _stream(stream))
 
 
 def gqe_decode(dims, cache_len, x_new, Wq, Wk, Wv, Wr, br, Wo, K_cache, V_cache, y, sel, w, ws, stream=None) -> None:

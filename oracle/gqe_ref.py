@@ -30,6 +30,9 @@ design notes of this repository):
   * shared head attends KV head 0;
   * scale 1/sqrt(dh), causal mask s <= t, no positional encoding or biases;
   * Wo rows: [concat (g-major, slot j) | slot g | shared];
+  * ablation variants ([AT] section 6): the hard and the weighted
+    concatenation keep the shared head; the weights of the weighted one are
+    the in-group probabilities of the selected experts (not renormalised);
   * decode step: the new token of sequence b sits at position cache_len[b],
     its K/V row is appended there and its queries attend positions
     0..cache_len[b] (the pages describe no decode procedure).
@@ -238,10 +241,29 @@ def combine(O, w, dims) -> np.ndarray:
     return np.concatenate([concat, slot, O[:, G * k]], axis=1)
 
 
+def combine_variant(O, p_sel, dims, mode: str) -> np.ndarray:
+    """Output construction of the ablation variants ([AT] section 6: a pure
+    hard concatenation, and a concatenation weighted directly by the router's
+    scores without the renormalised slot). Readings: both keep the shared
+    head; the scores are the in-group softmax probabilities of the selected
+    experts (not renormalised over the selected set).
+      mode "hard":     A = [concat | shared]
+      mode "weighted": A = [p_sel[g, j] * O[g, j] (concat) | shared]"""
+    G, k, dh = dims.G, dims.k, dims.dh
+    O = np.asarray(O, F64)
+    nr = O.shape[0]
+    routed = O[:, :G * k]
+    if mode == "weighted":
+        routed = routed * np.asarray(p_sel, F64).reshape(nr, G * k)[:, :, None]
+    elif mode != "hard":
+        raise ValueError(mode)
+    return np.concatenate([routed.reshape(nr, G * k * dh), O[:, G * k]], axis=1)
+
+
 # ---------------------------------------------------------------------------
 # GQE layer forward: [GS] "Architecture and routing", [AT] section 4.
 # ---------------------------------------------------------------------------
-def gqe_forward(x, Wq, Wk, Wv, Wr, br, Wo, dims, rows=None, forced_sel=None) -> dict:
+def gqe_forward(x, Wq, Wk, Wv, Wr, br, Wo, dims, rows=None, forced_sel=None, combine_mode: str = "slot") -> dict:
     """The whole layer for the query tokens ``rows`` (flat n = b*T + t).
 
     Steps, in the pages' order:
@@ -254,6 +276,8 @@ def gqe_forward(x, Wq, Wk, Wv, Wr, br, Wo, dims, rows=None, forced_sel=None) -> 
          shared head];  6. y = A Wo.
     Returns the intermediate values too (all float64, rows in ``rows`` order).
     ``forced_sel`` ([len(rows), G, k]) overrides the router's choice.
+    ``combine_mode`` "hard" / "weighted" selects an ablation variant of step 5
+    (``combine_variant``; Wo then has (G*k + 1)*dh rows).
     """
     B, T, D, G, M, k, dh = dims.B, dims.T, dims.D, dims.G, dims.M, dims.k, dims.dh
     X = _f64(x).reshape(B * T, D)
@@ -265,9 +289,10 @@ def gqe_forward(x, Wq, Wk, Wv, Wr, br, Wo, dims, rows=None, forced_sel=None) -> 
     Q = _project_q_selected(X[rows], Wq, sel, dims)
 
     O = attend_selected(Q, rows, K, V, dims)
-    A = combine(O, w, dims)
+    p_sel = np.take_along_axis(R["p"], sel, axis=2)
+    A = combine(O, w, dims) if combine_mode == "slot" else combine_variant(O, p_sel, dims, combine_mode)
     y = A @ _f64(Wo)
-    return {"rows": rows, "sel": sel, "w": w, "margin": R["margin"], "logits": R["logits"],
+    return {"rows": rows, "sel": sel, "w": w, "p_sel": p_sel, "margin": R["margin"], "logits": R["logits"],
             "p": R["p"], "K": K, "V": V, "Q": Q, "O": O, "A": A, "y": y}
 
 

@@ -50,6 +50,7 @@ def test_all_workloads_are_supported_and_sized():
         assert gqe.workspace_bytes(d, gqe.OP_DENSE) > 0
         assert gqe.workspace_bytes(d, gqe.OP_QPROJ) == 0
         assert gqe.workspace_bytes(d, gqe.OP_DECODE) > 0
+        assert gqe.workspace_bytes(d, gqe.OP_FORWARD_VARIANT) > gqe.workspace_bytes(d, gqe.OP_FORWARD)
 
 
 def test_decode_workspace_grows_with_the_cache_capacity():
@@ -85,6 +86,10 @@ def test_null_and_misaligned_pointers_are_rejected_before_any_launch():
     assert _raw("gqe_route", dp, P, P, None, P, P, None, P, P, None, P, small, None) == -3
     assert _raw("gqe_route", dp, P, P, None, P, P, None, P, P, None, P + 16, 1 << 30, None) == -3  # ws misaligned
     assert _raw("gqa_dense_forward", dp, P, P, P, P, P, None, P, 1 << 30, None) == -1
+    # gqe_forward_variant: unknown combine mode, then a valid mode without workspace
+    vargs = [P, P, P, P, P, None, P, P]
+    assert _raw("gqe_forward_variant", dp, 7, *vargs, P, 1 << 30, None) == -1
+    assert _raw("gqe_forward_variant", dp, 2, *vargs, None, 0, None) == -3
     # gqe_decode: null cache_len, misaligned x_new, missing workspace
     args = [P, P, P, P, P, P, None, P, P, P, P, P, P]
     assert _raw("gqe_decode", dp, None, *args[1:], P, 1 << 30, None) == -1

@@ -113,6 +113,42 @@ def test_dense_gqa_baseline(cases, name):
     assert_close_bf16(y, want["y"], "dense GQA y vs oracle")
 
 
+VARIANT_CODE = {"slot": 0, "hard": 1, "weighted": 2}
+
+
+def _variant_wo(d, seed=6):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(((d.G * d.k + 1) * 64, d.D), generator=g) * 0.02).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("name", ["tiny_b2_t256", "ragged_b3_t300", "pool4_k2_skewed_t384", "pool8_k4_t136"])
+@pytest.mark.parametrize("mode", ["hard", "weighted"])
+def test_combine_variants(cases, name, mode):
+    """The ablation variants of the output construction (no slot; hard or
+    probability-weighted concatenation) against the oracle's variant."""
+    import moe_gqa_query_gqe_b200 as gqe
+    d, inp, dev, st = cases[name]
+    Wo = _variant_wo(d)
+    ws = gqe.workspace(d, gqe.OP_FORWARD_VARIANT)
+    y = torch.full((d.B * d.T, d.D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    gqe.gqe_forward_variant(d, VARIANT_CODE[mode], dev["x"], dev["Wq"], dev["Wk"], dev["Wv"], dev["Wr"], dev["br"],
+                            Wo.cuda(), y, ws)
+    assert gqe.gqe_check_error() == 0
+    want = ref.gqe_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"], Wo, d,
+                           forced_sel=st["sel"].numpy(), combine_mode=mode)
+    assert_close_bf16(y, want["y"], f"{mode} variant y vs oracle")
+
+
+def test_slot_mode_of_the_variant_entry_is_gqe_forward(cases):
+    import moe_gqa_query_gqe_b200 as gqe
+    d, inp, dev, st = cases["pool4_k2_skewed_t384"]
+    ws = gqe.workspace(d, gqe.OP_FORWARD_VARIANT)
+    y = torch.empty((d.B * d.T, d.D), dtype=torch.bfloat16, device="cuda")
+    gqe.gqe_forward_variant(d, 0, dev["x"], dev["Wq"], dev["Wk"], dev["Wv"], dev["Wr"], dev["br"], dev["Wo"], y, ws)
+    assert gqe.gqe_check_error() == 0
+    assert torch.equal(y.cpu(), st["y"])
+
+
 def test_empty_segments_are_empty(cases):
     d, inp, dev, st = cases["empty_segments_bias20"]
     lens = np.diff(st["seg_off"].numpy()).reshape(d.B, d.G, d.M)

@@ -439,3 +439,56 @@ def test_decode_reads_exactly_the_first_cache_len_rows():
     K3[0, 11, 0] += 1.0
     assert not np.allclose(_dec(d, inp, x_new, K3, V, lens)["y"][0], base[0])
     np.testing.assert_array_equal(_dec(d, inp, x_new, K3, V, lens)["y"][1], base[1])
+
+
+# ---------------------------------------------------------------------------
+# Ablation variants of the output construction
+# ---------------------------------------------------------------------------
+def _variant(d, inp, mode, Wo, **kw):
+    return ref.gqe_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"], Wo, d,
+                           combine_mode=mode, **kw)
+
+
+def _wo_variant(d, seed=4):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(((d.G * d.k + 1) * d.dh, d.D), generator=g) * 0.4).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("G,M,k", [(2, 2, 1), (2, 3, 2)])
+def test_variant_hard_is_the_slot_construction_without_its_slot(G, M, k):
+    d, inp = _small(B=2, T=20, G=G, M=M, k=k)
+    full = _fwd(d, inp)
+    hard = _variant(d, inp, "hard", _wo_variant(d))
+    gk = d.G * d.k * d.dh
+    np.testing.assert_array_equal(hard["A"], np.concatenate([full["A"][:, :gk], full["A"][:, -d.dh:]], axis=1))
+    np.testing.assert_allclose(hard["y"], hard["A"] @ _wo_variant(d).double().numpy(), rtol=0, atol=1e-12)
+
+
+def test_variant_weighted_with_a_single_expert_equals_hard():
+    d, inp = _small(B=2, T=16, G=3, M=1, k=1)
+    Wo = _wo_variant(d)
+    np.testing.assert_allclose(_variant(d, inp, "weighted", Wo)["y"], _variant(d, inp, "hard", Wo)["y"],
+                               rtol=0, atol=1e-14)
+
+
+def test_variant_weighted_scales_by_the_hand_worked_probabilities():
+    """Token 0 of the hand-worked example: group 0 selects expert 0 with
+    in-group probability e/(1+e), group 1 expert 1 with e^2/(1+e^2) (not the
+    renormalised weight 1)."""
+    gold = load("worked_example_k1.txt")
+    d = gold["dims"]
+    inp = _as_inputs(gold)
+    Wo = torch.ones(((d.G * d.k + 1) * d.dh, d.D), dtype=torch.float64)
+    out = _variant(d, inp, "weighted", Wo)
+    p0 = gold["expect.p_t0"]
+    O0 = gold["expect.O"][0]
+    np.testing.assert_allclose(out["A"][0], [p0[0, 0] * O0[0], p0[1, 1] * O0[1], O0[2]], rtol=0, atol=1e-14)
+    assert abs(out["A"][0][0] - O0[0]) > 0.1  # the renormalised weight (1) would give O0[0]
+
+
+def test_planted_renormalised_weights_in_the_weighted_variant_are_caught(monkeypatch):
+    real = ref.combine_variant
+    monkeypatch.setattr(ref, "combine_variant",
+                        lambda O, p_sel, dims, mode: real(O, np.ones_like(p_sel), dims, mode))
+    with pytest.raises(AssertionError):
+        test_variant_weighted_scales_by_the_hand_worked_probabilities()
