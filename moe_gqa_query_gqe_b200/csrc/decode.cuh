@@ -189,19 +189,20 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecodePa
     if (r < R)
       for (int w = 0; w < 4; ++w) l[r] += red[w * p.rmax + r];
   __syncthreads();
-  // P.V: warp w takes keys k0+w, k0+w+4, ...; lane owns dims 2*lane, 2*lane+1
+  // P.V: warp w takes keys k0+w, k0+w+4, ... (32 rows per batch); lane owns
+  // dims 2*lane, 2*lane+1
   float o0[9], o1[9];
 #pragma unroll
   for (int r = 0; r < 9; ++r) o0[r] = o1[r] = 0.f;
-  for (int i0 = k0 + warp; i0 < k1; i0 += 4 * 8) {
-    uint32_t v2[8];
+  for (int i0 = k0 + warp; i0 < k1; i0 += 4 * 32) {
+    uint32_t v2[32];  // 32 V rows per warp in flight
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 32; ++u) {
       const int i = i0 + 4 * u;
       v2[u] = i < k1 ? reinterpret_cast<const uint32_t*>(p.Vc + (((size_t)b * p.T + i) * p.G + g) * 64)[lane] : 0u;
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 32; ++u) {
       const int i = i0 + 4 * u;
       if (i >= k1) break;
       const float v0 = bf16lo_to_f32(v2[u]), v1 = bf16hi_to_f32(v2[u]);

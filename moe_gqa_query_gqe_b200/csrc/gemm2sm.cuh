@@ -111,7 +111,7 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&f)[RM]) {
 // the decision (route.cuh), then a block scan over the chunk of packed 8-bit
 // per-expert flags gives each token its rank in its experts' lists and the
 // chunk's per-expert counts. Groups go eight at a time through s_tot.
-template <int RM>
+template <int RM, bool PR>
 __device__ void pair_route_epilogue(const GemmParams& p, uint32_t tm, int b, int c, int q, int lane,
                                     unsigned long long* s_tot) {
   const int row = q * 32 + lane;
@@ -134,8 +134,8 @@ __device__ void pair_route_epilogue(const GemmParams& p, uint32_t tm, int b, int
 #pragma unroll
         for (int e = 0; e < RM; ++e) l[e] += p.r_br ? p.r_br[g * RM + e] : 0.f;
         const size_t o = (n * G + g) * k;
-        chosen[gi] = route_decide<RM>(l, k, valid, p.r_sel + o, p.r_w + o, p.r_margin ? p.r_margin + n * G + g : nullptr,
-                                      p.r_p ? p.r_p + o : nullptr);
+        chosen[gi] = route_decide<RM, PR>(l, k, valid, p.r_sel + o, p.r_w + o,
+                                          p.r_margin ? p.r_margin + n * G + g : nullptr, PR ? p.r_p + o : nullptr);
         if (valid)
 #pragma unroll
           for (int e = 0; e < RM; ++e)
@@ -312,11 +312,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const uint32_t tm = tmem_base + a * kPairBN + (static_cast<uint32_t>(q * 32) << 16);
         const int c = t.n0 * 2 + (int)rank;  // this CTA's chunk of 128 tokens
         if (c < p.r_nch) {
-          switch (p.M) {
-            case 1: pair_route_epilogue<1>(p, tm, t.rb, c, q, lane, s_tot); break;
-            case 2: pair_route_epilogue<2>(p, tm, t.rb, c, q, lane, s_tot); break;
-            case 4: pair_route_epilogue<4>(p, tm, t.rb, c, q, lane, s_tot); break;
-            default: pair_route_epilogue<8>(p, tm, t.rb, c, q, lane, s_tot); break;
+          if (p.r_p == nullptr) {
+            switch (p.M) {
+              case 1: pair_route_epilogue<1, false>(p, tm, t.rb, c, q, lane, s_tot); break;
+              case 2: pair_route_epilogue<2, false>(p, tm, t.rb, c, q, lane, s_tot); break;
+              case 4: pair_route_epilogue<4, false>(p, tm, t.rb, c, q, lane, s_tot); break;
+              default: pair_route_epilogue<8, false>(p, tm, t.rb, c, q, lane, s_tot); break;
+            }
+          } else {  // the weighted-concatenation variant also writes the probabilities
+            switch (p.M) {
+              case 1: pair_route_epilogue<1, true>(p, tm, t.rb, c, q, lane, s_tot); break;
+              case 2: pair_route_epilogue<2, true>(p, tm, t.rb, c, q, lane, s_tot); break;
+              case 4: pair_route_epilogue<4, true>(p, tm, t.rb, c, q, lane, s_tot); break;
+              default: pair_route_epilogue<8, true>(p, tm, t.rb, c, q, lane, s_tot); break;
+            }
           }
         }
         tc_fence_before();

@@ -44,9 +44,9 @@ struct RouteParams {
 // set); margin = k-th largest minus (k+1)-th largest logit (+inf when k == M).
 // Returns the selected experts as a bit mask; when `out` is true writes
 // sel[.., j] (ascending expert order), w[.., j], the margin and, when `pr` is
-// not null, pr[.., j] = the selected expert's in-group softmax probability
+// PR is set, pr[.., j] = the selected expert's in-group softmax probability
 // over all M experts (not renormalised; the weighted-concatenation variant).
-template <int RM>
+template <int RM, bool PR = false>
 __device__ __forceinline__ uint32_t route_decide(const float (&l)[RM], int k, bool out, int32_t* sel, float* w,
                                                  float* margin, float* pr = nullptr) {
   uint32_t chosen = 0;
@@ -95,7 +95,7 @@ __device__ __forceinline__ uint32_t route_decide(const float (&l)[RM], int k, bo
     // all M experts for the full in-group softmax (mx is also the largest
     // logit overall: the best expert is always selected)
     float inv_all = 0.f;
-    if (pr) {
+    if constexpr (PR) {
       float den_all = 0.f;
 #pragma unroll
       for (int e = 0; e < RM; ++e) den_all += (chosen & (1u << e)) ? ex[e] : expf(l[e] - mx);
@@ -107,7 +107,7 @@ __device__ __forceinline__ uint32_t route_decide(const float (&l)[RM], int k, bo
       if (!(chosen & (1u << e))) continue;
       sel[j] = e;
       w[j] = ex[e] * inv;
-      if (pr) pr[j] = ex[e] * inv_all;
+      if constexpr (PR) pr[j] = ex[e] * inv_all;
       ++j;
     }
     if (margin) *margin = mg;
