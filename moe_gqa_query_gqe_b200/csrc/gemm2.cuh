@@ -5,9 +5,9 @@
 // pairs (gemm2sm.cuh).
 //
 //   A [rows, K] row-major (K-major operand): TMA tiles (dense rows), or rows
-//     gathered by a segment's token list with TMA tile::gather4 (the
-//     selected-expert query projection: only tokens that picked the expert are
-//     multiplied; each lane of the producer warp gathers 4 of the 128 rows).
+//     gathered by a segment's token list with 16-byte cp.async by eight
+//     copier warps (the selected-expert query projection: only tokens that
+//     picked the expert are multiplied).
 //   B [K, N] row-major weight (MN-major operand), 64 x 64 TMA boxes, 128-byte
 //     swizzle. The MMA N of a tile is the segment's remaining width rounded
 //     up to 64 (no work on columns past the segment).
@@ -16,7 +16,7 @@
 //   one tile overlaps the main loop of the next.
 //
 // Warp roles (one CTA per SM, 192 threads):
-//   warp 0     : TMA producer (lane 0; all 32 lanes issue the row gathers)
+//   warp 0     : TMA producer (lane 0)
 //   warp 1     : TMEM allocation + MMA issue (lane 0)
 //   warps 2..5 : epilogue (TMEM lanes 32*(warp%4) .. +31)
 #pragma once
@@ -153,34 +153,12 @@ __global__ void __launch_bounds__(G2Cfg<BN, STAGES, AMODE>::kThreads, 1)
       const G2Tile t = g2_decode<BN>(p, tile, prefix);
       int b_col;
       const CUtensorMap* tmb;
-      int tk0 = 0, tk1 = 0, tk2 = 0, tk3 = 0;
       if constexpr (AMODE == kATma) {
         b_col = p.seg[t.seg].b_col0 + t.n0;
         tmb = &p.tmB[t.seg];
-      } else if constexpr (AMODE == kAGatherLsu) {
-        b_col = (t.seg % (p.G * p.M)) * 64;
-        tmb = &p.tmB[0];
       } else {
         b_col = (t.seg % (p.G * p.M)) * 64;  // head h = g*M + e of segment (b, g, e)
         tmb = &p.tmB[0];
-        // rows 4*lane .. 4*lane+3 of the tile; rows past the segment re-read its
-        // first token (their results are never stored)
-        int tk[4];
-        const int first = p.seg_tok[t.row0];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int ci = t.row0 + 4 * lane + i;
-          int v = ci < t.row_end ? p.seg_tok[ci] : first;
-          if (v < 0 || v >= p.ntok) {
-            flag_bounds_error();
-            v = 0;
-          }
-          tk[i] = v;
-        }
-        tk0 = tk[0];
-        tk1 = tk[1];
-        tk2 = tk[2];
-        tk3 = tk[3];
       }
       const int nbox = t.nvalid / 64;
       for (int kb = 0; kb < nk; ++kb, ++it) {
@@ -205,10 +183,6 @@ __global__ void __launch_bounds__(G2Cfg<BN, STAGES, AMODE>::kThreads, 1)
           }
           for (int nb = 0; nb < nbox; ++nb)
             tma_load_2d(b_s + nb * 8192, tmb, &full[s], b_col + nb * 64, kb * kGemmBK);
-        }
-        if constexpr (AMODE == kAGather) {
-          __syncwarp();
-          tma_gather4(a_s + lane * 512, &p.tmA, &full[s], kb * kGemmBK, tk0, tk1, tk2, tk3);
         }
       }
     }

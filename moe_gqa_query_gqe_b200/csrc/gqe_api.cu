@@ -426,7 +426,7 @@ int do_qgather(const gqe_dims* d, const void* x, const void* Wq, const int32_t* 
   GemmParams p;
   memset(&p, 0, sizeof(p));
   GQE_TRY(tmap_rows(&p.tmB[0], Wq, d->D, wq_cols, wq_cols, 64));
-  GQE_TRY(tmap_rows(&p.tmA, x, N, d->D, d->D, 1));  // one-row box: gathered 4 rows at a time
+  GQE_TRY(tmap_rows(&p.tmA, x, N, d->D, d->D, 1));  // a valid map for the kernel's descriptor prefetch (rows are copied with cp.async)
   p.K = d->D;
   p.x = static_cast<const __nv_bfloat16*>(x);
   p.seg_off = seg_off;

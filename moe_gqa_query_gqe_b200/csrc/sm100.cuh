@@ -133,17 +133,6 @@ __device__ __forceinline__ void bulk_wait_read() {
 // All of this thread's bulk groups complete (writes performed).
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// Four rows (row0..row3) of a 2D tensor, columns [c0, c0 + box width), into
-// consecutive rows at dst. The tensor map's box is one row high.
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* tm, uint64_t* bar, int c0, int r0, int r1,
-                                            int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(tm)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-      : "memory");
-}
-
 // ---------------------------------------------------------------------------
 // cp.async (16-byte, zero-fill when src_bytes == 0) for gathered operands.
 // ---------------------------------------------------------------------------
