@@ -202,6 +202,71 @@ def run_reference(args, d, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def pool_study(steps: int, warmup: int) -> None:
+    """Expert-pool study: the layer at 32K tokens (D 1024, G 8) for pools of
+    M = 2, 4 and 8 experts per group with k selected, under near-balanced
+    routing and under the +2 bias on expert 0. Per configuration: one JSON
+    line with the GQE and dense step times (CUDA-graph replays, L2 flushed),
+    the speedup, the algorithmic flop ratio, and how unevenly the tokens
+    spread over the experts (largest and smallest segment over the mean)."""
+    import torch
+    import moe_gqa_query_gqe_b200 as gqe
+    from gqe_inputs import Dims, make_inputs
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def graph(fn):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            fn()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                fn()
+        torch.cuda.synchronize()
+        return g
+
+    def timed(g):
+        for _ in range(warmup):
+            flush.fill_(1)
+            g.replay()
+        evs = []
+        for _ in range(steps):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            b.record()
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in evs) / steps
+
+    for (M, k) in [(2, 1), (4, 1), (4, 2), (8, 1), (8, 2), (8, 4)]:
+        for bias0 in (0.0, 2.0):
+            d = Dims(B=1, T=32768, D=1024, G=8, M=M, k=k, bias0=bias0)
+            inp = make_inputs(d, seed=0, device="cuda")
+            N = d.B * d.T
+            ws, wd = gqe.workspace(d, gqe.OP_FORWARD), gqe.workspace(d, gqe.OP_DENSE)
+            y = torch.empty(N, d.D, dtype=torch.bfloat16, device="cuda")
+            y2 = torch.empty_like(y)
+            g1 = graph(lambda: gqe.gqe_forward(d, inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"],
+                                               inp["Wo"], y, ws))
+            g2 = graph(lambda: gqe.gqa_dense_forward(d, inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wo_dense"],
+                                                     y2, wd))
+            t_gqe, t_dense = timed(g1), timed(g2)
+            status = gqe.gqe_check_error()
+            seg = gqe.forward_views(d, ws)["seg_off"].diff().double()
+            mean = N * k / M
+            fl = flops_model(d)
+            print(json.dumps({"study": "expert_pool", "M": M, "k": k, "bias0": bias0, "T": d.T, "G": d.G,
+                              "gqe_ms": t_gqe, "dense_ms": t_dense, "speedup": t_dense / t_gqe,
+                              "flop_ratio": fl["dense_total"] / fl["gqe_total"],
+                              "segment_max_over_mean": float(seg.max() / mean),
+                              "segment_min_over_mean": float(seg.min() / mean), "status": status}), flush=True)
+            del g1, g2
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -211,6 +276,7 @@ def main():
     ap.add_argument("--impl", default="gqe", choices=["gqe", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle timing (rank 0, N=1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--study", choices=["pools"], help="print the expert-pool study lines instead of the bench line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -220,6 +286,9 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
+    if args.study == "pools":
+        pool_study(steps=min(args.steps, 20), warmup=args.warmup)
+        return
     if args.impl == "reference":
         run_reference(args, d, rank, world)
         return
