@@ -30,9 +30,13 @@ design notes of this repository):
   * shared head attends KV head 0;
   * scale 1/sqrt(dh), causal mask s <= t, no positional encoding or biases;
   * Wo rows: [concat (g-major, slot j) | slot g | shared];
-  * ablation variants ([AT] section 6): the hard and the weighted
-    concatenation keep the shared head; the weights of the weighted one are
-    the in-group probabilities of the selected experts (not renormalised);
+  * variants of the output construction ([AT] sections 4 and 6, [GS]
+    "Experimental results"): the hard and the weighted concatenation keep
+    the shared head; the weights of the weighted one are the in-group
+    probabilities of the selected experts (not renormalised); the single
+    global slot averages all selected outputs with those probabilities
+    renormalised over all groups; the no-shared-head variant keeps the
+    per-group slots;
   * decode step: the new token of sequence b sits at position cache_len[b],
     its K/V row is appended there and its queries attend positions
     0..cache_len[b] (the pages describe no decode procedure).
@@ -241,23 +245,53 @@ def combine(O, w, dims) -> np.ndarray:
     return np.concatenate([concat, slot, O[:, G * k]], axis=1)
 
 
-def combine_variant(O, p_sel, dims, mode: str) -> np.ndarray:
-    """Output construction of the ablation variants ([AT] section 6: a pure
-    hard concatenation, and a concatenation weighted directly by the router's
-    scores without the renormalised slot). Readings: both keep the shared
-    head; the scores are the in-group softmax probabilities of the selected
-    experts (not renormalised over the selected set).
-      mode "hard":     A = [concat | shared]
-      mode "weighted": A = [p_sel[g, j] * O[g, j] (concat) | shared]"""
+VARIANTS = ("hard", "weighted", "global_slot", "no_shared")
+
+
+def combine_width(dims, mode: str = "slot") -> int:
+    """Columns of A (= rows of Wo) for an output construction."""
+    G, k, dh = dims.G, dims.k, dims.dh
+    blocks = {"slot": G * k + G + 1, "hard": G * k + 1, "weighted": G * k + 1,
+              "global_slot": G * k + 2, "no_shared": G * k + G}
+    if mode not in blocks:
+        raise ValueError(mode)
+    return blocks[mode] * dh
+
+
+def combine_variant(O, w, p_sel, dims, mode: str) -> np.ndarray:
+    """Output construction of the variants of step 5.
+
+    [AT] section 6 (ablation): a pure hard concatenation, and a concatenation
+    weighted directly by the router's scores without the renormalised slot.
+    [GS] "Experimental results" words the ablation as removing the renormalised slot or
+    the shared head. [AT] section 4 can be read as ONE extra output, the
+    weighted average of all selected experts' outputs by their router scores.
+    Readings: the scores are the in-group softmax probabilities of the
+    selected experts (p_sel); the variants keep every part that they do not
+    name as removed.
+      "hard":        A = [concat | shared]
+      "weighted":    A = [p_sel[g, j] * O[g, j] (concat) | shared]
+      "global_slot": A = [concat | sum_{g,j} p_sel[g,j] O[g,j] / sum_{g,j} p_sel[g,j] | shared]
+      "no_shared":   A = [concat | per-group slot sum_j w[g,j] O[g,j]]"""
     G, k, dh = dims.G, dims.k, dims.dh
     O = np.asarray(O, F64)
     nr = O.shape[0]
-    routed = O[:, :G * k]
+    routed = O[:, :G * k]                       # [nr, G*k, dh], g-major, ascending expert
+    shared = O[:, G * k]
+    concat = routed.reshape(nr, G * k * dh)
+    if mode == "hard":
+        return np.concatenate([concat, shared], axis=1)
     if mode == "weighted":
-        routed = routed * np.asarray(p_sel, F64).reshape(nr, G * k)[:, :, None]
-    elif mode != "hard":
-        raise ValueError(mode)
-    return np.concatenate([routed.reshape(nr, G * k * dh), O[:, G * k]], axis=1)
+        p = np.asarray(p_sel, F64).reshape(nr, G * k)
+        return np.concatenate([(routed * p[:, :, None]).reshape(nr, G * k * dh), shared], axis=1)
+    if mode == "global_slot":
+        p = np.asarray(p_sel, F64).reshape(nr, G * k)
+        avg = np.einsum("nh,nhd->nd", p, routed) / p.sum(axis=1, keepdims=True)
+        return np.concatenate([concat, avg, shared], axis=1)
+    if mode == "no_shared":
+        slot = np.einsum("ngj,ngjd->ngd", np.asarray(w, F64), routed.reshape(nr, G, k, dh)).reshape(nr, G * dh)
+        return np.concatenate([concat, slot], axis=1)
+    raise ValueError(mode)
 
 
 # ---------------------------------------------------------------------------
@@ -276,8 +310,8 @@ def gqe_forward(x, Wq, Wk, Wv, Wr, br, Wo, dims, rows=None, forced_sel=None, com
          shared head];  6. y = A Wo.
     Returns the intermediate values too (all float64, rows in ``rows`` order).
     ``forced_sel`` ([len(rows), G, k]) overrides the router's choice.
-    ``combine_mode`` "hard" / "weighted" selects an ablation variant of step 5
-    (``combine_variant``; Wo then has (G*k + 1)*dh rows).
+    ``combine_mode`` (one of ``VARIANTS``) selects a variant of step 5
+    (``combine_variant``; Wo then has ``combine_width(dims, mode)`` rows).
     """
     B, T, D, G, M, k, dh = dims.B, dims.T, dims.D, dims.G, dims.M, dims.k, dims.dh
     X = _f64(x).reshape(B * T, D)
@@ -290,7 +324,7 @@ def gqe_forward(x, Wq, Wk, Wv, Wr, br, Wo, dims, rows=None, forced_sel=None, com
 
     O = attend_selected(Q, rows, K, V, dims)
     p_sel = np.take_along_axis(R["p"], sel, axis=2)
-    A = combine(O, w, dims) if combine_mode == "slot" else combine_variant(O, p_sel, dims, combine_mode)
+    A = combine(O, w, dims) if combine_mode == "slot" else combine_variant(O, w, p_sel, dims, combine_mode)
     y = A @ _f64(Wo)
     return {"rows": rows, "sel": sel, "w": w, "p_sel": p_sel, "margin": R["margin"], "logits": R["logits"],
             "p": R["p"], "K": K, "V": V, "Q": Q, "O": O, "A": A, "y": y}

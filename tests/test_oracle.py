@@ -449,9 +449,14 @@ def _variant(d, inp, mode, Wo, **kw):
                            combine_mode=mode, **kw)
 
 
-def _wo_variant(d, seed=4):
+def _wo_variant(d, mode="hard", seed=4):
     g = torch.Generator().manual_seed(seed)
-    return (torch.randn(((d.G * d.k + 1) * d.dh, d.D), generator=g) * 0.4).to(torch.bfloat16)
+    return (torch.randn((ref.combine_width(d, mode), d.D), generator=g) * 0.4).to(torch.bfloat16)
+
+
+def test_variant_widths_follow_the_construction():
+    d = Dims(B=1, T=1, D=64, G=8, M=2, k=1)
+    assert [ref.combine_width(d, m) // 64 for m in ("slot",) + ref.VARIANTS] == [17, 9, 9, 10, 16]
 
 
 @pytest.mark.parametrize("G,M,k", [(2, 2, 1), (2, 3, 2)])
@@ -489,6 +494,99 @@ def test_variant_weighted_scales_by_the_hand_worked_probabilities():
 def test_planted_renormalised_weights_in_the_weighted_variant_are_caught(monkeypatch):
     real = ref.combine_variant
     monkeypatch.setattr(ref, "combine_variant",
-                        lambda O, p_sel, dims, mode: real(O, np.ones_like(p_sel), dims, mode))
+                        lambda O, w, p_sel, dims, mode: real(O, w, np.ones_like(p_sel), dims, mode))
     with pytest.raises(AssertionError):
         test_variant_weighted_scales_by_the_hand_worked_probabilities()
+
+
+def test_variant_global_slot_of_the_hand_worked_example():
+    """The single global slot of the hand-worked example (G = 2, k = 1, dh = 1).
+    Token 0: group 0 keeps expert 0 (logits 1, 0: p = e/(1+e)), group 1 keeps
+    expert 1 of its pair (logits 0, 2: p = e^2/(1+e^2)); outputs 1 and 2.
+    Token 1: group 0 keeps expert 1 (logits 0, 1: p = e/(1+e)) with output
+    (e+3)/(e+1), group 1 keeps expert 0 (logits 3, 0: p = e^3/(1+e^3)) with
+    output 1. The slot is the probability-weighted average of the two."""
+    gold = load("worked_example_k1.txt")
+    d = gold["dims"]
+    inp = _as_inputs(gold)
+    Wo = torch.ones((ref.combine_width(d, "global_slot"), d.D), dtype=torch.float64)
+    out = _variant(d, inp, "global_slot", Wo)
+    e = math.e
+    pa, pb = e / (1 + e), e * e / (1 + e * e)
+    want0 = (pa * 1 + pb * 2) / (pa + pb)
+    pa, pb = e / (1 + e), e ** 3 / (1 + e ** 3)
+    want1 = (pa * (e + 3) / (e + 1) + pb * 1) / (pa + pb)
+    O = gold["expect.O"]
+    np.testing.assert_allclose(out["A"][0], [O[0][0], O[0][1], want0, O[0][2]], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(out["A"][1], [O[1][0], O[1][1], want1, O[1][2]], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(out["y"][:, 0], out["A"].sum(axis=1), rtol=0, atol=1e-13)
+
+
+def test_variant_global_slot_averages_equal_outputs_to_themselves():
+    """Whatever the probabilities, a weighted average of G*k copies of one
+    vector is that vector: pins the division by the summed probabilities."""
+    d = Dims(B=1, T=5, D=8, G=3, M=4, k=2, dh=4)
+    rng = np.random.default_rng(0)
+    u = rng.standard_normal((5, 1, 4))
+    O = np.concatenate([np.repeat(u, d.G * d.k, axis=1), rng.standard_normal((5, 1, 4))], axis=1)
+    p_sel = rng.uniform(0.05, 0.9, size=(5, d.G, d.k))
+    A = ref.combine_variant(O, None, p_sel, d, "global_slot")
+    gk = d.G * d.k * d.dh
+    np.testing.assert_allclose(A[:, gk:gk + d.dh], u[:, 0], rtol=0, atol=1e-14)
+    np.testing.assert_array_equal(A[:, -d.dh:], O[:, -1])
+
+
+def test_variant_global_slot_with_one_group_is_the_per_group_slot():
+    """With G = 1 the selected set of the only group is the set of all
+    selected experts, so the global slot is the GQE slot (same A)."""
+    d, inp = _small(B=2, T=18, G=1, M=3, k=2)
+    full = _fwd(d, inp)
+    glob = _variant(d, inp, "global_slot", _wo_variant(d, "global_slot"))
+    np.testing.assert_allclose(glob["A"], full["A"], rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("G,M,k", [(2, 2, 1), (3, 3, 2)])
+def test_variant_no_shared_is_the_slot_construction_without_the_shared_head(G, M, k):
+    d, inp = _small(B=2, T=20, G=G, M=M, k=k)
+    full = _fwd(d, inp)
+    Wo = _wo_variant(d, "no_shared")
+    out = _variant(d, inp, "no_shared", Wo)
+    np.testing.assert_array_equal(out["A"], full["A"][:, :-d.dh])
+    # the shared head's query weights no longer reach y
+    inp2 = dict(inp)
+    Wq = inp["Wq"].clone()
+    Wq[:, d.G * d.M * d.dh:] = 0
+    inp2["Wq"] = Wq
+    np.testing.assert_array_equal(_variant(d, inp2, "no_shared", Wo)["y"], out["y"])
+    assert not np.allclose(_fwd(d, inp2)["y"], full["y"])
+
+
+def test_planted_per_group_average_in_the_global_slot_is_caught(monkeypatch):
+    """A slot that averages the groups' renormalised slots (each group's
+    weights summing to 1, then divided by G) is a different construction."""
+    real = ref.combine_variant
+
+    def per_group_average(O, w, p_sel, dims, mode):
+        if mode != "global_slot":
+            return real(O, w, p_sel, dims, mode)
+        p = np.asarray(p_sel, np.float64)
+        return real(O, w, p / p.sum(axis=2, keepdims=True) / dims.G, dims, mode)
+
+    monkeypatch.setattr(ref, "combine_variant", per_group_average)
+    with pytest.raises(AssertionError):
+        test_variant_global_slot_of_the_hand_worked_example()
+
+
+def test_planted_unnormalised_global_slot_is_caught(monkeypatch):
+    real = ref.combine_variant
+
+    def unnormalised(O, w, p_sel, dims, mode):
+        A = real(O, w, p_sel, dims, mode)
+        if mode == "global_slot":
+            gk = dims.G * dims.k * dims.dh
+            A[:, gk:gk + dims.dh] *= np.asarray(p_sel, np.float64).reshape(A.shape[0], -1).sum(axis=1)[:, None]
+        return A
+
+    monkeypatch.setattr(ref, "combine_variant", unnormalised)
+    with pytest.raises(AssertionError):
+        test_variant_global_slot_averages_equal_outputs_to_themselves()
