@@ -78,11 +78,17 @@ enum gqe_op {
 
 /* Output construction of gqe_forward_variant. */
 enum gqe_combine_mode {
-  GQE_COMBINE_SLOT = 0,     /* GQE: [hard concat | renormalised slot per group | shared] */
-  GQE_COMBINE_HARD = 1,     /* ablation: [hard concat | shared], no slot                 */
-  GQE_COMBINE_WEIGHTED = 2  /* ablation: [concat, each selected output scaled by its
-                               expert's in-group probability (not renormalised) |
-                               shared], no slot                                           */
+  GQE_COMBINE_SLOT = 0,         /* GQE: [hard concat | renormalised slot per group | shared] */
+  GQE_COMBINE_HARD = 1,         /* ablation: [hard concat | shared], no slot                 */
+  GQE_COMBINE_WEIGHTED = 2,     /* ablation: [concat, each selected output scaled by its
+                                   expert's in-group probability (not renormalised) |
+                                   shared], no slot                                           */
+  GQE_COMBINE_GLOBAL_SLOT = 3,  /* [hard concat | ONE slot: all selected outputs averaged
+                                   with their in-group probabilities renormalised over
+                                   all G*k selected experts | shared]                         */
+  GQE_COMBINE_NO_SHARED = 4     /* ablation: [hard concat | renormalised slot per group],
+                                   no shared head (neither its query nor its attention
+                                   is computed)                                               */
 };
 
 /* Workspace bytes the operation needs for these dims (0 if none); returns 0
@@ -234,13 +240,19 @@ int gqe_forward_host(const gqe_dims* d, const void* x_host, const void* Wq,
  * besides the full design (hard concatenation, a renormalised weighted slot
  * and the always-on shared head) the ablation trains a pure hard
  * concatenation and a concatenation weighted directly by the router's scores
- * without the renormalised slot. This library's reading: both variants keep
- * the shared head (the page does not say they drop it), and the "router's
- * scores" are the in-group softmax probabilities of the selected experts.
+ * without the renormalised slot; the gist.science summary, "Experimental
+ * results", words the same ablation as removing the renormalised slot or the
+ * shared head; the article's section 4 can be read as ONE weighted-average
+ * slot over all selected experts. This library's readings: the variants keep
+ * every part they do not name as removed, and the "router's scores" are the
+ * in-group softmax probabilities of the selected experts.
  *
- * Wo: [(G*k + G + 1)*dh, D] for GQE_COMBINE_SLOT (identical to gqe_forward),
- *     [(G*k + 1)*dh, D] for the two variants (rows: concat g-major, slot j;
- *     then the shared head).
+ * Wo rows, in A's column order (concat g-major, slot j; slots; shared):
+ *     GQE_COMBINE_SLOT         (G*k + G + 1)*dh  (identical to gqe_forward)
+ *     GQE_COMBINE_HARD         (G*k + 1)*dh
+ *     GQE_COMBINE_WEIGHTED     (G*k + 1)*dh
+ *     GQE_COMBINE_GLOBAL_SLOT  (G*k + 2)*dh
+ *     GQE_COMBINE_NO_SHARED    (G*k + G)*dh
  * ws: gqe_workspace_bytes(d, GQE_OP_FORWARD_VARIANT). An unknown mode returns
  * GQE_ERR_INVALID_ARG. Everything else as gqe_forward.
  */

@@ -297,7 +297,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   } else {
     // ---- epilogue (both CTAs): this CTA's 128 rows ----------------------------------
     const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
-    const int row = q * 32 + lane;
     const uint32_t acce_c = mapa_shared(smem_u32(acc_empty), 0);
     uint8_t* stage_out = smem + L::kStageOut + q * 2 * L::kOutBytes;  // this warp's two staging buffers
     uint32_t nstore = 0;                                               // chunks staged by this warp

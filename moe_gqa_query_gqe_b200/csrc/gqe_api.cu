@@ -110,7 +110,6 @@ inline int cuda_status(cudaError_t e) {
   g_last_cuda_error = e;
   return GQE_ERR_CUDA;
 }
-inline int launch_status() { return cuda_status(cudaGetLastError()); }
 
 // Launch with programmatic stream serialization: the kernel may be scheduled
 // while the previous kernel in the stream is still finishing (every kernel of
@@ -302,9 +301,30 @@ FwdWs carve_forward(Carver& c, const gqe_dims* d) {
   return f;
 }
 
+// Columns of A, i.e. rows of Wo, for an output construction (gqe_combine_mode).
+int combine_cols(const gqe_dims* d, int mode) {
+  const int Gk = d->G * d->k;
+  switch (mode) {
+    case GQE_COMBINE_SLOT: return (Gk + d->G + 1) * 64;
+    case GQE_COMBINE_HARD:
+    case GQE_COMBINE_WEIGHTED: return (Gk + 1) * 64;
+    case GQE_COMBINE_GLOBAL_SLOT: return (Gk + 2) * 64;
+    case GQE_COMBINE_NO_SHARED: return (Gk + d->G) * 64;
+    default: return 0;
+  }
+}
+
+// The widest A among the variants other than GQE_COMBINE_SLOT (workspace of
+// gqe_forward_variant).
+int variant_max_cols(const gqe_dims* d) {
+  int c = 0;
+  for (int m = GQE_COMBINE_HARD; m <= GQE_COMBINE_NO_SHARED; ++m) c = std::max(c, combine_cols(d, m));
+  return c;
+}
+
 size_t combine_ws_bytes(const gqe_dims* d) {
   if (d->k == 1) return 0;  // A is read straight from O (see do_combine)
-  return align256((size_t)d->B * d->T * (d->G * d->k + d->G + 1) * 64 * 2);
+  return align256((size_t)d->B * d->T * combine_cols(d, GQE_COMBINE_SLOT) * 2);
 }
 
 struct DenseWs {
@@ -468,7 +488,7 @@ int sm_count() {
 
 // Persistent two-tile attention (attn2.cuh).
 int do_attn2(const gqe_dims* d, const void* Q, int Hq, const void* K, const void* V, void* O, bool dense,
-             cudaStream_t st) {
+             bool shared, cudaStream_t st) {
   const long long N = (long long)d->B * d->T;
   Attn2Params p;
   memset(&p, 0, sizeof(p));
@@ -483,7 +503,7 @@ int do_attn2(const gqe_dims* d, const void* Q, int Hq, const void* K, const void
   p.Ha = Hq;
   int nrs = 0;
   for (int g = 0; g < d->G; ++g) p.rs[nrs++] = AttnRowSet{g * rr, rr, g, 0};
-  if (!dense) p.rs[nrs++] = AttnRowSet{d->G * d->k, 1, 0, 1};
+  if (shared) p.rs[nrs++] = AttnRowSet{d->G * d->k, 1, 0, 1};
   p.nrs = nrs;
   p.npairs_max = (int)cdiv((long long)d->T * rr, 256);
   const long long items = (long long)p.npairs_max * d->B * nrs;
@@ -495,50 +515,67 @@ int do_attn2(const gqe_dims* d, const void* Q, int Hq, const void* K, const void
   return launch_pdl(attn2_fwd_kernel, dim3(grid), dim3(kA2Threads), A2Smem::kBytes, st, p);
 }
 
-int do_combine(const gqe_dims* d, const void* O, const float* w, const void* Wo, void* y, __nv_bfloat16* A,
-               cudaStream_t st) {
+// k = 1: the renormalised weight of the one selected expert is exactly 1, so
+// the slot of group g is O[:, g] itself and the projection reads A's blocks
+// straight from O (blocks [0, G) and [G, 2G) are O's routed blocks, block 2G
+// the shared head). KA is (2G + 1)*64, or 2G*64 without the shared head.
+int project_from_o(const gqe_dims* d, const void* O, const void* Wo, void* y, int KA, cudaStream_t st) {
   const long long N = (long long)d->B * d->T;
-  const int KA = (d->G * d->k + d->G + 1) * 64;
-  if (d->k == 1) {
-    // renormalised weights over one selected expert are exactly 1: the slot of
-    // group g is O[:, g] itself, so the projection reads A's blocks from O
-    GemmParams p;
-    memset(&p, 0, sizeof(p));
-    const int Ha = d->G + 1;
-    GQE_TRY(tmap_rows(&p.tmA, O, N, Ha * 64, Ha * 64, kGemmBM));
-    GQE_TRY(tmap_rows(&p.tmB[0], Wo, KA, d->D, d->D, 64));
-    p.seg[0] = GemmSeg{d->D, 0, 0, 0, (long long)d->D, static_cast<__nv_bfloat16*>(y)};
-    GQE_TRY(tmap_rows(&p.tmC[0], y, N, d->D, d->D, 32));
-    p.nseg = 1;
-    p.ntn = (int)cdiv(d->D, kG2DenseBN);
-    p.rows = (int)N;
-    p.K = KA;
-    p.amap_G = d->G;
-    p.r_tile0 = 0x7fffffff;
-    return launch_gemm_pair(p, cdiv(N, kPairBM) * p.ntn, st);
-  }
-  CombineParams cp{static_cast<const __nv_bfloat16*>(O), w, A, N, d->G, d->k, 0};
-  const long long warps = N;
-  const long long blocks = std::min<long long>(cdiv(warps * 32, 256), 148ll * 16);
-  GQE_TRY(launch_pdl(combine_build_kernel, dim3((unsigned)blocks), dim3(256), 0, st, cp));
-  const DenseSeg seg = {Wo, d->D, 0, d->D, y, (long long)d->D, 0};
-  return gemm_dense(A, N, KA, &seg, 1, st);
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  const int Ha = d->G + 1;
+  GQE_TRY(tmap_rows(&p.tmA, O, N, Ha * 64, Ha * 64, kGemmBM));
+  GQE_TRY(tmap_rows(&p.tmB[0], Wo, KA, d->D, d->D, 64));
+  p.seg[0] = GemmSeg{d->D, 0, 0, 0, (long long)d->D, static_cast<__nv_bfloat16*>(y)};
+  GQE_TRY(tmap_rows(&p.tmC[0], y, N, d->D, d->D, 32));
+  p.nseg = 1;
+  p.ntn = (int)cdiv(d->D, kG2DenseBN);
+  p.rows = (int)N;
+  p.K = KA;
+  p.amap_G = d->G;
+  p.r_tile0 = 0x7fffffff;
+  return launch_gemm_pair(p, cdiv(N, kPairBM) * p.ntn, st);
 }
 
-// Output construction of the ablation variants (no slot): A = [concat |
-// shared] with the concatenated outputs as they are (hard) or each scaled by
-// its expert's in-group probability (weighted); y = A Wo with Wo of
-// (G*k + 1)*64 rows. The hard variant's A is O itself.
-int do_combine_variant(const gqe_dims* d, int mode, const void* O, const float* p_sel, const void* Wo, void* y,
-                       __nv_bfloat16* A, cudaStream_t st) {
-  const long long N = (long long)d->B * d->T;
-  const int KA = (d->G * d->k + 1) * 64;
-  const DenseSeg seg = {Wo, d->D, 0, d->D, y, (long long)d->D, 0};
-  if (mode == GQE_COMBINE_HARD) return gemm_dense(O, N, KA, &seg, 1, st);
-  CombineParams cp{static_cast<const __nv_bfloat16*>(O), p_sel, A, N, d->G, d->k, 1};
-  const long long blocks = std::min<long long>(cdiv(N * 32, 256), 148ll * 16);
+// A = combine(O, w) by combine_build_kernel, then y = A Wo.
+int build_and_project(const gqe_dims* d, const CombineParams& cp, int KA, const void* Wo, void* y, cudaStream_t st) {
+  const long long blocks = std::min<long long>(cdiv(cp.N * 32, 256), 148ll * 16);
   GQE_TRY(launch_pdl(combine_build_kernel, dim3((unsigned)blocks), dim3(256), 0, st, cp));
-  return gemm_dense(A, N, KA, &seg, 1, st);
+  const DenseSeg seg = {Wo, d->D, 0, d->D, y, (long long)d->D, 0};
+  return gemm_dense(cp.A, cp.N, KA, &seg, 1, st);
+}
+
+int do_combine(const gqe_dims* d, const void* O, const float* w, const void* Wo, void* y, __nv_bfloat16* A,
+               cudaStream_t st) {
+  const int KA = combine_cols(d, GQE_COMBINE_SLOT);
+  if (d->k == 1) return project_from_o(d, O, Wo, y, KA, st);
+  const CombineParams cp{static_cast<const __nv_bfloat16*>(O), w, A, (long long)d->B * d->T, d->G, d->k,
+                         0, kSlotPerGroup, 1};
+  return build_and_project(d, cp, KA, Wo, y, st);
+}
+
+// Output construction of the variants (gqe_combine_mode), y = A Wo with Wo of
+// combine_cols(d, mode) rows. The hard variant's A is O itself.
+int do_combine_variant(const gqe_dims* d, int mode, const void* O, const float* w, const float* p_sel,
+                       const void* Wo, void* y, __nv_bfloat16* A, cudaStream_t st) {
+  const long long N = (long long)d->B * d->T;
+  const int KA = combine_cols(d, mode);
+  const __nv_bfloat16* Ob = static_cast<const __nv_bfloat16*>(O);
+  switch (mode) {
+    case GQE_COMBINE_HARD: {
+      const DenseSeg seg = {Wo, d->D, 0, d->D, y, (long long)d->D, 0};
+      return gemm_dense(O, N, KA, &seg, 1, st);
+    }
+    case GQE_COMBINE_WEIGHTED:
+      return build_and_project(d, CombineParams{Ob, p_sel, A, N, d->G, d->k, 1, kNoSlot, 1}, KA, Wo, y, st);
+    case GQE_COMBINE_GLOBAL_SLOT:
+      return build_and_project(d, CombineParams{Ob, p_sel, A, N, d->G, d->k, 0, kGlobalSlot, 1}, KA, Wo, y, st);
+    case GQE_COMBINE_NO_SHARED:
+      if (d->k == 1) return project_from_o(d, O, Wo, y, KA, st);
+      return build_and_project(d, CombineParams{Ob, w, A, N, d->G, d->k, 0, kSlotPerGroup, 0}, KA, Wo, y, st);
+    default:
+      return GQE_ERR_INVALID_ARG;
+  }
 }
 
 int check_ptrs(std::initializer_list<const void*> ps) {
@@ -618,7 +655,7 @@ size_t gqe_workspace_bytes(const gqe_dims* d, int op) {
       carve_forward(c, d);
       const size_t N = (size_t)d->B * d->T;
       c.take<float>(N * d->G * d->k);                                      // probabilities
-      c.take<__nv_bfloat16>(N * (size_t)(d->G * d->k + 1) * 64);            // variant A
+      c.take<__nv_bfloat16>(N * (size_t)variant_max_cols(d));              // variant A
       return c.off;
     }
     default: return 0;
@@ -658,7 +695,7 @@ int gqe_attn(const gqe_dims* d, const void* Q, const void* K, const void* V, voi
   GQE_TRY(check_dims(d));
   GQE_TRY(check_ptrs({Q, K, V, O}));
   GQE_TRY(check_device());
-  return do_attn2(d, Q, d->G * d->k + 1, K, V, O, false, static_cast<cudaStream_t>(stream));
+  return do_attn2(d, Q, d->G * d->k + 1, K, V, O, false, true, static_cast<cudaStream_t>(stream));
 }
 
 int gqe_combine(const gqe_dims* d, const void* O, const float* w, const void* Wo, void* y, void* ws, size_t ws_bytes,
@@ -681,23 +718,26 @@ int do_forward(const gqe_dims* d, int mode, const void* x, const void* Wq, const
   __nv_bfloat16* A2 = nullptr;
   if (mode != GQE_COMBINE_SLOT) {
     p_sel = c.take<float>(N * d->G * d->k);
-    A2 = c.take<__nv_bfloat16>(N * (size_t)(d->G * d->k + 1) * 64);
+    A2 = c.take<__nv_bfloat16>(N * (size_t)variant_max_cols(d));
   }
+  // Without the shared head neither its query nor its attention is computed
+  // (its column of Q and O is left unwritten and is never read).
+  const bool shared = mode != GQE_COMBINE_NO_SHARED;
   // one pair-GEMM launch over x: K, V, the shared head's query and the router
   // (logits and decisions), then the compaction and the selected queries
   DenseSeg segs[3];
   kv_segments(d, Wq, Wk, Wv, f.Q, f.K, f.V, segs);
   GemmParams p;
   long long dense_tiles = 0, route_tiles = 0;
-  GQE_TRY(dense_params(p, x, (long long)d->B * d->T, d->D, segs, 3, &dense_tiles));
+  GQE_TRY(dense_params(p, x, (long long)d->B * d->T, d->D, segs, shared ? 3 : 2, &dense_tiles));
   GQE_TRY(add_route_tiles(p, d, Wr, br, f.sel, f.w, f.margin, f.route, dense_tiles, &route_tiles));
-  p.r_p = mode == GQE_COMBINE_WEIGHTED ? p_sel : nullptr;
+  p.r_p = (mode == GQE_COMBINE_WEIGHTED || mode == GQE_COMBINE_GLOBAL_SLOT) ? p_sel : nullptr;
   GQE_TRY(launch_gemm_pair(p, dense_tiles + route_tiles, st));
   GQE_TRY(route_finish(d, f.sel, f.seg_off, f.seg_tok, f.row_map, f.route, st));
   GQE_TRY(do_qgather(d, x, Wq, f.sel, f.seg_off, f.seg_tok, f.Q, st));
-  GQE_TRY(do_attn2(d, f.Q, d->G * d->k + 1, f.K, f.V, f.O, false, st));
+  GQE_TRY(do_attn2(d, f.Q, d->G * d->k + 1, f.K, f.V, f.O, false, shared, st));
   if (mode == GQE_COMBINE_SLOT) return do_combine(d, f.O, f.w, Wo, y, f.A, st);
-  return do_combine_variant(d, mode, f.O, p_sel, Wo, y, A2, st);
+  return do_combine_variant(d, mode, f.O, f.w, p_sel, Wo, y, A2, st);
 }
 
 int gqe_forward(const gqe_dims* d, const void* x, const void* Wq, const void* Wk, const void* Wv, const void* Wr,
@@ -714,8 +754,7 @@ int gqe_forward_variant(const gqe_dims* d, int mode, const void* x, const void* 
                         const void* Wr, const float* br, const void* Wo, void* y, void* ws, size_t ws_bytes,
                         void* stream) {
   GQE_TRY(check_dims(d));
-  if (mode != GQE_COMBINE_SLOT && mode != GQE_COMBINE_HARD && mode != GQE_COMBINE_WEIGHTED)
-    return GQE_ERR_INVALID_ARG;
+  if (mode < GQE_COMBINE_SLOT || mode > GQE_COMBINE_NO_SHARED) return GQE_ERR_INVALID_ARG;
   GQE_TRY(check_ptrs({x, Wq, Wk, Wv, Wr, Wo, y}));
   if (br && !aligned16(br)) return GQE_ERR_INVALID_ARG;
   GQE_TRY(check_ws(ws, ws_bytes, gqe_workspace_bytes(d, GQE_OP_FORWARD_VARIANT)));
@@ -813,7 +852,7 @@ int gqa_dense_forward(const gqe_dims* d, const void* x, const void* Wq, const vo
       {Wv, G * 64, 0, G * 64, w.V, (long long)G * 64, 0},
   };
   GQE_TRY(gemm_dense(x, N, d->D, segs, 3, st));
-  GQE_TRY(do_attn2(d, w.Q, H, w.K, w.V, w.O, true, st));
+  GQE_TRY(do_attn2(d, w.Q, H, w.K, w.V, w.O, true, false, st));
   const DenseSeg so = {Wo_dense, d->D, 0, d->D, y, (long long)d->D, 0};
   return gemm_dense(w.O, N, H * 64, &so, 1, st);
 }

@@ -10,6 +10,7 @@ import torch
 
 import moe_gqa_query_gqe_b200 as gqe
 from moe_gqa_query_gqe_b200 import lib
+import oracle.gqe_ref as ref
 from gqe_inputs import CONFIGS, Dims
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -53,6 +54,18 @@ def test_all_workloads_are_supported_and_sized():
         assert gqe.workspace_bytes(d, gqe.OP_FORWARD_VARIANT) > gqe.workspace_bytes(d, gqe.OP_FORWARD)
 
 
+def test_variant_workspace_holds_the_widest_variant():
+    """Beyond gqe_forward's workspace, the variants need the selected
+    experts' probabilities (fp32) and their own A (bf16, the widest of the
+    non-slot constructions)."""
+    for d in (CONFIGS["main_b8_t2048"], Dims(B=2, T=136, D=256, G=8, M=8, k=4), Dims(B=1, T=5, D=128, G=1, M=8, k=2)):
+        N = d.B * d.T
+        widest = max(ref.combine_width(d, m) for m in ref.VARIANTS)
+        extra = gqe.workspace_bytes(d, gqe.OP_FORWARD_VARIANT) - gqe.workspace_bytes(d, gqe.OP_FORWARD)
+        assert extra >= N * d.G * d.k * 4 + N * widest * 2
+        assert extra <= N * d.G * d.k * 4 + N * widest * 2 + 512  # two 256-byte alignments
+
+
 def test_decode_workspace_grows_with_the_cache_capacity():
     d = Dims(B=4, T=1024, D=256, G=4, M=2, k=1)
     small = gqe.workspace_bytes(d, gqe.OP_DECODE)
@@ -88,8 +101,10 @@ def test_null_and_misaligned_pointers_are_rejected_before_any_launch():
     assert _raw("gqa_dense_forward", dp, P, P, P, P, P, None, P, 1 << 30, None) == -1
     # gqe_forward_variant: unknown combine mode, then a valid mode without workspace
     vargs = [P, P, P, P, P, None, P, P]
-    assert _raw("gqe_forward_variant", dp, 7, *vargs, P, 1 << 30, None) == -1
-    assert _raw("gqe_forward_variant", dp, 2, *vargs, None, 0, None) == -3
+    for bad_mode in (-1, 5, 7):
+        assert _raw("gqe_forward_variant", dp, bad_mode, *vargs, P, 1 << 30, None) == -1
+    for mode in range(5):
+        assert _raw("gqe_forward_variant", dp, mode, *vargs, None, 0, None) == -3
     # gqe_decode: null cache_len, misaligned x_new, missing workspace
     args = [P, P, P, P, P, P, None, P, P, P, P, P, P]
     assert _raw("gqe_decode", dp, None, *args[1:], P, 1 << 30, None) == -1

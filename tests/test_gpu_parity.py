@@ -11,29 +11,15 @@ import pytest
 import torch
 
 import oracle.gqe_ref as ref
-from gqe_inputs import CONFIGS, Dims, make_inputs
+from gqe_inputs import CONFIGS, make_inputs
+
+from _cases import SMALL
 
 pytestmark = pytest.mark.gpu
 
 if torch.cuda.is_available():
     from _gpu import (assert_close_bf16, check_selection, errors, f64, reference_attention, run_dense,
                       run_forward, run_stages, to_dev)
-
-# sizes the oracle finishes in seconds; several tiles and ragged tails
-SMALL = {
-    "tiny_b2_t256": CONFIGS["tiny_b2_t256"],
-    "ragged_b3_t300": Dims(B=3, T=300, D=256, G=4, M=2, k=1),
-    "pool4_k2_skewed_t384": Dims(B=1, T=384, D=512, G=8, M=4, k=2, bias0=2.0),
-    "single_token_b4": Dims(B=4, T=1, D=128, G=2, M=4, k=1),
-    "one_group_g1_m8_k2": Dims(B=2, T=200, D=192, G=1, M=8, k=2),
-    "k_equals_m_t260": Dims(B=1, T=260, D=128, G=4, M=2, k=2),
-    "pool8_k4_t136": Dims(B=2, T=136, D=256, G=8, M=8, k=4),
-    # +20 router bias on expert 0: every token picks it, the other experts'
-    # segments are empty
-    "empty_segments_bias20": Dims(B=2, T=160, D=256, G=4, M=4, k=1, bias0=20.0),
-    "one_token_b1_t1": Dims(B=1, T=1, D=128, G=4, M=2, k=1),
-}
-
 
 @pytest.fixture(scope="module")
 def cases():
@@ -111,42 +97,6 @@ def test_dense_gqa_baseline(cases, name):
     assert status == 0
     want = ref.gqa_dense_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wo_dense"], d)
     assert_close_bf16(y, want["y"], "dense GQA y vs oracle")
-
-
-VARIANT_CODE = {"slot": 0, "hard": 1, "weighted": 2}
-
-
-def _variant_wo(d, seed=6):
-    g = torch.Generator().manual_seed(seed)
-    return (torch.randn(((d.G * d.k + 1) * 64, d.D), generator=g) * 0.02).to(torch.bfloat16)
-
-
-@pytest.mark.parametrize("name", ["tiny_b2_t256", "ragged_b3_t300", "pool4_k2_skewed_t384", "pool8_k4_t136"])
-@pytest.mark.parametrize("mode", ["hard", "weighted"])
-def test_combine_variants(cases, name, mode):
-    """The ablation variants of the output construction (no slot; hard or
-    probability-weighted concatenation) against the oracle's variant."""
-    import moe_gqa_query_gqe_b200 as gqe
-    d, inp, dev, st = cases[name]
-    Wo = _variant_wo(d)
-    ws = gqe.workspace(d, gqe.OP_FORWARD_VARIANT)
-    y = torch.full((d.B * d.T, d.D), float("nan"), dtype=torch.bfloat16, device="cuda")
-    gqe.gqe_forward_variant(d, VARIANT_CODE[mode], dev["x"], dev["Wq"], dev["Wk"], dev["Wv"], dev["Wr"], dev["br"],
-                            Wo.cuda(), y, ws)
-    assert gqe.gqe_check_error() == 0
-    want = ref.gqe_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"], Wo, d,
-                           forced_sel=st["sel"].numpy(), combine_mode=mode)
-    assert_close_bf16(y, want["y"], f"{mode} variant y vs oracle")
-
-
-def test_slot_mode_of_the_variant_entry_is_gqe_forward(cases):
-    import moe_gqa_query_gqe_b200 as gqe
-    d, inp, dev, st = cases["pool4_k2_skewed_t384"]
-    ws = gqe.workspace(d, gqe.OP_FORWARD_VARIANT)
-    y = torch.empty((d.B * d.T, d.D), dtype=torch.bfloat16, device="cuda")
-    gqe.gqe_forward_variant(d, 0, dev["x"], dev["Wq"], dev["Wk"], dev["Wv"], dev["Wr"], dev["br"], dev["Wo"], y, ws)
-    assert gqe.gqe_check_error() == 0
-    assert torch.equal(y.cpu(), st["y"])
 
 
 def test_empty_segments_are_empty(cases):
