@@ -52,6 +52,24 @@ def flops_model(d) -> dict:
     return {"gqe": f, "gqe_total": sum(f.values()), "dense": dense, "dense_total": sum(dense.values())}
 
 
+def stage_rooflines(d, stage_ms: dict, peaks: dict) -> dict:
+    """Roofline of each of the four stage calls. Routing is bound by HBM: it
+    reads x and writes the decisions, their weights, margins, token lists and
+    row map (algorithmic bytes). The other three stages are tensor-bound:
+    their algorithmic flops over the stage time, against the bf16 peak."""
+    N = d.B * d.T
+    fl = flops_model(d)["gqe"]
+    route_bytes = 2 * N * d.D + 2 * d.D * d.G * d.M + 4 * N * d.G * d.k * 4 + 4 * N * d.G + 4 * (d.B * d.G * d.M + 1)
+    out = {"route": {"bound": "hbm", "unit": "GB/s", "algorithmic": route_bytes,
+                     "achieved": route_bytes / (stage_ms["route"] / 1e3) / 1e9, "peak": peaks["hbm_gbs"]}}
+    for name, flops in (("qproj", fl["q_proj"] + fl["kv_proj"]), ("attention", fl["attention"]), ("combine", fl["wo"])):
+        out[name] = {"bound": "tensor", "unit": "TFLOP/s", "algorithmic": flops,
+                     "achieved": flops / (stage_ms[name] / 1e3) / 1e12, "peak": peaks["bf16_tflops"]}
+    for v in out.values():
+        v["frac"] = v["achieved"] / v["peak"]
+    return out
+
+
 def load_peaks() -> dict:
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
@@ -461,7 +479,8 @@ def main():
             "tflops": fl["gqe_total"] / (ms_per_step / 1e3) / 1e12 * world,
             "frac_bf16_peak": fl["gqe_total"] / (ms_per_step / 1e3) / 1e12 / peaks["bf16_tflops"],
             "dense_gqa_ms_per_step": dense_ms, "speedup_vs_dense": dense_ms / ms_per_step,
-            "stage_ms": stage_avg, "roofline": roofline, "clocks": clocks,
+            "stage_ms": stage_avg, "stage_roofline": stage_rooflines(d, stage_avg, peaks), "roofline": roofline,
+            "clocks": clocks,
             "e2e": {"value": job_throughput(world, N, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": N * d.D * 2, "d2h_bytes_per_step": N * d.D * 2,
                     "entry": "gqe_forward_host"},
