@@ -285,6 +285,62 @@ def pool_study(steps: int, warmup: int) -> None:
             del g1, g2
 
 
+def decode_study(steps: int, warmup: int) -> None:
+    """Decode step (gqe_decode): one new token per sequence against caches of
+    L positions, for the main layer's shape (D 1024, G 8, M 2, k 1). Per
+    configuration: one JSON line with the step time (CUDA-graph replays, L2
+    flushed between them), tokens/s, the bytes the step must read (the K/V
+    cache rows up to each new token, plus the weights) and that rate as a
+    fraction of the measured HBM bandwidth."""
+    import torch
+    import moe_gqa_query_gqe_b200 as gqe
+    from gqe_inputs import Dims, make_decode_inputs
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    peaks = load_peaks()
+    for (B, L) in [(8, 32767), (64, 4095), (1, 131071)]:
+        d = Dims(B=B, T=L + 1, D=1024, G=8, M=2, k=1)
+        inp = {kk: v.cuda() for kk, v in make_decode_inputs(d, [L] * B, seed=0, device="cpu").items()}
+        y = torch.empty(B, d.D, dtype=torch.bfloat16, device="cuda")
+        sel = torch.empty(B, d.G, d.k, dtype=torch.int32, device="cuda")
+        w = torch.empty(B, d.G, d.k, dtype=torch.float32, device="cuda")
+        ws = gqe.workspace(d, gqe.OP_DECODE)
+
+        def step():
+            gqe.gqe_decode(d, inp["cache_len"], inp["x_new"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"],
+                           inp["Wo"], inp["K_cache"], inp["V_cache"], y, sel, w, ws)
+
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            step()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                step()
+        torch.cuda.synchronize()
+        evs = []
+        for i in range(warmup + steps):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            b.record()
+            if i >= warmup:
+                evs.append((a, b))
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+        cache_bytes = B * (L + 1) * d.G * 64 * 2 * 2
+        weight_bytes = sum(inp[kk].numel() * inp[kk].element_size() for kk in ("Wq", "Wk", "Wv", "Wr", "Wo"))
+        gbs = (cache_bytes + weight_bytes) / (ms / 1e3) / 1e9
+        print(json.dumps({"study": "decode", "B": B, "L": L, "D": d.D, "G": d.G, "M": d.M, "k": d.k,
+                          "us_per_step": ms * 1e3, "tokens_per_s": B / (ms / 1e3),
+                          "bytes_per_step": cache_bytes + weight_bytes, "achieved_gbs": gbs,
+                          "peak_gbs": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
+                          "status": gqe.gqe_check_error()}), flush=True)
+        del g
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -294,7 +350,8 @@ def main():
     ap.add_argument("--impl", default="gqe", choices=["gqe", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle timing (rank 0, N=1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--study", choices=["pools"], help="print the expert-pool study lines instead of the bench line")
+    ap.add_argument("--study", choices=["pools", "decode"],
+                    help="print the expert-pool or decode-step study lines instead of the bench line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -306,6 +363,9 @@ def main():
 
     if args.study == "pools":
         pool_study(steps=min(args.steps, 20), warmup=args.warmup)
+        return
+    if args.study == "decode":
+        decode_study(steps=min(args.steps, 20), warmup=args.warmup)
         return
     if args.impl == "reference":
         run_reference(args, d, rank, world)
