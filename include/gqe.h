@@ -313,6 +313,17 @@ int gqe_check_error(void* stream);
  * calling host thread ("no error" if there was none). */
 const char* gqe_last_cuda_error(void);
 
+/*
+ * gqe_selftest_wait_timeout -- failure-detection self-test. Enqueues on
+ * `stream` one small kernel that waits on a pipeline barrier nothing will
+ * ever complete, with the same bounded wait as every kernel of the library.
+ * After about 2 s the wait gives up. It records a timeout in the device error
+ * word and the kernel returns; it does not trap. The next gqe_check_error
+ * then returns GQE_ERR_TIMEOUT, and the context stays usable. Returns
+ * GQE_ERR_CUDA if the launch fails.
+ */
+int gqe_selftest_wait_timeout(void* stream);
+
 /* Static description of a status code. */
 const char* gqe_status_string(int status);
 

@@ -578,6 +578,20 @@ int do_combine_variant(const gqe_dims* d, int mode, const void* O, const float* 
   }
 }
 
+// Self-test of the bounded waits: one thread waits on an mbarrier that no
+// thread arrives on, so the wait runs out, records the timeout and returns.
+__global__ void selftest_wait_kernel() {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag);
+}
+
 int check_ptrs(std::initializer_list<const void*> ps) {
   for (const void* p : ps)
     if (p == nullptr || !aligned16(p)) return GQE_ERR_INVALID_ARG;
@@ -870,6 +884,12 @@ int gqe_check_error(void* stream) {
 }
 
 const char* gqe_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_error); }
+
+int gqe_selftest_wait_timeout(void* stream) {
+  GQE_TRY(check_device());
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  return cuda_status(cudaGetLastError());
+}
 
 const char* gqe_status_string(int status) {
   switch (status) {

@@ -25,7 +25,7 @@ COMBINE_SLOT, COMBINE_HARD, COMBINE_WEIGHTED, COMBINE_GLOBAL_SLOT, COMBINE_NO_SH
 # every symbol include/gqe.h declares
 EXPORTS = ("gqe_workspace_bytes", "gqe_validate_dims", "gqe_route", "gqe_route_noalloc", "gqe_qproj", "gqe_attn", "gqe_combine",
            "gqe_forward", "gqe_forward_variant", "gqe_forward_host", "gqe_decode", "gqa_dense_forward", "gqe_check_error", "gqe_status_string", "gqe_last_cuda_error",
-           "gqe_version")
+           "gqe_selftest_wait_timeout", "gqe_version")
 
 
 class GqeDims(ctypes.Structure):
@@ -67,6 +67,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "gqe_check_error": (ctypes.c_int, [vp]),
         "gqe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "gqe_last_cuda_error": (ctypes.c_char_p, []),
+        "gqe_selftest_wait_timeout": (ctypes.c_int, [vp]),
         "gqe_version": (ctypes.c_int, []),
     }
     for name, (res, args) in sig.items():
@@ -183,6 +184,12 @@ def gqa_dense_forward(dims, x, Wq, Wk, Wv, Wo_dense, y, ws, stream=None) -> None
 
 def gqe_check_error(stream=None) -> int:
     return int(load().gqe_check_error(_stream(stream)))
+
+
+def gqe_selftest_wait_timeout(stream=None) -> None:
+    """Enqueue the bounded-wait self-test: the next gqe_check_error returns
+    GQE_ERR_TIMEOUT (-5) after about 2 s."""
+    _call("gqe_selftest_wait_timeout", _stream(stream))
 
 
 def gqe_status_string(code: int) -> str:

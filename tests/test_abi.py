@@ -117,3 +117,8 @@ def test_valid_call_without_a_device_reports_no_device():
     d = lib.dims_struct(Dims(B=1, T=64, D=256, G=4, M=2, k=1))
     P = 1 << 20
     assert _raw("gqe_attn", ctypes.byref(d), P, P, P, P, None, 0, None) == -6
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device answer")
+def test_wait_self_test_without_a_device_reports_no_device():
+    assert _raw("gqe_selftest_wait_timeout", None) == -6
