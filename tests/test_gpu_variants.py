@@ -21,7 +21,7 @@ pytestmark = pytest.mark.gpu
 
 if torch.cuda.is_available():
     import moe_gqa_query_gqe_b200 as gqe
-    from _gpu import assert_close_bf16, run_stages, to_dev
+    from _gpu import assert_close_bf16, f64, run_dense, run_forward, run_stages, to_dev
 
     MODE = {"slot": gqe.COMBINE_SLOT, "hard": gqe.COMBINE_HARD, "weighted": gqe.COMBINE_WEIGHTED,
             "global_slot": gqe.COMBINE_GLOBAL_SLOT, "no_shared": gqe.COMBINE_NO_SHARED}
@@ -83,3 +83,20 @@ def test_no_shared_variant_never_reads_the_shared_head(cases, name):
     Wq[:, d.G * d.M * 64:] = float("nan")
     y1 = _run(d, dev, "no_shared", Wo, Wq=Wq)
     assert torch.equal(y0.cpu(), y1.cpu())
+
+
+def test_k_equals_m_with_zero_slot_and_shared_rows_is_dense_gqa():
+    """With k = M every expert is selected and the concatenation is in head
+    order (h = g*M + e). With Wo's concatenation rows set to Wo_dense and its
+    slot and shared rows set to zero, the layer is the dense GQA layer up to
+    rounding (the GQE invariant, checked here on the GPU's two paths)."""
+    d = SMALL["k_equals_m_t260"]
+    inp = make_inputs(d, seed=0)
+    dev = to_dev(inp)
+    Wo = torch.zeros((d.wo_rows, d.D), dtype=torch.bfloat16)
+    Wo[:d.G * d.k * 64] = inp["Wo_dense"]
+    y, _, status = run_forward(d, dict(dev, Wo=Wo.cuda()))
+    assert status == 0
+    yd, _, status = run_dense(d, dev)
+    assert status == 0
+    assert_close_bf16(y, f64(yd), "GQE with k = M and zero slot/shared rows vs dense GQA")
