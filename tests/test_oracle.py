@@ -590,3 +590,29 @@ def test_planted_unnormalised_global_slot_is_caught(monkeypatch):
     monkeypatch.setattr(ref, "combine_variant", unnormalised)
     with pytest.raises(AssertionError):
         test_variant_global_slot_averages_equal_outputs_to_themselves()
+
+
+# ---------------------------------------------------------------------------
+# The skewed-routing input recipe against its closed form
+# ---------------------------------------------------------------------------
+def test_skewed_recipe_expert0_shares_match_the_closed_form():
+    """x ~ N(0, 1) and Wr ~ N(0, 0.02^2) make the logits of a group nearly
+    independent N(0, s^2), s = 0.02 sqrt(D). With the +2 bias on expert 0 of
+    M = 4, expert 0 ranks first with probability E[Phi(Z + 2/s)^3] and lands
+    in the top 2 with probability E[Phi^3 + 3 Phi^2 (1 - Phi)], Z ~ N(0, 1)
+    (numerical integration). The oracle's routing of 4096 tokens x 8 groups
+    must match both to 0.015."""
+    d = Dims(B=1, T=4096, D=2048, G=8, M=4, k=2, bias0=2.0)
+    inp = make_inputs(d, seed=0)
+    r = ref.route(inp["x"], inp["Wr"], inp["br"], d.G, d.M, d.k)
+    rank1 = float(np.mean(np.argmax(r["p"], axis=2) == 0))
+    top2 = float(np.mean(np.any(r["sel"] == 0, axis=2)))
+    a0 = 2.0 / (0.02 * math.sqrt(d.D))
+    z = np.linspace(-10.0, 10.0, 40001)
+    phi = np.exp(-0.5 * z * z) / math.sqrt(2.0 * math.pi)
+    Phi = np.array([0.5 * (1.0 + math.erf((v + a0) / math.sqrt(2.0))) for v in z])
+    want1 = float(np.trapezoid(phi * Phi ** 3, z))
+    want2 = float(np.trapezoid(phi * (Phi ** 3 + 3.0 * Phi ** 2 * (1.0 - Phi)), z))
+    assert abs(rank1 - want1) < 0.015, (rank1, want1)
+    assert abs(top2 - want2) < 0.015, (top2, want2)
+    assert 0.85 < want1 < 0.88 and 0.96 < want2 < 0.975
