@@ -10,8 +10,6 @@ constexpr int kGemmBM = 128;
 constexpr int kGemmBK = 64;
 constexpr int kMaxGemmSegs = 3;
 
-enum GemmAMode : int { kATma = 0, kAGatherLsu = 2 };
-
 // One output segment of a dense (TMA-A) launch: columns [b_col0, b_col0+n_cols)
 // of the weight behind tmB[seg], written to C[:, c_col0 + ...] with row stride ldc.
 struct GemmSeg {

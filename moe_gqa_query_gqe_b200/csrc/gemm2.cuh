@@ -1,24 +1,23 @@
-// gemm2.cuh -- persistent single-CTA tcgen05 GEMM: C = A * B, bf16 in, fp32
-// accumulate in TMEM. Used for the router logits (with the routing epilogue)
-// and for the selected-expert query projection when the head's weight slice
-// is too large to stay resident (D > 1024); the dense projections run on CTA
-// pairs (gemm2sm.cuh).
+// gemm2.cuh -- persistent single-CTA tcgen05 GEMM for the selected-expert
+// query projection when the head's weight slice is too large to stay resident
+// in shared memory (D > 1024; qgather.cuh covers D <= 1024): for every expert
+// segment s = (b, g, e), Q rows of the tokens that picked expert e of group g
+// are x[token] * Wq[:, head g*M+e], written to token-major Q at slot (g, j).
 //
-//   A [rows, K] row-major (K-major operand): TMA tiles (dense rows), or rows
-//     gathered by a segment's token list with 16-byte cp.async by eight
-//     copier warps (the selected-expert query projection: only tokens that
-//     picked the expert are multiplied).
-//   B [K, N] row-major weight (MN-major operand), 64 x 64 TMA boxes, 128-byte
-//     swizzle. The MMA N of a tile is the segment's remaining width rounded
-//     up to 64 (no work on columns past the segment).
-//   Tiles of 128 x BN; persistent CTAs walk the tile list round-robin. The
-//   TMEM accumulator is double-buffered (2 x BN columns), so the epilogue of
-//   one tile overlaps the main loop of the next.
+//   A [rows, K] (K-major operand): rows gathered by the segment's token list
+//     with 16-byte cp.async by eight copier warps, so only tokens that picked
+//     the expert are multiplied.
+//   B [K, 64] slice of the row-major weight (MN-major operand), streamed in
+//     64 x 64 TMA boxes with 128-byte swizzle alongside the A rows.
+//   Tiles of 128 rows of one segment; persistent CTAs walk the tile list
+//   round-robin. The TMEM accumulator is double-buffered (2 x BN columns),
+//   so the epilogue of one tile overlaps the main loop of the next.
 //
-// Warp roles (one CTA per SM, 192 threads):
-//   warp 0     : TMA producer (lane 0)
+// Warp roles (one CTA per SM, 448 threads):
+//   warp 0     : TMA producer of the weight boxes (lane 0)
 //   warp 1     : TMEM allocation + MMA issue (lane 0)
-//   warps 2..5 : epilogue (TMEM lanes 32*(warp%4) .. +31)
+//   warps 2..5 : epilogue (TMEM lanes 32*(warp%4) .. +31), rows scattered to Q
+//   warps 6..13: A copiers
 #pragma once
 
 #include "gemm.cuh"
@@ -28,63 +27,47 @@ namespace gqe {
 
 constexpr int kG2MaxSegsSmem = 8192;  // gather mode: segment tile prefix kept in shared memory
 
-template <int BN, int STAGES, int AMODE>
+template <int BN, int STAGES>
 struct G2Cfg {
-  // kAGatherLsu: 8 more warps copy the gathered A rows with cp.async
-  static constexpr int kThreads = AMODE == kAGatherLsu ? 448 : 192;
+  static constexpr int kThreads = 448;  // 8 of the 14 warps copy the gathered A rows
   static constexpr int kABytes = kGemmBM * kGemmBK * 2;  // 16 KB
   static constexpr int kBBytes = BN * kGemmBK * 2;       // BN/64 boxes of 8 KB
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kBarOffset = STAGES * kStageBytes;
   static constexpr int kPrefixOffset = kBarOffset + 256;
-  static constexpr int kBytesBase = kPrefixOffset + 1024;  // + (nsegs+1)*4 in gather mode
+  static constexpr int kBytesBase = kPrefixOffset + 1024;  // + (nsegs+1)*4 for the tile prefix
 };
 
 struct G2Tile {
-  int m0;        // first row (dense) / first compacted row offset within the segment (gather)
-  int seg;       // dense: output segment; gather: expert segment
-  int n0;        // first column of the segment
-  int nvalid;    // columns computed (multiple of 64, <= BN)
-  int row0, row_end;  // gather: compacted row range of the tile
+  int m0;             // first compacted row offset within the segment
+  int seg;            // expert segment
+  int nvalid;         // columns computed (64: one head)
+  int row0, row_end;  // compacted row range of the tile
 };
 
-template <int BN>
 __device__ __forceinline__ G2Tile g2_decode(const GemmParams& p, int tile, const int* s_prefix) {
   G2Tile t;
-  if (s_prefix == nullptr) {
-    const int mt = tile / p.ntn, nt = tile % p.ntn;
-    t.m0 = mt * kGemmBM;
-    t.seg = 0;
-    for (int s = 1; s < p.nseg; ++s)
-      if (nt >= p.seg[s].tile_start) t.seg = s;
-    t.n0 = (nt - p.seg[t.seg].tile_start) * BN;
-    const int rem = p.seg[t.seg].n_cols - t.n0;
-    t.nvalid = rem >= BN ? BN : ((rem + 63) / 64) * 64;
-    t.row0 = t.row_end = 0;
-  } else {
-    // largest s with s_prefix[s] <= tile
-    int lo = 0, hi = p.nsegs_q - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s_prefix[mid] <= tile) lo = mid; else hi = mid - 1;
-    }
-    t.seg = lo;
-    const int mt = tile - s_prefix[lo];
-    t.m0 = mt * kGemmBM;
-    t.row0 = p.seg_off[lo] + t.m0;
-    t.row_end = min(p.seg_off[lo + 1], p.seg_off[p.nsegs_q]);
-    t.n0 = 0;
-    t.nvalid = 64;
+  // largest s with s_prefix[s] <= tile
+  int lo = 0, hi = p.nsegs_q - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_prefix[mid] <= tile) lo = mid; else hi = mid - 1;
   }
+  t.seg = lo;
+  const int mt = tile - s_prefix[lo];
+  t.m0 = mt * kGemmBM;
+  t.row0 = p.seg_off[lo] + t.m0;
+  t.row_end = min(p.seg_off[lo + 1], p.seg_off[p.nsegs_q]);
+  t.nvalid = 64;
   return t;
 }
 
-template <int BN, int STAGES, int AMODE>
-__global__ void __launch_bounds__(G2Cfg<BN, STAGES, AMODE>::kThreads, 1)
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(G2Cfg<BN, STAGES>::kThreads, 1)
     gemm2_kernel(const __grid_constant__ GemmParams p, int total_tiles) {
   pdl_wait();
   pdl_trigger();
-  using C = G2Cfg<BN, STAGES, AMODE>;
+  using C = G2Cfg<BN, STAGES>;
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -99,29 +82,27 @@ __global__ void __launch_bounds__(G2Cfg<BN, STAGES, AMODE>::kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nk = (p.K + kGemmBK - 1) / kGemmBK;
 
-  if constexpr (AMODE != kATma) {
-    // tile prefix over the expert segments: s_prefix[s] = tiles before segment s
-    if (warp == 0) {
-      int before = 0;
-      for (int s0 = 0; s0 < p.nsegs_q; s0 += 32) {
-        const int s = s0 + lane;
-        const int len = s < p.nsegs_q ? p.seg_off[s + 1] - p.seg_off[s] : 0;
-        const int nt = (len + kGemmBM - 1) / kGemmBM;
-        int incl = nt;
+  // tile prefix over the expert segments: s_prefix[s] = tiles before segment s
+  if (warp == 0) {
+    int before = 0;
+    for (int s0 = 0; s0 < p.nsegs_q; s0 += 32) {
+      const int s = s0 + lane;
+      const int len = s < p.nsegs_q ? p.seg_off[s + 1] - p.seg_off[s] : 0;
+      const int nt = (len + kGemmBM - 1) / kGemmBM;
+      int incl = nt;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int u = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += u;
-        }
-        if (s < p.nsegs_q) s_prefix[s] = before + incl - nt;
-        before += __shfl_sync(0xffffffffu, incl, 31);
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
       }
-      if (lane == 0) s_prefix[p.nsegs_q] = before;
+      if (s < p.nsegs_q) s_prefix[s] = before + incl - nt;
+      before += __shfl_sync(0xffffffffu, incl, 31);
     }
+    if (lane == 0) s_prefix[p.nsegs_q] = before;
   }
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], AMODE == kAGatherLsu ? 1 + 256 : 1);
+      mbar_init(&full[s], 1 + 256);  // the weight boxes' arrival + one per copier thread
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -134,53 +115,33 @@ __global__ void __launch_bounds__(G2Cfg<BN, STAGES, AMODE>::kThreads, 1)
   if (warp == 1) tmem_alloc(tmem_slot, 2 * BN);
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&p.tmA);
-    for (int s = 0; s < (AMODE == kATma ? p.nseg : 1); ++s) tma_prefetch_desc(&p.tmB[s]);
+    tma_prefetch_desc(&p.tmB[0]);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t smem_base = smem_u32(smem);
-  int ntiles = total_tiles;
-  if constexpr (AMODE != kATma) ntiles = min(total_tiles, s_prefix[p.nsegs_q]);
-  const int* prefix = AMODE != kATma ? s_prefix : nullptr;
+  const int ntiles = min(total_tiles, s_prefix[p.nsegs_q]);
+  const int* prefix = s_prefix;
 
   if (warp == 0) {
-    // ---- TMA producer: A tiles (dense rows or gathered rows) and B tiles -------
+    // ---- TMA producer: the weight boxes of every stage ---------------------------
     uint32_t it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
-      const G2Tile t = g2_decode<BN>(p, tile, prefix);
-      int b_col;
-      const CUtensorMap* tmb;
-      if constexpr (AMODE == kATma) {
-        b_col = p.seg[t.seg].b_col0 + t.n0;
-        tmb = &p.tmB[t.seg];
-      } else {
-        b_col = (t.seg % (p.G * p.M)) * 64;  // head h = g*M + e of segment (b, g, e)
-        tmb = &p.tmB[0];
-      }
+      const G2Tile t = g2_decode(p, tile, prefix);
+      const int b_col = (t.seg % (p.G * p.M)) * 64;  // head h = g*M + e of segment (b, g, e)
+      const CUtensorMap* tmb = &p.tmB[0];
       const int nbox = t.nvalid / 64;
       for (int kb = 0; kb < nk; ++kb, ++it) {
         const int s = it % STAGES;
         bool w_ok = true;
         if (lane == 0) w_ok = mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort_flag);
         if (!(ok = __shfl_sync(0xffffffffu, w_ok, 0))) break;
-        uint8_t* a_s = smem + s * C::kStageBytes;
-        uint8_t* b_s = a_s + C::kABytes;
+        uint8_t* b_s = smem + s * C::kStageBytes + C::kABytes;
         if (lane == 0) {
-          mbar_arrive_expect_tx(&full[s], (AMODE == kAGatherLsu ? 0 : C::kABytes) + nbox * 8192);
-          if constexpr (AMODE == kATma) {
-            int a_col = kb * kGemmBK;
-            if (p.amap_G > 0) {
-              // k-block kb of A = [concat (G) | slot (G) | shared]: for k = 1 each
-              // slot equals its group's output (weight exactly 1), so both
-              // halves read O's routed columns and the last block its shared one
-              const int blk = kb < 2 * p.amap_G ? kb % p.amap_G : p.amap_G;
-              a_col = blk * kGemmBK;
-            }
-            tma_load_2d(a_s, &p.tmA, &full[s], a_col, t.m0);
-          }
+          mbar_arrive_expect_tx(&full[s], nbox * 8192);
           for (int nb = 0; nb < nbox; ++nb)
             tma_load_2d(b_s + nb * 8192, tmb, &full[s], b_col + nb * 64, kb * kGemmBK);
         }
@@ -192,7 +153,7 @@ __global__ void __launch_bounds__(G2Cfg<BN, STAGES, AMODE>::kThreads, 1)
       uint32_t it = 0, tcount = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++tcount) {
-        const G2Tile t = g2_decode<BN>(p, tile, prefix);
+        const G2Tile t = g2_decode(p, tile, prefix);
         const uint32_t a = tcount & 1;
         if (!(ok = mbar_wait(&acc_empty[a], ((tcount >> 1) & 1) ^ 1, abort_flag))) break;
         tc_fence_after();
@@ -202,7 +163,7 @@ __global__ void __launch_bounds__(G2Cfg<BN, STAGES, AMODE>::kThreads, 1)
           const int s = it % STAGES;
           if (!(ok = mbar_wait(&full[s], (it / STAGES) & 1, abort_flag))) break;
           // rows copied by cp.async (generic proxy) are read by the MMA (async proxy)
-          if constexpr (AMODE == kAGatherLsu) fence_proxy_async_smem();
+          fence_proxy_async_smem();
           tc_fence_after();
           const uint32_t a_addr = smem_base + s * C::kStageBytes;
           const uint32_t b_addr = a_addr + C::kABytes;
@@ -216,86 +177,78 @@ __global__ void __launch_bounds__(G2Cfg<BN, STAGES, AMODE>::kThreads, 1)
       }
     }
   } else if (warp >= 6) {
-    if constexpr (AMODE == kAGatherLsu) {
-      // ---- A copiers (warps 6..13): 16-byte chunk c of rows r = i*32 + ct/8 -------
-      // The token rows of the next tile are fetched while this tile's copies run,
-      // so no copier waits on a token-list load at a tile boundary.
-      const int ct = tid - 192;  // 0..255
-      const int c = ct & 7;
-      uint32_t it = 0;
-      bool ok = true;
-      auto fetch_rows = [&](int tile, int (&tk)[4]) {
-        const G2Tile t = g2_decode<BN>(p, tile, prefix);
-        const int first = p.seg_tok[t.row0];
+    // ---- A copiers (warps 6..13): 16-byte chunk c of rows r = i*32 + ct/8 -------
+    // The token rows of the next tile are fetched while this tile's copies run,
+    // so no copier waits on a token-list load at a tile boundary.
+    const int ct = tid - 192;  // 0..255
+    const int c = ct & 7;
+    uint32_t it = 0;
+    bool ok = true;
+    auto fetch_rows = [&](int tile, int (&tk)[4]) {
+      const G2Tile t = g2_decode(p, tile, prefix);
+      const int first = p.seg_tok[t.row0];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = i * 32 + (ct >> 3);
-          tk[i] = (t.row0 + r < t.row_end) ? p.seg_tok[t.row0 + r] : first;
-        }
-      };
-      int tk_cur[4] = {0, 0, 0, 0}, tk_next[4] = {0, 0, 0, 0};
-      if ((int)blockIdx.x < ntiles) fetch_rows(blockIdx.x, tk_cur);
-      for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
-        if (tile + (int)gridDim.x < ntiles) fetch_rows(tile + gridDim.x, tk_next);
-        uint32_t dst_off[4];
-        const __nv_bfloat16* src[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = i * 32 + (ct >> 3);
-          int v = tk_cur[i];
-          if (v < 0 || v >= p.ntok) {
-            flag_bounds_error();
-            v = 0;
-          }
-          src[i] = p.x + (size_t)v * p.K + c * 8;
-          dst_off[i] = r * 128 + ((c ^ (r & 7)) << 4);
-        }
-        for (int kb = 0; kb < nk; ++kb, ++it) {
-          const int s = it % STAGES;
-          if (!(ok = mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort_flag))) break;
-          const uint32_t a_addr = smem_base + s * C::kStageBytes;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) cp_async_16_full(a_addr + dst_off[i], src[i] + kb * kGemmBK);
-          cp_async_mbar_arrive_noinc(&full[s]);  // arrives when these copies land; no wait here
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) tk_cur[i] = tk_next[i];
+      for (int i = 0; i < 4; ++i) {
+        const int r = i * 32 + (ct >> 3);
+        tk[i] = (t.row0 + r < t.row_end) ? p.seg_tok[t.row0 + r] : first;
       }
-      asm volatile("cp.async.wait_all;" ::: "memory");  // nothing may be in flight when the CTA exits
+    };
+    int tk_cur[4] = {0, 0, 0, 0}, tk_next[4] = {0, 0, 0, 0};
+    if ((int)blockIdx.x < ntiles) fetch_rows(blockIdx.x, tk_cur);
+    for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+      if (tile + (int)gridDim.x < ntiles) fetch_rows(tile + gridDim.x, tk_next);
+      uint32_t dst_off[4];
+      const __nv_bfloat16* src[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = i * 32 + (ct >> 3);
+        int v = tk_cur[i];
+        if (v < 0 || v >= p.ntok) {
+          flag_bounds_error();
+          v = 0;
+        }
+        src[i] = p.x + (size_t)v * p.K + c * 8;
+        dst_off[i] = r * 128 + ((c ^ (r & 7)) << 4);
+      }
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = it % STAGES;
+        if (!(ok = mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, abort_flag))) break;
+        const uint32_t a_addr = smem_base + s * C::kStageBytes;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) cp_async_16_full(a_addr + dst_off[i], src[i] + kb * kGemmBK);
+        cp_async_mbar_arrive_noinc(&full[s]);  // arrives when these copies land; no wait here
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tk_cur[i] = tk_next[i];
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // nothing may be in flight when the CTA exits
   } else {
     // ---- epilogue ---------------------------------------------------------------
     const int q = warp & 3;
     const int row = q * 32 + lane;
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tcount) {
-      const G2Tile t = g2_decode<BN>(p, tile, prefix);
+      const G2Tile t = g2_decode(p, tile, prefix);
       const uint32_t a = tcount & 1;
       const bool ok = mbar_wait(&acc_full[a], (tcount >> 1) & 1, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       __nv_bfloat16* dst_row = nullptr;
-      if constexpr (AMODE == kATma) {
-        const GemmSeg& sg = p.seg[t.seg];
-        if (t.m0 + row < p.rows) dst_row = sg.C + (size_t)(t.m0 + row) * sg.ldc + sg.c_col0 + t.n0;
-      } else {
-        const int ci = t.row0 + row;
-        if (ci < t.row_end) {
-          const int GM = p.G * p.M;
-          const int n = p.seg_tok[ci];
-          const int g = (t.seg % GM) / p.M, e = t.seg % p.M;
-          if (n >= 0 && n < p.ntok) {
-            int j = 0;
-            for (int jj = 0; jj < p.k; ++jj)
-              if (p.sel[((size_t)n * p.G + g) * p.k + jj] == e) j = jj;
-            dst_row = p.Q + ((size_t)n * p.Ha + g * p.k + j) * 64;
-          } else {
-            flag_bounds_error();
-          }
+      const int ci = t.row0 + row;
+      if (ci < t.row_end) {
+        const int GM = p.G * p.M;
+        const int n = p.seg_tok[ci];
+        const int g = (t.seg % GM) / p.M, e = t.seg % p.M;
+        if (n >= 0 && n < p.ntok) {
+          int j = 0;
+          for (int jj = 0; jj < p.k; ++jj)
+            if (p.sel[((size_t)n * p.G + g) * p.k + jj] == e) j = jj;
+          dst_row = p.Q + ((size_t)n * p.Ha + g * p.k + j) * 64;
+        } else {
+          flag_bounds_error();
         }
       }
-      int ncols = t.nvalid;
-      if constexpr (AMODE == kATma) ncols = min(t.nvalid, p.seg[t.seg].n_cols - t.n0);
+      const int ncols = t.nvalid;
       const uint32_t tm = tmem_base + a * BN + (static_cast<uint32_t>(q * 32) << 16);
       for (int cc = 0; cc < t.nvalid / 32; ++cc) {
         uint32_t r[32];

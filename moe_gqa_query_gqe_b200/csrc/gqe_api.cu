@@ -139,15 +139,14 @@ int set_smem(K kernel, int bytes) {
 
 constexpr int kG2DenseBN = kPairBN;
 constexpr int kG2GatherStages = 8;
-constexpr int kG2GatherMode = kAGatherLsu;
 
 int sm_count();
 
-template <int BN, int STAGES, int AMODE>
+template <int BN, int STAGES>
 int launch_gemm2(const GemmParams& p, long long tiles, cudaStream_t st) {
-  using C = G2Cfg<BN, STAGES, AMODE>;
-  auto kern = gemm2_kernel<BN, STAGES, AMODE>;
-  const int smem = C::kBytesBase + (AMODE != kATma ? (p.nsegs_q + 1) * 4 : 0);
+  using C = G2Cfg<BN, STAGES>;
+  auto kern = gemm2_kernel<BN, STAGES>;
+  const int smem = C::kBytesBase + (p.nsegs_q + 1) * 4;
   if (int e = set_smem(kern, smem)) return e;
   if (tiles <= 0) return GQE_OK;
   if (tiles > 0x7fffffffll) return GQE_ERR_UNSUPPORTED;
@@ -469,7 +468,7 @@ int do_qgather(const gqe_dims* d, const void* x, const void* Wq, const int32_t* 
     const int grid = (int)std::min<long long>(tiles_max, sm_count());
     return launch_pdl(qgather_kernel, dim3(grid), dim3(kQgThreads), qg_smem, st, p, qg_stages);
   }
-  return launch_gemm2<64, kG2GatherStages, kG2GatherMode>(p, tiles_max, st);
+  return launch_gemm2<64, kG2GatherStages>(p, tiles_max, st);
 }
 
 int do_qproj(const gqe_dims* d, const void* x, const void* Wq, const void* Wk, const void* Wv, const int32_t* sel,
