@@ -18,8 +18,9 @@ from _cases import SMALL
 pytestmark = pytest.mark.gpu
 
 if torch.cuda.is_available():
-    from _gpu import (assert_close_bf16, check_selection, errors, f64, reference_attention, run_dense,
+    from _gpu import (assert_close_bf16, check_selection, f64, reference_attention, run_dense,
                       run_forward, run_stages, to_dev)
+
 
 @pytest.fixture(scope="module")
 def cases():
