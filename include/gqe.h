@@ -144,6 +144,9 @@ int gqe_route(const gqe_dims* d, const void* x, const void* Wr, const float* br,
  *   rounded up to 256 bytes) is larger than 1048576.
  * - The first call on each device looks up the array's device address (with
  *   that device current); make that first call before any stream capture.
+ *   The address is kept for the life of the process: do not use this entry
+ *   point on a device after cudaDeviceReset (or any teardown of its primary
+ *   context) in the same process, since the array then moves.
  * - Every call on a device shares the one array and leaves its contents
  *   behind. Nothing in it needs to start at zero (every entry is written
  *   before it is read), but calls that overlap on the GPU (different streams
@@ -227,6 +230,11 @@ int gqe_forward(const gqe_dims* d, const void* x, const void* Wq,
  * call enqueues the copy of x_host into the workspace, the forward pass and
  * the copy of y back to y_host, all on `stream` (pin both host buffers for the
  * copies to be asynchronous). Weights are device pointers.
+ * Host-buffer lifetime: the call returns once the work is enqueued. x_host
+ * must stay allocated and unmodified, and y_host allocated and unread, until
+ * the stream has passed the call (cudaStreamSynchronize, or an event recorded
+ * after it). With pinned memory from a caching allocator, a buffer released
+ * early can be handed out again and overwritten before its copy has run.
  * ws: gqe_workspace_bytes(d, GQE_OP_FORWARD_HOST).
  */
 int gqe_forward_host(const gqe_dims* d, const void* x_host, const void* Wq,

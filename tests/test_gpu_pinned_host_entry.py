@@ -30,7 +30,10 @@ def test_host_entry_matches_device_entry(name):
     y_dev, _, status = run_forward(d, dev)
     assert status == 0
     ws = gqe.workspace(d, gqe.OP_FORWARD_HOST)
-    y_host = _host_forward(d, dev, inp["x"].pin_memory(), ws)
+    # the copies are asynchronous: x_host must stay allocated and unchanged
+    # until the stream has passed the call
+    x_host = inp["x"].pin_memory()
+    y_host = _host_forward(d, dev, x_host, ws)
     torch.cuda.synchronize()
     assert gqe.gqe_check_error() == 0
     assert torch.equal(y_host, y_dev.cpu())
@@ -44,8 +47,13 @@ def test_host_entry_back_to_back_calls_at_the_main_shape():
     dev = to_dev(inp)
     x2 = make_inputs(d, seed=1)["x"]
     ws = gqe.workspace(d, gqe.OP_FORWARD_HOST)
-    y1 = _host_forward(d, dev, inp["x"].pin_memory(), ws)
-    y2 = _host_forward(d, dev, x2.pin_memory(), ws)
+    # Both pinned inputs are held until the stream has passed both calls: the
+    # library's copies are asynchronous, and a pinned buffer freed earlier can
+    # be handed out again (and overwritten) before its copy has read it.
+    x1_host = inp["x"].pin_memory()
+    x2_host = x2.pin_memory()
+    y1 = _host_forward(d, dev, x1_host, ws)
+    y2 = _host_forward(d, dev, x2_host, ws)
     torch.cuda.synchronize()
     assert gqe.gqe_check_error() == 0
     want1, _, s1 = run_forward(d, dev)
