@@ -201,6 +201,76 @@ def oracle_sample(d, budget_s: float, max_steps: int | None = None):
     return d1.T, times
 
 
+NEAR_TIE = 1e-4  # top-k margin (logit units) under which either choice is accepted
+
+
+def oracle_leg(d, inp: dict, sel_gpu, y_gpu, budget_s: float, extra_routes=()) -> tuple[dict, dict]:
+    """The CPU-baseline leg: the fp64 oracle, as it stands, timed on whole
+    sequences of the timed run's own batch (sequence i of the batch at sample
+    i, cycling), on the host cores, for about ``budget_s`` seconds.
+
+    The same oracle outputs also score the timed run: per sequence, the GPU's
+    expert selections against the oracle's (bit-exact, except near-tie
+    decisions whose margin is below 1e-4, which are counted and accepted) and
+    the GPU's y against the oracle's y (rel-L2 and max-abs; the oracle is
+    rerun, untimed, with the GPU's selections where a near tie flipped).
+    ``extra_routes`` are (name, dims, x, Wr, br, sel_gpu) of other workloads
+    whose selections are scored the same way (routing only)."""
+    import numpy as np
+    import oracle.gqe_ref as ref
+    d1 = d.with_(B=1)
+    w = {kk: v.cpu() for kk, v in inp.items() if kk != "x"}
+    x_all = inp["x"]
+    sel_all = sel_gpu.cpu().numpy().astype(np.int64)
+    y_all = y_gpu.cpu().double().numpy()
+    times, checked = [], {}
+    worst = {"rel_l2": 0.0, "max_abs": 0.0}
+    ties = {"decisions": 0, "near_ties": 0, "flipped_near_ties": 0, "mismatches_beyond_tie": 0}
+    t_all = time.time()
+    i = 0
+    while True:
+        b = i % d.B
+        xs = x_all[b * d.T:(b + 1) * d.T].cpu()
+        t0 = time.perf_counter()
+        out = ref.gqe_forward(xs, w["Wq"], w["Wk"], w["Wv"], w["Wr"], w["br"], w["Wo"], d1)
+        times.append(time.perf_counter() - t0)
+        if b not in checked:
+            sg = sel_all[b * d.T:(b + 1) * d.T]
+            r = ref.route(xs, w["Wr"], w["br"], d.G, d.M, d.k)
+            differ = np.any(sg != r["sel"], axis=2)
+            near = r["margin"] < NEAR_TIE
+            ties["decisions"] += differ.size
+            ties["near_ties"] += int(near.sum())
+            ties["flipped_near_ties"] += int((differ & near).sum())
+            ties["mismatches_beyond_tie"] += int((differ & ~near).sum())
+            want = out["y"]
+            if differ.any():
+                want = ref.gqe_forward(xs, w["Wq"], w["Wk"], w["Wv"], w["Wr"], w["br"], w["Wo"], d1,
+                                       forced_sel=sg)["y"]
+            diff = y_all[b * d.T:(b + 1) * d.T] - want
+            worst["rel_l2"] = max(worst["rel_l2"], float(np.linalg.norm(diff) / np.linalg.norm(want)))
+            worst["max_abs"] = max(worst["max_abs"], float(np.abs(diff).max()))
+            checked[b] = True
+        i += 1
+        if time.time() - t_all >= budget_s and i >= 1:
+            break
+    sec = sum(times) / len(times)
+    cpu = {"value": d.T / sec, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+           "sample": f"{len(times)} x one full sequence ({d.T} tokens, all rows) of the timed batch, fp64"}
+    parity = {"sequences_checked": len(checked), "of_sequences": d.B, "rows": len(checked) * d.T,
+              "worst_rel_l2": worst["rel_l2"], "worst_max_abs": worst["max_abs"],
+              "bars": {"rel_l2": 5e-3, "max_abs": 1e-2, "near_tie_margin": NEAR_TIE}, **ties}
+    for name, dx, x, Wr, br, sg in extra_routes:
+        r = ref.route(x.cpu(), Wr.cpu(), br.cpu(), dx.G, dx.M, dx.k)
+        sg = sg.cpu().numpy().astype(np.int64)
+        differ = np.any(sg != r["sel"], axis=2)
+        near = r["margin"] < NEAR_TIE
+        parity[name] = {"decisions": int(differ.size), "near_ties": int(near.sum()),
+                        "flipped_near_ties": int((differ & near).sum()),
+                        "mismatches_beyond_tie": int((differ & ~near).sum())}
+    return cpu, parity
+
+
 def run_reference(args, d, rank, world):
     """The oracle arm: the fp64 CPU oracle as it stands, on host cores."""
     if rank != 0:
@@ -341,6 +411,84 @@ def decode_study(steps: int, warmup: int) -> None:
         del g
 
 
+def long_context(names, steps: int, warmup: int, seed: int, peaks: dict, flush) -> tuple[dict, list]:
+    """The layer at long context: per workload, the GQE forward and the same
+    library's dense GQA forward as CUDA-graph replays (L2 flushed before each,
+    CUDA events on the launching stream), the routed attention alone (its
+    C-ABI call on the forward's own Q/K/V), and the GPU's routing decisions
+    for scoring against the oracle. The million-token workload takes one
+    warm-up and two timed steps per arm (about 2 and 3 s a step)."""
+    import torch
+    import moe_gqa_query_gqe_b200 as gqe
+    from gqe_inputs import CONFIGS, make_inputs
+    out, routes = {}, []
+    stream = torch.cuda.current_stream()
+    for name in names:
+        d = CONFIGS[name]
+        big = d.B * d.T > (1 << 18)
+        n_steps, n_warm = (2, 1) if big else (max(3, min(steps, 10)), max(3, warmup))
+        inp = make_inputs(d, seed=seed, device="cuda")
+        N = d.B * d.T
+        ws, wd = gqe.workspace(d, gqe.OP_FORWARD), gqe.workspace(d, gqe.OP_DENSE)
+        y = torch.empty(N, d.D, dtype=torch.bfloat16, device="cuda")
+        yd = torch.empty_like(y)
+
+        def graph(fn):
+            side = torch.cuda.Stream()
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):
+                fn()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                fn()
+            torch.cuda.synchronize()
+            return g
+
+        def timed(fn, n, w):
+            evs = []
+            for i in range(w + n):
+                flush.fill_(1)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                if i >= w:
+                    evs.append((a, b))
+            torch.cuda.synchronize()
+            return sum(a.elapsed_time(b) for a, b in evs) / n
+
+        g1 = graph(lambda: gqe.gqe_forward(d, inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"],
+                                           inp["Wo"], y, ws))
+        t_gqe = timed(g1.replay, n_steps, n_warm)
+        st1 = gqe.gqe_check_error()
+        del g1
+        v = gqe.forward_views(d, ws)
+        t_attn = timed(lambda: gqe.gqe_attn(d, v["Q"], v["K"], v["V"], v["O"]), n_steps, 1)
+        st2 = gqe.gqe_check_error()
+        g2 = graph(lambda: gqe.gqa_dense_forward(d, inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wo_dense"],
+                                                 yd, wd))
+        t_dense = timed(g2.replay, n_steps, n_warm)
+        st3 = gqe.gqe_check_error()
+        del g2
+        fl = flops_model(d)
+        attn_tf = fl["gqe"]["attention"] / (t_attn / 1e3) / 1e12
+        margin = v["margin"]
+        out[name] = {"T": d.T, "B": d.B, "steps": n_steps, "warmup": n_warm, "ms_per_step": t_gqe,
+                     "tokens_per_s": N / (t_gqe / 1e3), "dense_ms": t_dense, "speedup_vs_dense": t_dense / t_gqe,
+                     "flop_ratio": fl["dense_total"] / fl["gqe_total"],
+                     "tflops": fl["gqe_total"] / (t_gqe / 1e3) / 1e12,
+                     "attention_ms": t_attn, "attention_tflops": attn_tf,
+                     "attention_frac": attn_tf / peaks["bf16_tflops"],
+                     "attention_frac_sustained": attn_tf / peaks["bf16_tflops_sustained"],
+                     "gpu_margin_below_1e-4": int((margin < NEAR_TIE).sum().item()),
+                     "status": [st1, st2, st3]}
+        routes.append((name, d, inp["x"].cpu(), inp["Wr"].cpu(), inp["br"].cpu(), v["sel"].cpu()))
+        del inp, ws, wd, y, yd, v, margin
+        torch.cuda.empty_cache()
+    return out, routes
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -350,6 +498,8 @@ def main():
     ap.add_argument("--impl", default="gqe", choices=["gqe", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle timing (rank 0, N=1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--long", default="long_b1_t32768,million_b1_t1048576",
+                    help="comma-separated long-context workloads timed after the headline (empty: none)")
     ap.add_argument("--study", choices=["pools", "decode"],
                     help="print the expert-pool or decode-step study lines instead of the bench line")
     args = ap.parse_args()
@@ -547,11 +697,14 @@ def main():
             "gpu_launches": launches_per_step * args.steps,
             "timing": "each step one CUDA-graph replay of gqe_forward; stage_ms from the four stage calls"}
 
+    # long-context keys: one GPU, headline workload only (a scaling run keeps its timed work short)
+    long_names = [n for n in args.long.split(",") if n] if (args.workload == DEFAULT_WORKLOAD and world == 1) else []
+    routes = []
+    if long_names:
+        line["long_ctx"], routes = long_context(long_names, args.steps, args.warmup, rank, peaks, flush)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tokens, times = oracle_sample(d, args.cpu_budget)
-        sec = sum(times) / len(times)
-        line["cpu_baseline"] = {"value": tokens / sec, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
-                                "sample": f"{len(times)} x one full sequence ({tokens} tokens) of the workload, fp64"}
+        sel_fwd = gqe.forward_views(d, ws_fwd)["sel"]
+        line["cpu_baseline"], line["parity"] = oracle_leg(d, inp, sel_fwd, y, args.cpu_budget, routes)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
