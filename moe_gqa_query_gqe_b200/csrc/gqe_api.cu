@@ -591,6 +591,40 @@ __global__ void selftest_wait_kernel() {
   if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag);
 }
 
+// Streams and events of the host-buffer entry point, created once per device
+// and reused (guarded by g_pipe_mutex while a call enqueues its work).
+constexpr int kHostChunks = 8;
+constexpr int kPipeDevices = 64;
+struct HostPipe {
+  cudaStream_t h2d, d2h;
+  cudaEvent_t start, done, in[kHostChunks], out[kHostChunks];
+  bool ready;
+};
+std::mutex g_pipe_mutex;
+HostPipe g_pipe[kPipeDevices];
+
+int host_pipe(HostPipe** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GQE_ERR_NO_DEVICE;
+  if (dev < 0 || dev >= kPipeDevices) return GQE_ERR_UNSUPPORTED;
+  HostPipe& hp = g_pipe[dev];
+  if (!hp.ready) {
+    HostPipe n;
+    GQE_TRY(cuda_status(cudaStreamCreateWithFlags(&n.h2d, cudaStreamNonBlocking)));
+    GQE_TRY(cuda_status(cudaStreamCreateWithFlags(&n.d2h, cudaStreamNonBlocking)));
+    GQE_TRY(cuda_status(cudaEventCreateWithFlags(&n.start, cudaEventDisableTiming)));
+    GQE_TRY(cuda_status(cudaEventCreateWithFlags(&n.done, cudaEventDisableTiming)));
+    for (int i = 0; i < kHostChunks; ++i) {
+      GQE_TRY(cuda_status(cudaEventCreateWithFlags(&n.in[i], cudaEventDisableTiming)));
+      GQE_TRY(cuda_status(cudaEventCreateWithFlags(&n.out[i], cudaEventDisableTiming)));
+    }
+    n.ready = true;
+    hp = n;
+  }
+  *out = &hp;
+  return GQE_OK;
+}
+
 int check_ptrs(std::initializer_list<const void*> ps) {
   for (const void* p : ps)
     if (p == nullptr || !aligned16(p)) return GQE_ERR_INVALID_ARG;
@@ -780,17 +814,55 @@ int gqe_forward_host(const gqe_dims* d, const void* x_host, const void* Wq, cons
                      void* stream) {
   GQE_TRY(check_dims(d));
   if (x_host == nullptr || y_host == nullptr) return GQE_ERR_INVALID_ARG;
+  GQE_TRY(check_ptrs({Wq, Wk, Wv, Wr, Wo}));
+  if (br && !aligned16(br)) return GQE_ERR_INVALID_ARG;
   GQE_TRY(check_ws(ws, ws_bytes, gqe_workspace_bytes(d, GQE_OP_FORWARD_HOST)));
+  GQE_TRY(check_device());
   Carver c{static_cast<uint8_t*>(ws)};
   carve_forward(c, d);
-  const size_t xbytes = (size_t)d->B * d->T * d->D * 2;
-  void* x_dev = c.take<__nv_bfloat16>((size_t)d->B * d->T * d->D);
-  void* y_dev = c.take<__nv_bfloat16>((size_t)d->B * d->T * d->D);
+  uint8_t* x_dev = reinterpret_cast<uint8_t*>(c.take<__nv_bfloat16>((size_t)d->B * d->T * d->D));
+  uint8_t* y_dev = reinterpret_cast<uint8_t*>(c.take<__nv_bfloat16>((size_t)d->B * d->T * d->D));
+  const uint8_t* xh = static_cast<const uint8_t*>(x_host);
+  uint8_t* yh = static_cast<uint8_t*>(y_host);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  GQE_TRY(cuda_status(cudaMemcpyAsync(x_dev, x_host, xbytes, cudaMemcpyHostToDevice, st)));
-  GQE_TRY(gqe_forward(d, x_dev, Wq, Wk, Wv, Wr, br, Wo, y_dev, ws, ws_bytes, stream));
-  GQE_TRY(cuda_status(cudaMemcpyAsync(y_host, y_dev, xbytes, cudaMemcpyDeviceToHost, st)));
-  return GQE_OK;
+  const size_t seq_bytes = (size_t)d->T * d->D * 2;
+  const int nch = std::min(d->B, kHostChunks);
+  if (nch == 1) {
+    GQE_TRY(cuda_status(cudaMemcpyAsync(x_dev, xh, d->B * seq_bytes, cudaMemcpyHostToDevice, st)));
+    GQE_TRY(do_forward(d, GQE_COMBINE_SLOT, x_dev, Wq, Wk, Wv, Wr, br, Wo, y_dev, ws, st));
+    return cuda_status(cudaMemcpyAsync(yh, y_dev, d->B * seq_bytes, cudaMemcpyDeviceToHost, st));
+  }
+  // Sequences are independent: chunk ci (whole sequences) is copied in on
+  // the h2d stream, projected and attended on `stream`, and copied out on
+  // the d2h stream, so the two copy directions and the forward passes of
+  // different chunks overlap. The forward passes share the workspace in
+  // stream order; x_dev and y_dev lie past the whole batch's forward
+  // workspace.
+  std::lock_guard<std::mutex> lock(g_pipe_mutex);
+  HostPipe* hp = nullptr;
+  GQE_TRY(host_pipe(&hp));
+  GQE_TRY(cuda_status(cudaEventRecord(hp->start, st)));  // earlier work on `stream` may still read x_dev
+  GQE_TRY(cuda_status(cudaStreamWaitEvent(hp->h2d, hp->start, 0)));
+  int rc = GQE_OK;
+  for (int ci = 0; ci < nch && rc == GQE_OK; ++ci) {
+    const int b0 = (int)((long long)d->B * ci / nch), b1 = (int)((long long)d->B * (ci + 1) / nch);
+    gqe_dims dc = *d;
+    dc.B = b1 - b0;
+    const size_t off = (size_t)b0 * seq_bytes, bytes = (size_t)dc.B * seq_bytes;
+    if ((rc = cuda_status(cudaMemcpyAsync(x_dev + off, xh + off, bytes, cudaMemcpyHostToDevice, hp->h2d)))) break;
+    if ((rc = cuda_status(cudaEventRecord(hp->in[ci], hp->h2d)))) break;
+    if ((rc = cuda_status(cudaStreamWaitEvent(st, hp->in[ci], 0)))) break;
+    if ((rc = do_forward(&dc, GQE_COMBINE_SLOT, x_dev + off, Wq, Wk, Wv, Wr, br, Wo, y_dev + off, ws, st))) break;
+    if ((rc = cuda_status(cudaEventRecord(hp->out[ci], st)))) break;
+    if ((rc = cuda_status(cudaStreamWaitEvent(hp->d2h, hp->out[ci], 0)))) break;
+    rc = cuda_status(cudaMemcpyAsync(yh + off, y_dev + off, bytes, cudaMemcpyDeviceToHost, hp->d2h));
+  }
+  // join: `stream` continues only after every copy this call enqueued (also on error)
+  const int rj0 = cuda_status(cudaEventRecord(hp->in[0], hp->h2d));
+  const int rj1 = rj0 ? rj0 : cuda_status(cudaStreamWaitEvent(st, hp->in[0], 0));
+  const int rj2 = cuda_status(cudaEventRecord(hp->done, hp->d2h));
+  const int rj3 = rj2 ? rj2 : cuda_status(cudaStreamWaitEvent(st, hp->done, 0));
+  return rc ? rc : (rj1 ? rj1 : rj3);
 }
 
 int gqe_decode(const gqe_dims* d, const int32_t* cache_len, const void* x_new, const void* Wq, const void* Wk,
