@@ -10,6 +10,23 @@ NEAR_TIE = 1e-4          # top-k margin (logit units) under which either choice 
 REL_L2_MAX = 5e-3        # bf16 output tolerances against the oracle
 MAX_ABS_MAX = 1e-2
 
+# Per parity case: decisions checked, near ties, near ties decided the other
+# way, and the worst rel-L2 / max-abs of any bf16 tensor compared. Printed at
+# the end of the run (tests/conftest.py) so the counts reach the run's log.
+REPORT: dict = {}
+
+
+def _report(case, **kw):
+    if case is None:
+        return
+    r = REPORT.setdefault(case, {"decisions": 0, "near_ties": 0, "flipped": 0, "rel_l2": 0.0, "max_abs": 0.0,
+                                 "worst": ""})
+    for key in ("decisions", "near_ties", "flipped"):
+        r[key] += kw.get(key, 0)
+    if "rel_l2" in kw and kw["rel_l2"] >= r["rel_l2"]:
+        r["rel_l2"], r["worst"] = kw["rel_l2"], kw.get("what", "")
+    r["max_abs"] = max(r["max_abs"], kw.get("max_abs", 0.0))
+
 
 def to_dev(inp: dict) -> dict:
     return {k: v.cuda() for k, v in inp.items()}
@@ -74,15 +91,16 @@ def errors(got, want) -> dict:
             "finite": bool(np.isfinite(got).all())}
 
 
-def assert_close_bf16(got, want, what: str, rel_l2=REL_L2_MAX, max_abs=MAX_ABS_MAX) -> dict:
+def assert_close_bf16(got, want, what: str, rel_l2=REL_L2_MAX, max_abs=MAX_ABS_MAX, case=None) -> dict:
     e = errors(got, want)
+    _report(case, rel_l2=e["rel_l2"], max_abs=e["max_abs"], what=what)
     assert e["finite"], f"{what}: non-finite values"
     assert e["rel_l2"] <= rel_l2, f"{what}: rel-L2 {e['rel_l2']:.3e} > {rel_l2:.1e}"
     assert e["max_abs"] <= max_abs, f"{what}: max-abs {e['max_abs']:.3e} > {max_abs:.1e}"
     return e
 
 
-def check_selection(d, x, Wr, br, gpu_sel, rows=None) -> dict:
+def check_selection(d, x, Wr, br, gpu_sel, rows=None, case=None) -> dict:
     """Selections must equal the oracle's except on near-tie decisions
     (oracle margin < NEAR_TIE), which are accepted either way and reported."""
     x = x.cpu()
@@ -94,6 +112,7 @@ def check_selection(d, x, Wr, br, gpu_sel, rows=None) -> dict:
     differ = np.any(g != r["sel"], axis=2)
     near = r["margin"] < NEAR_TIE
     bad = differ & ~near
+    _report(case, decisions=int(differ.size), near_ties=int(near.sum()), flipped=int((differ & near).sum()))
     assert not bad.any(), f"{int(bad.sum())} selections differ with margin >= {NEAR_TIE}"
     return {"near_ties": int(near.sum()), "flipped_near_ties": int((differ & near).sum()), "oracle": r}
 

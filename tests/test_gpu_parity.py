@@ -37,7 +37,7 @@ def cases():
 def test_route_selection_and_compaction(cases, name):
     d, inp, dev, st = cases[name]
     assert st["status"] == 0
-    chk = check_selection(d, inp["x"], inp["Wr"], inp["br"], st["sel"])
+    chk = check_selection(d, inp["x"], inp["Wr"], inp["br"], st["sel"], case=name)
     r = chk["oracle"]
     same = np.all(st["sel"].numpy() == r["sel"], axis=2)
     np.testing.assert_allclose(st["w"].numpy()[same], r["w"][same], rtol=0, atol=2e-6)
@@ -57,9 +57,9 @@ def test_projection_stage(cases, name):
     full = ref.gqe_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"], inp["Wo"], d,
                            forced_sel=st["sel"].numpy())
     N = d.B * d.T
-    assert_close_bf16(st["K"], full["K"].reshape(N, d.G, 64), "K")
-    assert_close_bf16(st["V"], full["V"].reshape(N, d.G, 64), "V")
-    assert_close_bf16(st["Q"], full["Q"], "Q (selected experts + shared head)")
+    assert_close_bf16(st["K"], full["K"].reshape(N, d.G, 64), "K", case=name)
+    assert_close_bf16(st["V"], full["V"].reshape(N, d.G, 64), "V", case=name)
+    assert_close_bf16(st["Q"], full["Q"], "Q", case=name)
 
 
 @pytest.mark.parametrize("name", list(SMALL))
@@ -67,7 +67,7 @@ def test_attention_stage(cases, name):
     d, inp, dev, st = cases[name]
     rows = np.arange(d.B * d.T)
     want = reference_attention(d, st["Q"], st["K"], st["V"], rows)
-    assert_close_bf16(st["O"], want, "O")
+    assert_close_bf16(st["O"], want, "O", case=name)
 
 
 @pytest.mark.parametrize("name", list(SMALL))
@@ -75,7 +75,7 @@ def test_combine_stage(cases, name):
     d, inp, dev, st = cases[name]
     A = ref.combine(f64(st["O"]), f64(st["w"]), d)
     want = A @ f64(inp["Wo"])
-    assert_close_bf16(st["y"], want, "y from GPU O and w")
+    assert_close_bf16(st["y"], want, "y-combine", case=name)
 
 
 @pytest.mark.parametrize("name", list(SMALL))
@@ -87,7 +87,7 @@ def test_layer_end_to_end(cases, name):
     assert torch.equal(y.cpu(), st["y"])
     full = ref.gqe_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"], inp["Wo"], d,
                            forced_sel=st["sel"].numpy())
-    assert_close_bf16(y, full["y"], "GQE y vs oracle")
+    assert_close_bf16(y, full["y"], "y", case=name)
 
 
 @pytest.mark.parametrize("name", ["tiny_b2_t256", "ragged_b3_t300", "pool4_k2_skewed_t384", "pool8_k4_t136",
@@ -97,7 +97,7 @@ def test_dense_gqa_baseline(cases, name):
     y, _, status = run_dense(d, dev)
     assert status == 0
     want = ref.gqa_dense_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wo_dense"], d)
-    assert_close_bf16(y, want["y"], "dense GQA y vs oracle")
+    assert_close_bf16(y, want["y"], "dense-y", case=name)
 
 
 def test_empty_segments_are_empty(cases):
@@ -157,7 +157,7 @@ def test_repeat_calls_are_bitwise_identical_at_the_main_shape():
 
 # ---- the workloads at full size: sampled query rows against the oracle ----
 
-def _sampled_parity(d, n_uniform, seed=0, dense=True):
+def _sampled_parity(d, n_uniform, seed=0, dense=True, case=None):
     inp = make_inputs(d, seed=0, device="cpu")
     dev = to_dev(inp)
     y, ws, status = run_forward(d, dev)
@@ -166,19 +166,19 @@ def _sampled_parity(d, n_uniform, seed=0, dense=True):
     views = gqe.forward_views(d, ws)
     sel = views["sel"].cpu()
     rows = ref.sample_rows(d.B, d.T, n_uniform=n_uniform, seed=seed)
-    chk = check_selection(d, inp["x"], inp["Wr"], inp["br"], sel, rows=rows)
+    chk = check_selection(d, inp["x"], inp["Wr"], inp["br"], sel, rows=rows, case=case)
     seg_off = views["seg_off"].cpu().numpy()
     assert seg_off[-1] == d.B * d.T * d.G * d.k
     counts = np.diff(seg_off)
     full = ref.gqe_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"], inp["Wo"], d,
                            rows=rows, forced_sel=sel.numpy()[rows])
-    e = assert_close_bf16(y.cpu()[rows], full["y"], "GQE y (sampled rows)")
+    e = assert_close_bf16(y.cpu()[rows], full["y"], "y-sampled", case=case)
     out = {"gqe": e, "near_ties": chk["near_ties"], "segments": counts}
     if dense:
         yd, _, status = run_dense(d, dev)
         assert status == 0
         want = ref.gqa_dense_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wo_dense"], d, rows=rows)
-        out["dense"] = assert_close_bf16(yd.cpu()[rows], want["y"], "dense y (sampled rows)")
+        out["dense"] = assert_close_bf16(yd.cpu()[rows], want["y"], "dense-y-sampled", case=case)
     return out
 
 
@@ -190,18 +190,19 @@ def test_main_layer_b8_t2048_full_rows():
     assert status == 0
     import moe_gqa_query_gqe_b200 as gqe
     sel = gqe.forward_views(d, ws)["sel"].cpu()
-    check_selection(d, inp["x"], inp["Wr"], inp["br"], sel)
+    check_selection(d, inp["x"], inp["Wr"], inp["br"], sel, case="main_b8_t2048")
     full = ref.gqe_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"], inp["Wo"], d,
                            forced_sel=sel.numpy())
-    assert_close_bf16(y, full["y"], "GQE y, main layer")
+    assert_close_bf16(y, full["y"], "y", case="main_b8_t2048")
 
 
 def test_long_context_t32768_sampled():
-    _sampled_parity(CONFIGS["long_b1_t32768"], n_uniform=256)
+    _sampled_parity(CONFIGS["long_b1_t32768"], n_uniform=256, case="long_b1_t32768 (sampled)")
 
 
 def test_skewed_pool4_k2_t131072_sampled():
-    out = _sampled_parity(CONFIGS["skewed_b1_t131072_m4k2"], n_uniform=128, dense=False)
+    out = _sampled_parity(CONFIGS["skewed_b1_t131072_m4k2"], n_uniform=128, dense=False,
+                          case="skewed_b1_t131072_m4k2 (sampled)")
     seg = out["segments"].reshape(8, 4)
     # expert 0 carries the +2.0 router bias: it is in the top-2 of most tokens
     assert np.all(seg[:, 0] > 0.9 * 131072)
@@ -209,4 +210,5 @@ def test_skewed_pool4_k2_t131072_sampled():
 
 @pytest.mark.slow
 def test_million_tokens_sampled():
-    _sampled_parity(CONFIGS["million_b1_t1048576"], n_uniform=96, dense=False)
+    _sampled_parity(CONFIGS["million_b1_t1048576"], n_uniform=96, dense=False,
+                    case="million_b1_t1048576 (sampled)")
