@@ -13,14 +13,15 @@
 // kernels with the B new tokens seen as one sequence of B tokens. This file
 // holds the cache-side kernels:
 //   decode_append_kernel : K/V row of the new token -> cache position L_b
-//   decode_attn_kernel   : split-K attention. CTA (split s, group g, seq b)
-//                          takes keys [s*chunk, min((s+1)*chunk, L_b+1)) for
-//                          the R = k (+1 shared in group 0) query rows of the
-//                          group: scores in shared memory (log2 domain), the
-//                          chunk's max m and sum l per row, and the partial
-//                          output sum_s 2^(score - m) V_s. CUDA cores: at
-//                          R <= 9 rows per key the tensor cores would idle;
-//                          the bound is the cache read (2 * 128 B per key).
+//   decode_attn_kernel   : split-K attention. CTA (split s, seq b) takes
+//                          keys [s*chunk, min((s+1)*chunk, L_b+1)) of all
+//                          groups (one contiguous range of the cache) for
+//                          every query row: scores in shared memory (log2
+//                          domain), the chunk's max m and sum l per row, and
+//                          the partial output sum_s 2^(score - m) V_s. CUDA
+//                          cores: at <= 9 rows per key the tensor cores would
+//                          idle; the bound is the cache read (2 * 128 B per
+//                          key and group).
 //   decode_merge_kernel  : one warp per (sequence, query slot) merges the
 //                          chunks: O = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
 #pragma once
@@ -29,8 +30,10 @@
 
 namespace gqe {
 
-constexpr int kDecChunk = 1024;    // keys per attention CTA
-constexpr int kDecThreads = 128;
+constexpr int kDecChunk = 256;    // keys per attention CTA
+constexpr int kDecThreads = 256;  // 8 warps
+constexpr int kDecWarps = kDecThreads / 32;
+constexpr int kDecUnroll = 8;     // key quads whose loads each lane keeps in flight
 
 struct DecodeParams {
   const __nv_bfloat16* Q;    // [B, Ha, 64]: slot g*k+j routed, slot G*k shared
@@ -73,171 +76,193 @@ __global__ void __launch_bounds__(256) decode_append_kernel(const DecodeParams p
   }
 }
 
+// Shared memory of decode_attn_kernel, in floats: queries q [Ha][64] (log2
+// domain), scores / probabilities sc [Ha][kDecChunk], chunk max and sum
+// ml [Ha][2], per-warp partial outputs red [kDecWarps][rmax][64].
+__host__ __device__ inline int dec_smem_floats(int Ha, int rmax) {
+  return Ha * 64 + Ha * kDecChunk + Ha * 2 + kDecWarps * rmax * 64;
+}
+
+// Query slot of row j of group g: the group's k selected experts, then (group
+// 0 only) the shared head.
+__device__ __forceinline__ int dec_slot(const DecodeParams& p, int g, int j) {
+  return j < p.k ? g * p.k + j : p.G * p.k;
+}
+
+// CTA (split s, sequence b): keys [s*kDecChunk, min((s+1)*kDecChunk, L_b+1))
+// of ALL groups, so the CTA streams one contiguous range of the cache
+// ([key][group][64] rows). Warp w takes groups g = w % gs + gs*t (gs =
+// min(G, 8)) and, when G < 8, every (8/G)-th quad of keys. A quad is 4 keys;
+// lane l reads 16 bytes (dims 8c..8c+7, c = l % 8) of key l / 8 of the quad,
+// so one warp load moves four whole 128-byte rows. KR bounds the rows of a
+// group (k, plus the shared head in group 0).
+template <int KR>
 __global__ void __launch_bounds__(kDecThreads) decode_attn_kernel(const DecodeParams p) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ float dsm[];
-  const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int s = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int R = p.k + (g == 0 ? 1 : 0);
-  float* q = dsm;                       // [rmax][64], scaled to the log2 domain
-  float* sc = q + p.rmax * 64;          // [rmax][kDecChunk]
-  float* red = sc + p.rmax * kDecChunk;  // [4][rmax][64] partial outputs / [4][rmax] reductions
+  const int c = lane & 7, kq = lane >> 3;  // 16-byte piece of a row, key within the quad
+  float* q = dsm;
+  float* sc = q + p.Ha * 64;
+  float* ml = sc + p.Ha * kDecChunk;
+  float* red = ml + p.Ha * 2;
   const int L = dec_len(p, b);
-  const int nkeys = L + 1;
-  const int k0 = s * kDecChunk, k1 = min(k0 + kDecChunk, nkeys);
-  const size_t base = ((size_t)(b * p.G + g) * p.rmax) * p.nsplit + s;  // + r * nsplit
+  const int k0 = s * kDecChunk, k1 = min(k0 + kDecChunk, L + 1);
   if (L < 0 || k0 >= k1) {
-    for (int i = tid; i < p.rmax; i += kDecThreads) {
-      p.part_ml[(base + (size_t)i * p.nsplit) * 2] = -INFINITY;
-      p.part_ml[(base + (size_t)i * p.nsplit) * 2 + 1] = 0.f;
+    for (int i = tid; i < p.G * p.rmax; i += kDecThreads) {
+      const size_t at = ((size_t)(b * p.G) * p.rmax + i) * p.nsplit + s;
+      p.part_ml[at * 2] = -INFINITY;
+      p.part_ml[at * 2 + 1] = 0.f;
     }
     return;
   }
-  for (int i = tid; i < R * 64; i += kDecThreads) {
-    const int r = i / 64, d = i % 64;
-    const int slot = r < p.k ? g * p.k + r : p.G * p.k;
-    q[i] = __bfloat162float(p.Q[((size_t)b * p.Ha + slot) * 64 + d]) * p.scale_log2;
+  const int n = k1 - k0, nq = (n + 3) >> 2;
+  const int gs = min(p.G, kDecWarps), wpg = kDecWarps / gs;  // warps per group
+  for (int i = tid; i < p.Ha * 64; i += kDecThreads)
+    q[i] = __bfloat162float(p.Q[(size_t)b * p.Ha * 64 + i]) * p.scale_log2;
+  __syncthreads();
+
+  // ---- scores: sc[slot][key] = q[slot] . K[key, group of slot] ------------------
+  for (int g = warp % gs; g < p.G; g += gs) {
+    const int R = p.k + (g == 0 ? 1 : 0);
+    float qr[KR][8];
+#pragma unroll
+    for (int j = 0; j < KR; ++j)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) qr[j][e] = j < R ? q[dec_slot(p, g, j) * 64 + 8 * c + e] : 0.f;
+    for (int qa = warp / gs; qa < nq; qa += wpg * kDecUnroll) {
+      uint4 u[kDecUnroll];
+#pragma unroll
+      for (int t = 0; t < kDecUnroll; ++t) {
+        const int i = k0 + 4 * (qa + t * wpg) + kq;
+        u[t] = i < k1 ? reinterpret_cast<const uint4*>(p.Kc + (((size_t)b * p.T + i) * p.G + g) * 64)[c]
+                      : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int t = 0; t < kDecUnroll; ++t) {
+        const int key = 4 * (qa + t * wpg) + kq;  // within the chunk
+        const uint32_t w4[4] = {u[t].x, u[t].y, u[t].z, u[t].w};
+        float kf[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          kf[2 * e] = bf16lo_to_f32(w4[e]);
+          kf[2 * e + 1] = bf16hi_to_f32(w4[e]);
+        }
+#pragma unroll
+        for (int j = 0; j < KR; ++j) {
+          if (j >= R) break;
+          float part = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) part = fmaf(qr[j][e], kf[e], part);
+          part += __shfl_xor_sync(0xffffffffu, part, 1);
+          part += __shfl_xor_sync(0xffffffffu, part, 2);
+          part += __shfl_xor_sync(0xffffffffu, part, 4);
+          if (c == 0 && key < n) sc[dec_slot(p, g, j) * kDecChunk + key] = part;
+        }
+      }
+    }
   }
   __syncthreads();
 
-  // scores: each thread takes two keys per pass (both rows' loads in flight
-  // before the math), kDecThreads * 2 keys per pass over the chunk
-  float mloc[9];
+  // ---- per row: chunk max, 2^(score - max), their sum ---------------------------
+  for (int r = warp; r < p.Ha; r += kDecWarps) {
+    float* row = sc + r * kDecChunk;
+    float m = -INFINITY;
+    for (int i = lane; i < n; i += 32) m = fmaxf(m, row[i]);
 #pragma unroll
-  for (int r = 0; r < 9; ++r) mloc[r] = -INFINITY;
-  for (int i0 = k0 + tid; i0 < k1; i0 += 2 * kDecThreads) {
-    const int i1 = i0 + kDecThreads;
-    uint4 u[2][8];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int i = h ? i1 : i0;
-      if (i < k1) {
-        const uint4* kp = reinterpret_cast<const uint4*>(p.Kc + (((size_t)b * p.T + i) * p.G + g) * 64);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) u[h][c] = kp[c];
-      }
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float l = 0.f;
+    for (int i = lane; i < n; i += 32) {
+      const float e = exp2f(row[i] - m);
+      row[i] = e;
+      l += e;
     }
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int i = h ? i1 : i0;
-      if (i >= k1) break;
-      float kv[64];
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) {
+      ml[r * 2] = m;
+      ml[r * 2 + 1] = l;
+    }
+  }
+  __syncthreads();
+
+  // ---- P.V: partial output of every row over this chunk -------------------------
+  for (int g = warp % gs; g < p.G; g += gs) {
+    const int R = p.k + (g == 0 ? 1 : 0);
+    float acc[KR][8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint32_t w4[4] = {u[h][c].x, u[h][c].y, u[h][c].z, u[h][c].w};
+    for (int j = 0; j < KR; ++j)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
+    for (int qa = warp / gs; qa < nq; qa += wpg * kDecUnroll) {
+      uint4 u[kDecUnroll];
+#pragma unroll
+      for (int t = 0; t < kDecUnroll; ++t) {
+        const int i = k0 + 4 * (qa + t * wpg) + kq;
+        u[t] = i < k1 ? reinterpret_cast<const uint4*>(p.Vc + (((size_t)b * p.T + i) * p.G + g) * 64)[c]
+                      : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int t = 0; t < kDecUnroll; ++t) {
+        const int key = 4 * (qa + t * wpg) + kq;
+        const uint32_t w4[4] = {u[t].x, u[t].y, u[t].z, u[t].w};
+        float vf[8];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          kv[c * 8 + 2 * e] = bf16lo_to_f32(w4[e]);
-          kv[c * 8 + 2 * e + 1] = bf16hi_to_f32(w4[e]);
+          vf[2 * e] = bf16lo_to_f32(w4[e]);
+          vf[2 * e + 1] = bf16hi_to_f32(w4[e]);
+        }
+#pragma unroll
+        for (int j = 0; j < KR; ++j) {
+          if (j >= R) break;
+          const float pr = key < n ? sc[dec_slot(p, g, j) * kDecChunk + key] : 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[j][e] = fmaf(pr, vf[e], acc[j][e]);
         }
       }
+    }
+    // sum over the four keys of a quad (lanes c, c+8, c+16, c+24)
 #pragma unroll
-      for (int r = 0; r < 9; ++r) {
-        if (r >= R) break;
-        float acc = 0.f;
+    for (int j = 0; j < KR; ++j)
 #pragma unroll
-        for (int d = 0; d < 64; ++d) acc = fmaf(q[r * 64 + d], kv[d], acc);
-        sc[r * kDecChunk + (i - k0)] = acc;
-        mloc[r] = fmaxf(mloc[r], acc);
+      for (int e = 0; e < 8; ++e) {
+        acc[j][e] += __shfl_xor_sync(0xffffffffu, acc[j][e], 8);
+        acc[j][e] += __shfl_xor_sync(0xffffffffu, acc[j][e], 16);
+      }
+    if (kq == 0) {
+#pragma unroll
+      for (int j = 0; j < KR; ++j) {
+        if (j >= R) break;
+        if (wpg == 1) {
+          float* dst = p.part_o + (((size_t)(b * p.G + g) * p.rmax + j) * p.nsplit + s) * 64 + 8 * c;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) dst[e] = acc[j][e];
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) red[(warp * p.rmax + j) * 64 + 8 * c + e] = acc[j][e];
+        }
       }
     }
   }
-  // chunk max per row
-#pragma unroll
-  for (int r = 0; r < 9; ++r) {
-    if (r >= R) break;
-    float v = mloc[r];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    if (lane == 0) red[warp * p.rmax + r] = v;
-  }
-  __syncthreads();
-  float m[9], l[9];
-#pragma unroll
-  for (int r = 0; r < 9; ++r) {
-    m[r] = -INFINITY;
-    l[r] = 0.f;
-    if (r < R)
-      for (int w = 0; w < 4; ++w) m[r] = fmaxf(m[r], red[w * p.rmax + r]);
-  }
-  __syncthreads();
-  // probabilities (unnormalised) and their sum per row
-  float lloc[9];
-#pragma unroll
-  for (int r = 0; r < 9; ++r) lloc[r] = 0.f;
-  for (int i = tid; i < k1 - k0; i += kDecThreads) {
-#pragma unroll
-    for (int r = 0; r < 9; ++r) {
-      if (r >= R) break;
-      const float e = exp2f(sc[r * kDecChunk + i] - m[r]);
-      sc[r * kDecChunk + i] = e;
-      lloc[r] += e;
+  if (wpg > 1) {
+    // groups shared by several warps (G < 8): warps g, g + G, ... hold partial sums
+    __syncthreads();
+    for (int i = tid; i < p.G * p.rmax * 64; i += kDecThreads) {
+      const int g = i / (p.rmax * 64), j = (i / 64) % p.rmax, d = i % 64;
+      if (j >= p.k + (g == 0 ? 1 : 0)) continue;
+      float a = 0.f;
+      for (int t = 0; t < wpg; ++t) a += red[((g + t * gs) * p.rmax + j) * 64 + d];
+      p.part_o[(((size_t)(b * p.G + g) * p.rmax + j) * p.nsplit + s) * 64 + d] = a;
     }
   }
-#pragma unroll
-  for (int r = 0; r < 9; ++r) {
-    if (r >= R) break;
-    float v = lloc[r];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0) red[warp * p.rmax + r] = v;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int r = 0; r < 9; ++r)
-    if (r < R)
-      for (int w = 0; w < 4; ++w) l[r] += red[w * p.rmax + r];
-  __syncthreads();
-  // P.V: warp w takes keys k0+w, k0+w+4, ... (32 rows per batch); lane owns
-  // dims 2*lane, 2*lane+1
-  float o0[9], o1[9];
-#pragma unroll
-  for (int r = 0; r < 9; ++r) o0[r] = o1[r] = 0.f;
-  for (int i0 = k0 + warp; i0 < k1; i0 += 4 * 32) {
-    uint32_t v2[32];  // 32 V rows per warp in flight
-#pragma unroll
-    for (int u = 0; u < 32; ++u) {
-      const int i = i0 + 4 * u;
-      v2[u] = i < k1 ? reinterpret_cast<const uint32_t*>(p.Vc + (((size_t)b * p.T + i) * p.G + g) * 64)[lane] : 0u;
-    }
-#pragma unroll
-    for (int u = 0; u < 32; ++u) {
-      const int i = i0 + 4 * u;
-      if (i >= k1) break;
-      const float v0 = bf16lo_to_f32(v2[u]), v1 = bf16hi_to_f32(v2[u]);
-#pragma unroll
-      for (int r = 0; r < 9; ++r) {
-        if (r >= R) break;
-        const float pr = sc[r * kDecChunk + (i - k0)];
-        o0[r] = fmaf(pr, v0, o0[r]);
-        o1[r] = fmaf(pr, v1, o1[r]);
-      }
-    }
-  }
-#pragma unroll
-  for (int r = 0; r < 9; ++r) {
-    if (r >= R) break;
-    red[(warp * p.rmax + r) * 64 + 2 * lane] = o0[r];
-    red[(warp * p.rmax + r) * 64 + 2 * lane + 1] = o1[r];
-  }
-  __syncthreads();
-  for (int i = tid; i < R * 64; i += kDecThreads) {
-    const int r = i / 64, d = i % 64;
-    float acc = 0.f;
-    for (int w = 0; w < 4; ++w) acc += red[(w * p.rmax + r) * 64 + d];
-    p.part_o[(base + (size_t)r * p.nsplit) * 64 + d] = acc;
-  }
-  if (tid < R) {
-    float mr = 0.f, lr = 0.f;
-#pragma unroll
-    for (int r = 0; r < 9; ++r)
-      if (r == tid) {
-        mr = m[r];
-        lr = l[r];
-      }
-    p.part_ml[(base + (size_t)tid * p.nsplit) * 2] = mr;
-    p.part_ml[(base + (size_t)tid * p.nsplit) * 2 + 1] = lr;
+  for (int i = tid; i < p.G * p.rmax; i += kDecThreads) {
+    const int g = i / p.rmax, j = i % p.rmax;
+    const size_t at = ((size_t)(b * p.G + g) * p.rmax + j) * p.nsplit + s;
+    const bool used = j < p.k + (g == 0 ? 1 : 0);
+    p.part_ml[at * 2] = used ? ml[dec_slot(p, g, j) * 2] : -INFINITY;
+    p.part_ml[at * 2 + 1] = used ? ml[dec_slot(p, g, j) * 2 + 1] : 0.f;
   }
 }
 

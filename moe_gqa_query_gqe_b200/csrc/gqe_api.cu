@@ -625,6 +625,24 @@ int host_pipe(HostPipe** out) {
   return GQE_OK;
 }
 
+// decode_attn_kernel instantiated for the rows of a group (k, plus the shared
+// head in group 0): one CTA per (chunk of keys, sequence).
+template <int KR>
+int launch_decode_attn_kr(const DecodeParams& dp, cudaStream_t st) {
+  const int smem = dec_smem_floats(dp.Ha, dp.rmax) * 4;
+  GQE_TRY(set_smem(decode_attn_kernel<KR>, smem));
+  return launch_pdl(decode_attn_kernel<KR>, dim3(dp.nsplit, dp.B), dim3(kDecThreads), smem, st, dp);
+}
+int launch_decode_attn(const DecodeParams& dp, cudaStream_t st) {
+  switch (dp.k) {
+    case 1: return launch_decode_attn_kr<2>(dp, st);
+    case 2: return launch_decode_attn_kr<3>(dp, st);
+    case 4: return launch_decode_attn_kr<5>(dp, st);
+    case 8: return launch_decode_attn_kr<9>(dp, st);
+    default: return GQE_ERR_UNSUPPORTED;
+  }
+}
+
 int check_ptrs(std::initializer_list<const void*> ps) {
   for (const void* p : ps)
     if (p == nullptr || !aligned16(p)) return GQE_ERR_INVALID_ARG;
@@ -911,9 +929,7 @@ int gqe_decode(const gqe_dims* d, const int32_t* cache_len, const void* x_new, c
   const long long pieces = (long long)d->B * d->G * 64 / 8 * 2;
   GQE_TRY(launch_pdl(decode_append_kernel, dim3((unsigned)std::min<long long>(cdiv(pieces, 256), 4096)), dim3(256), 0,
                      st, dp));
-  const int attn_smem = f.rmax * (64 + kDecChunk + 4 * 64) * 4;
-  GQE_TRY(set_smem(decode_attn_kernel, attn_smem));
-  GQE_TRY(launch_pdl(decode_attn_kernel, dim3(f.nsplit, d->G, d->B), dim3(kDecThreads), attn_smem, st, dp));
+  GQE_TRY(launch_decode_attn(dp, st));
   const long long warps = (long long)d->B * dp.Ha;
   GQE_TRY(launch_pdl(decode_merge_kernel, dim3((unsigned)cdiv(warps * 32, 256)), dim3(256), 0, st, dp));
   return do_combine(&t, f.O, w, Wo, y, f.A, st);
