@@ -25,10 +25,11 @@ constexpr int kMaxRowSets = 72;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct AttnRowSet {
-  int h0;   // first Q/O head of the set
+  int h0;   // first Q head of the set
   int rr;   // rows per token (1, 2, 4 or 8)
   int kvg;  // KV head the set attends
   int tm;   // which Q tensor map (box height rr)
+  int ob;   // first 64-wide output block of the set in a token's output row
 };
 
 }  // namespace gqe

@@ -54,7 +54,15 @@ struct Attn2Params {
   CUtensorMap tmQ[2];  // [B*T, Ha, 64] boxes (64, rr, 128/rr)
   CUtensorMap tmK;     // [B*T, G, 64] box (64, 1, 128)
   CUtensorMap tmV;
-  __nv_bfloat16* O;    // [B*T, Ha, 64]
+  __nv_bfloat16* O;    // [B*T, o_ld, 64]: row r of a set goes to block ob + r % rr
+  // Fused output construction (GQE with k > 1): when w is set, the routed
+  // sets also write each token's slot sum_j w[n,g,j] O[n,g*k+j] to block
+  // slot_blk0 + g, so O is the whole operand A = [concat | slots | shared]
+  // of the output projection.
+  const float* w;      // [B*T, G, k] renormalised weights, or null
+  int slot_blk0;       // G*k
+  int G;
+  int o_ld;            // 64-wide blocks per token row of O
   int B, T, Ha, nrs, npairs_max, total_items;
   float scale_log2;    // log2(e) / sqrt(dh)
   AttnRowSet rs[kMaxRowSets];
@@ -419,30 +427,64 @@ __global__ void __launch_bounds__(kA2Threads, 1) attn2_fwd_kernel(const __grid_c
       }
       if (!ok) break;
       // ---- epilogue: O / l -> bf16 ------------------------------------------------
+      const int rr = it.rs.rr, jslot = row % rr;
+      const size_t n_tok = (size_t)it.b * p.T + (tok < p.T ? tok : 0);
+      // slot weights of this row's token (fused output construction)
+      const bool slot = p.w != nullptr && it.rs.ob < p.slot_blk0;
+      float wj[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        wj[i] = (slot && i < rr && tok < p.T) ? p.w[(n_tok * p.G + it.rs.kvg) * rr + i] : 0.f;
       const bool w_ok = mbar_wait(&pv_done[t], (cnt - 1) & 1, abort_flag);
       if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
       tc_fence_after();
       const float inv = 1.f / l_run;
-      __nv_bfloat16* dst =
-          (tok < p.T) ? p.O + ((size_t)(it.b * p.T + tok) * p.Ha + it.rs.h0 + (row % it.rs.rr)) * 64 : nullptr;
+      __nv_bfloat16* dst = (tok < p.T) ? p.O + (n_tok * p.o_ld + it.rs.ob + jslot) * 64 : nullptr;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t o[32];
         tmem_ld32(tm_o + h * 32, o);
-        if (dst) {
-          uint32_t pk[16];
+        uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+        if (dst) {
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             st_global_v4(dst + h * 32 + i * 8, pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+        if (slot) {
+          // The token's rr rows are lanes base .. base+rr-1 of this warp.
+          // Every one of them sums the rr bf16 outputs (fp32, in slot
+          // order, as the separate combine kernel does); the first stores.
+          const int base = lane - jslot;
+          float acc[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) acc[c] = 0.f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if (i >= rr) break;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const uint32_t u = __shfl_sync(0xffffffffu, pk[c], base + i);
+              acc[2 * c] = fmaf(wj[i], bf16lo_to_f32(u), acc[2 * c]);
+              acc[2 * c + 1] = fmaf(wj[i], bf16hi_to_f32(u), acc[2 * c + 1]);
+            }
+          }
+          if (dst && jslot == 0) {
+            __nv_bfloat16* sd = p.O + (n_tok * p.o_ld + p.slot_blk0 + it.rs.kvg) * 64 + h * 32;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              st_global_v4(sd + i * 8, pack_bf16x2(acc[8 * i], acc[8 * i + 1]), pack_bf16x2(acc[8 * i + 2], acc[8 * i + 3]),
+                           pack_bf16x2(acc[8 * i + 4], acc[8 * i + 5]), pack_bf16x2(acc[8 * i + 6], acc[8 * i + 7]));
+          }
         }
       }
       tc_fence_before();
     }
   }
 
+  __syncwarp();  // lanes that skipped a single-lane role wait for it, so every warp arrives whole
   tc_fence_before();
   __syncthreads();
   if (*abort_flag) {

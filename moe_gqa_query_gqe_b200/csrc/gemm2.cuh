@@ -267,6 +267,7 @@ __global__ void __launch_bounds__(G2Cfg<BN, STAGES>::kThreads, 1)
     }
   }
 
+  __syncwarp();  // lanes that skipped a single-lane role wait for it, so every warp arrives whole
   tc_fence_before();
   __syncthreads();
   if (*abort_flag) {

@@ -374,6 +374,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const unsigned long long t0 = globaltimer_ns();
     while (globaltimer_ns() - t0 < 100000ull) {}
   }
+  __syncwarp();  // lanes that skipped a single-lane role wait for it, so every warp arrives whole
   cluster_sync();  // no CTA leaves while its peer's MMAs or arrivals may still reach it
   if (warp == 1) {
     tc_fence_after();

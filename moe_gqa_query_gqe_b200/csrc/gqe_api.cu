@@ -485,9 +485,12 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
-// Persistent two-tile attention (attn2.cuh).
+// Persistent two-tile attention (attn2.cuh). With slot_w set (GQE, k > 1),
+// O is the output projection's operand A [N, G*k + G + 1, 64]: the routed
+// rows in their concatenation blocks, each token's per-group slot (weights
+// slot_w) in blocks G*k .. G*k+G-1, the shared head in the last block.
 int do_attn2(const gqe_dims* d, const void* Q, int Hq, const void* K, const void* V, void* O, bool dense,
-             bool shared, cudaStream_t st) {
+             bool shared, cudaStream_t st, const float* slot_w = nullptr) {
   const long long N = (long long)d->B * d->T;
   Attn2Params p;
   memset(&p, 0, sizeof(p));
@@ -500,9 +503,13 @@ int do_attn2(const gqe_dims* d, const void* Q, int Hq, const void* K, const void
   p.B = d->B;
   p.T = d->T;
   p.Ha = Hq;
+  p.w = slot_w;
+  p.G = d->G;
+  p.slot_blk0 = d->G * d->k;
+  p.o_ld = slot_w ? d->G * d->k + d->G + 1 : Hq;
   int nrs = 0;
-  for (int g = 0; g < d->G; ++g) p.rs[nrs++] = AttnRowSet{g * rr, rr, g, 0};
-  if (shared) p.rs[nrs++] = AttnRowSet{d->G * d->k, 1, 0, 1};
+  for (int g = 0; g < d->G; ++g) p.rs[nrs++] = AttnRowSet{g * rr, rr, g, 0, g * rr};
+  if (shared) p.rs[nrs++] = AttnRowSet{d->G * d->k, 1, 0, 1, slot_w ? d->G * d->k + d->G : d->G * d->k};
   p.nrs = nrs;
   p.npairs_max = (int)cdiv((long long)d->T * rr, 256);
   const long long items = (long long)p.npairs_max * d->B * nrs;
@@ -800,6 +807,13 @@ int do_forward(const gqe_dims* d, int mode, const void* x, const void* Wq, const
   GQE_TRY(launch_gemm_pair(p, dense_tiles + route_tiles, st));
   GQE_TRY(route_finish(d, f.sel, f.seg_off, f.seg_tok, f.row_map, f.route, st));
   GQE_TRY(do_qgather(d, x, Wq, f.sel, f.seg_off, f.seg_tok, f.Q, st));
+  if (mode == GQE_COMBINE_SLOT && d->k > 1) {
+    // the attention writes A itself (concatenation, per-group slots, shared
+    // head), then y = A Wo: no separate combine pass over O
+    GQE_TRY(do_attn2(d, f.Q, d->G * d->k + 1, f.K, f.V, f.A, false, true, st, f.w));
+    const DenseSeg seg = {Wo, d->D, 0, d->D, y, (long long)d->D, 0};
+    return gemm_dense(f.A, (long long)d->B * d->T, combine_cols(d, GQE_COMBINE_SLOT), &seg, 1, st);
+  }
   GQE_TRY(do_attn2(d, f.Q, d->G * d->k + 1, f.K, f.V, f.O, false, shared, st));
   if (mode == GQE_COMBINE_SLOT) return do_combine(d, f.O, f.w, Wo, y, f.A, st);
   return do_combine_variant(d, mode, f.O, f.w, p_sel, Wo, y, A2, st);

@@ -34,15 +34,17 @@ constexpr int kQgMaxK = 1024;  // resident weight slice: K x 64 bf16 <= 128 KB
 constexpr int kQgBarBytes = 512;
 
 // Shared memory: `stages` A stages of 16 KB, the resident weight slice (nk
-// boxes of 8 KB), barriers, the tile prefix over the segments. As many
-// stages as fit (the gather is bound by the bytes in flight).
+// boxes of 8 KB), barriers, the tile prefix over the segments and a copy of
+// the segment offsets. As many stages as fit (the gather is bound by the
+// bytes in flight).
 struct QgLayout {
   int stages, nk;
   __host__ __device__ int a_off(int s) const { return s * 16384; }
   __host__ __device__ int b_off() const { return stages * 16384; }
   __host__ __device__ int bar_off() const { return b_off() + nk * 8192; }
   __host__ __device__ int prefix_off() const { return bar_off() + kQgBarBytes; }
-  __host__ __device__ int bytes(int nsegs) const { return prefix_off() + (nsegs + 1) * 4 + 1024; }
+  __host__ __device__ int segoff_off(int nsegs) const { return prefix_off() + (nsegs + 1) * 4; }
+  __host__ __device__ int bytes(int nsegs) const { return segoff_off(nsegs) + (nsegs + 1) * 4 + 1024; }
 };
 
 __global__ void __launch_bounds__(kQgThreads, 1) qgather_kernel(const __grid_constant__ GemmParams p, int stages) {
@@ -61,16 +63,22 @@ __global__ void __launch_bounds__(kQgThreads, 1) qgather_kernel(const __grid_con
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(b_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* s_prefix = reinterpret_cast<int*>(smem + L.prefix_off());
+  int* s_segoff = reinterpret_cast<int*>(smem + L.segoff_off(p.nsegs_q));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int GM = p.G * p.M;
 
+  // Segment offsets into shared memory, all loads in flight at once (the
+  // copiers and the epilogue then find every tile's rows without a
+  // dependent global load at the tile boundary).
+  for (int s = tid; s <= p.nsegs_q; s += kQgThreads) s_segoff[s] = p.seg_off[s];
+  __syncthreads();
   if (warp == 0) {
     // tile prefix over the expert segments: s_prefix[s] = tiles before segment s
     int before = 0;
     for (int s0 = 0; s0 < p.nsegs_q; s0 += 32) {
       const int s = s0 + lane;
-      const int len = s < p.nsegs_q ? p.seg_off[s + 1] - p.seg_off[s] : 0;
+      const int len = s < p.nsegs_q ? s_segoff[s + 1] - s_segoff[s] : 0;
       const int nt = (len + kGemmBM - 1) / kGemmBM;
       int incl = nt;
 #pragma unroll
@@ -182,8 +190,8 @@ __global__ void __launch_bounds__(kQgThreads, 1) qgather_kernel(const __grid_con
     uint32_t tcount = 0;
     for (int tile = first; tile < last; ++tile, ++tcount) {
       const int seg = seg_of(tile);
-      const int row0 = p.seg_off[seg] + (tile - s_prefix[seg]) * kGemmBM;
-      const int row_end = min(p.seg_off[seg + 1], p.seg_off[p.nsegs_q]);
+      const int row0 = s_segoff[seg] + (tile - s_prefix[seg]) * kGemmBM;
+      const int row_end = min(s_segoff[seg + 1], s_segoff[p.nsegs_q]);
       // destination row first: its dependent loads overlap the accumulation
       __nv_bfloat16* dst_row = nullptr;
       const int ci = row0 + row;
@@ -233,8 +241,8 @@ __global__ void __launch_bounds__(kQgThreads, 1) qgather_kernel(const __grid_con
     // loaded values until the tile boundary, so the loads do not stall here.
     auto fetch_rows = [&](int tile, int (&tk)[4]) {
       const int seg = seg_of(tile);
-      const int row0 = p.seg_off[seg] + (tile - s_prefix[seg]) * kGemmBM;
-      const int row_end = min(p.seg_off[seg + 1], p.seg_off[p.nsegs_q]);
+      const int row0 = s_segoff[seg] + (tile - s_prefix[seg]) * kGemmBM;
+      const int row_end = min(s_segoff[seg + 1], s_segoff[p.nsegs_q]);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int r = i * 32 + (ct >> 3);
@@ -275,6 +283,7 @@ __global__ void __launch_bounds__(kQgThreads, 1) qgather_kernel(const __grid_con
     asm volatile("cp.async.wait_all;" ::: "memory");  // nothing may be in flight when the CTA exits
   }
 
+  __syncwarp();  // lanes that skipped a single-lane role wait for it, so every warp arrives whole
   tc_fence_before();
   __syncthreads();
   if (*abort_flag) {
