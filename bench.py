@@ -588,9 +588,11 @@ def main():
         return g
 
     # kernels launched per forward step: K/V + shared-query + router pair GEMM,
-    # scan, compaction, selected-query gather, attention, Wo (+ the combine
-    # build when k > 1)
-    launches_per_step = 6 + (0 if d.k == 1 else 1)
+    # routing scan and compaction (one launch when the per-chunk counts fit a
+    # block's shared memory, else two), selected-query gather, attention
+    # (which also builds the output operand when k > 1), Wo
+    n_counts = d.B * d.G * d.M * ((d.T + 127) // 128)
+    launches_per_step = 4 + (1 if n_counts <= 4096 else 2)
 
     def barrier():
         if world > 1:

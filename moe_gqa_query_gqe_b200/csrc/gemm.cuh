@@ -51,6 +51,11 @@ struct GemmParams {
   float* r_p;          // [B*T, G, k] in-group probabilities of the selected experts, or null
   int32_t* r_counts;   // [B][nch][G*M]
   int r_B, r_T, r_nch;
+  // Router merged into a dense segment's tiles instead of separate routing
+  // tiles: columns 64..127 of that segment's 128-column tiles are the router
+  // logits (B columns from tmR), decided in the same epilogue. Needs every
+  // 128-row block to be one chunk of one sequence (T % 128 == 0). -1: none.
+  int r_merge_seg;
   // A column remap for the k = 1 combine: A = [O_routed | O_routed | O_shared]
   // read straight from O ([N, (G+1)*64]); 0 disables the remap
   int amap_G;

@@ -214,7 +214,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&p.tmA);
     for (int s = 0; s < p.nseg; ++s) tma_prefetch_desc(&p.tmB[s]);
-    if (p.r_tile0 < total_tiles) tma_prefetch_desc(&p.tmR);
+    if (p.r_tile0 < total_tiles || p.r_merge_seg >= 0) tma_prefetch_desc(&p.tmR);
   }
   tc_fence_before();
   cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
@@ -231,8 +231,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const PairTile t = pair_decode(p, tile);
         const int half = t.nvalid / 2;  // columns of B this CTA holds
         const int nbox = half / 64;
-        const bool rt = t.seg < 0;
-        const int b_col = rt ? (int)rank * half : p.seg[t.seg].b_col0 + t.n0 + (int)rank * half;
+        // routing tile, or the odd CTA's half of a tile carrying the router
+        const bool rt = t.seg < 0 || (t.seg == p.r_merge_seg && rank == 1);
+        const int b_col = t.seg < 0 ? (int)rank * half : (rt ? 0 : p.seg[t.seg].b_col0 + t.n0 + (int)rank * half);
         const CUtensorMap* tmb = rt ? &p.tmR : &p.tmB[t.seg];
         const int a_row = t.m0 + (int)rank * 128;
         for (int kb = 0; kb < nk; ++kb, ++it) {
@@ -307,26 +308,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       const bool ok = mbar_wait(&acc_full[a], (tcount >> 1) & 1, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
+      // routing decisions of this CTA's 128 tokens (chunk c of sequence b)
+      // from the logits at TMEM column tm
+      auto route = [&](uint32_t tm, int b, int c) {
+        if (p.r_p == nullptr) {
+          switch (p.M) {
+            case 1: pair_route_epilogue<1, false>(p, tm, b, c, q, lane, s_tot); break;
+            case 2: pair_route_epilogue<2, false>(p, tm, b, c, q, lane, s_tot); break;
+            case 4: pair_route_epilogue<4, false>(p, tm, b, c, q, lane, s_tot); break;
+            default: pair_route_epilogue<8, false>(p, tm, b, c, q, lane, s_tot); break;
+          }
+        } else {  // the weighted-concatenation variant also writes the probabilities
+          switch (p.M) {
+            case 1: pair_route_epilogue<1, true>(p, tm, b, c, q, lane, s_tot); break;
+            case 2: pair_route_epilogue<2, true>(p, tm, b, c, q, lane, s_tot); break;
+            case 4: pair_route_epilogue<4, true>(p, tm, b, c, q, lane, s_tot); break;
+            default: pair_route_epilogue<8, true>(p, tm, b, c, q, lane, s_tot); break;
+          }
+        }
+      };
       if (t.seg < 0) {
         const uint32_t tm = tmem_base + a * kPairBN + (static_cast<uint32_t>(q * 32) << 16);
         const int c = t.n0 * 2 + (int)rank;  // this CTA's chunk of 128 tokens
-        if (c < p.r_nch) {
-          if (p.r_p == nullptr) {
-            switch (p.M) {
-              case 1: pair_route_epilogue<1, false>(p, tm, t.rb, c, q, lane, s_tot); break;
-              case 2: pair_route_epilogue<2, false>(p, tm, t.rb, c, q, lane, s_tot); break;
-              case 4: pair_route_epilogue<4, false>(p, tm, t.rb, c, q, lane, s_tot); break;
-              default: pair_route_epilogue<8, false>(p, tm, t.rb, c, q, lane, s_tot); break;
-            }
-          } else {  // the weighted-concatenation variant also writes the probabilities
-            switch (p.M) {
-              case 1: pair_route_epilogue<1, true>(p, tm, t.rb, c, q, lane, s_tot); break;
-              case 2: pair_route_epilogue<2, true>(p, tm, t.rb, c, q, lane, s_tot); break;
-              case 4: pair_route_epilogue<4, true>(p, tm, t.rb, c, q, lane, s_tot); break;
-              default: pair_route_epilogue<8, true>(p, tm, t.rb, c, q, lane, s_tot); break;
-            }
-          }
-        }
+        if (c < p.r_nch) route(tm, t.rb, c);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acce_c + 8 * a);
@@ -360,6 +364,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           bulk_commit();
         }
         ++nstore;
+      }
+      if (t.seg == p.r_merge_seg) {
+        // columns 64..127 are this CTA's tokens' router logits (one chunk)
+        const int row0 = t.m0 + (int)rank * 128;
+        if (row0 < p.rows) route(tm + 64, row0 / p.r_T, (row0 % p.r_T) / kRouteChunk);
       }
       tc_fence_before();
       __syncwarp();

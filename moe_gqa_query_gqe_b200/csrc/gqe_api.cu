@@ -238,6 +238,7 @@ int dense_params(GemmParams& p, const void* A, long long rows, int K, const Dens
   p.K = K;
   *tiles = nt > 0 ? cdiv(rows, kPairBM) * nt : 0;
   p.r_tile0 = 0x7fffffff;
+  p.r_merge_seg = -1;
   return GQE_OK;
 }
 
@@ -406,9 +407,16 @@ int route_finish(const gqe_dims* d, int32_t* sel, int32_t* seg_off, int32_t* seg
   rp.k = d->k;
   rp.nch = (int)cdiv(d->T, kRouteChunk);
   const int nseg = d->B * d->G * d->M;
-  GQE_TRY(launch_pdl(route_scan_kernel, dim3(1), dim3(1024), nseg * 4, st, rp));
   const long long rows = (long long)d->B * d->T * d->G * d->k;
   const long long blocks = std::min<long long>(cdiv(rows, 256), (long long)sm_count() * 8);
+  const long long ncnt = (long long)nseg * rp.nch;
+  if (ncnt <= kRouteFusedMax) {
+    // counts small enough for every block to scan them itself: one launch
+    const int smem = (int)(ncnt + nseg + 1) * 4;
+    return launch_pdl(route_scan_finalize_kernel, dim3((unsigned)std::max<long long>(blocks, 1)), dim3(256), smem, st,
+                      rp);
+  }
+  GQE_TRY(launch_pdl(route_scan_kernel, dim3(1), dim3(1024), nseg * 4, st, rp));
   return launch_pdl(route_finalize_kernel, dim3((unsigned)std::max<long long>(blocks, 1)), dim3(256), 0, st, rp);
 }
 
@@ -416,6 +424,7 @@ int do_route(const gqe_dims* d, const void* x, const void* Wr, const float* br, 
              float* margin, int32_t* seg_off, int32_t* seg_tok, int32_t* row_map, RouteWs rw, cudaStream_t st) {
   GemmParams p;
   memset(&p, 0, sizeof(p));
+  p.r_merge_seg = -1;
   const long long N = (long long)d->B * d->T;
   GQE_TRY(tmap_rows(&p.tmA, x, N, d->D, d->D, kGemmBM));
   p.rows = (int)N;
@@ -444,6 +453,7 @@ int do_qgather(const gqe_dims* d, const void* x, const void* Wq, const int32_t* 
   const int wq_cols = (G * M + 1) * 64;
   GemmParams p;
   memset(&p, 0, sizeof(p));
+  p.r_merge_seg = -1;
   GQE_TRY(tmap_rows(&p.tmB[0], Wq, d->D, wq_cols, wq_cols, 64));
   GQE_TRY(tmap_rows(&p.tmA, x, N, d->D, d->D, 1));  // a valid map for the kernel's descriptor prefetch (rows are copied with cp.async)
   p.K = d->D;
@@ -540,6 +550,7 @@ int project_from_o(const gqe_dims* d, const void* O, const void* Wo, void* y, in
   p.K = KA;
   p.amap_G = d->G;
   p.r_tile0 = 0x7fffffff;
+  p.r_merge_seg = -1;
   return launch_gemm_pair(p, cdiv(N, kPairBM) * p.ntn, st);
 }
 
@@ -804,6 +815,13 @@ int do_forward(const gqe_dims* d, int mode, const void* x, const void* Wq, const
   GQE_TRY(dense_params(p, x, (long long)d->B * d->T, d->D, segs, shared ? 3 : 2, &dense_tiles));
   GQE_TRY(add_route_tiles(p, d, Wr, br, f.sel, f.w, f.margin, f.route, dense_tiles, &route_tiles));
   p.r_p = (mode == GQE_COMBINE_WEIGHTED || mode == GQE_COMBINE_GLOBAL_SLOT) ? p_sel : nullptr;
+  if (shared && d->T % kRouteChunk == 0) {
+    // the router logits fill the second half of the shared head's 128-column
+    // tiles (the same x tile), so no separate routing tiles are launched
+    p.r_merge_seg = 2;
+    p.r_tile0 = (int)dense_tiles;
+    route_tiles = 0;
+  }
   GQE_TRY(launch_gemm_pair(p, dense_tiles + route_tiles, st));
   GQE_TRY(route_finish(d, f.sel, f.seg_off, f.seg_tok, f.row_map, f.route, st));
   GQE_TRY(do_qgather(d, x, Wq, f.sel, f.seg_off, f.seg_tok, f.Q, st));

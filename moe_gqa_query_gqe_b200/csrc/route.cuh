@@ -193,4 +193,87 @@ __global__ void __launch_bounds__(256) route_finalize_kernel(const RouteParams p
   }
 }
 
+// Scan and compaction in one launch, for problems whose per-chunk counts fit
+// in shared memory (B * nch * G*M <= kRouteFusedMax). Every block rebuilds,
+// from the counts, the exclusive prefixes it needs (segment offsets over all
+// segments, chunk bases within each segment) in its own shared memory, then
+// places its (token, group, selection) items as route_finalize_kernel does;
+// block 0 also writes seg_off. The counts are a few KB, so the redundant
+// per-block scan costs less than a second launch.
+constexpr int kRouteFusedMax = 4096;
+
+__global__ void __launch_bounds__(256) route_scan_finalize_kernel(const RouteParams p) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ int sh[];
+  const int GM = p.G * p.M, Gk = p.G * p.k;
+  const int nseg = p.B * GM;
+  const int ncnt = nseg * p.nch;
+  int* s_base = sh;            // [B][nch][GM]: chunk base within its segment
+  int* s_off = sh + ncnt;      // [nseg + 1]: segment offsets
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < ncnt; i += blockDim.x) s_base[i] = p.counts[i];
+  __syncthreads();
+  // per segment (one warp each): exclusive scan over its chunks, in place
+  for (int sgi = warp; sgi < nseg; sgi += blockDim.x >> 5) {
+    const int b = sgi / GM, ge = sgi % GM;
+    int running = 0;
+    for (int c0 = 0; c0 < p.nch; c0 += 32) {
+      const int c = c0 + lane;
+      const int idx = (b * p.nch + c) * GM + ge;
+      const int v = c < p.nch ? s_base[idx] : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      if (c < p.nch) s_base[idx] = running + incl - v;
+      running += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_off[sgi] = running;  // the segment's total, scanned below
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int running = 0;
+    for (int s0 = 0; s0 < nseg; s0 += 32) {
+      const int sgi = s0 + lane;
+      const int v = sgi < nseg ? s_off[sgi] : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      if (sgi < nseg) s_off[sgi] = running + incl - v;
+      running += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) s_off[nseg] = running;
+  }
+  __syncthreads();
+  if (blockIdx.x == 0)
+    for (int i = tid; i <= nseg; i += blockDim.x) p.seg_off[i] = s_off[i];
+  const long long total = (long long)p.B * p.T * Gk;
+  for (long long i = blockIdx.x * (long long)blockDim.x + tid; i < total; i += (long long)gridDim.x * blockDim.x) {
+    const long long n = i / Gk;
+    const int g = (int)(i % Gk) / p.k;
+    const int b = (int)(n / p.T), c = (int)(n % p.T) / kRouteChunk;
+    const int packed = p.sel[i];
+    const int e = packed & 0xFF, rank = packed >> 8;
+    p.sel[i] = e;
+    if (e >= p.M || rank < 0 || rank >= kRouteChunk) {
+      flag_bounds_error();
+      continue;
+    }
+    const int ge = g * p.M + e;
+    const long long dst = (long long)s_off[b * GM + ge] + s_base[(b * p.nch + c) * GM + ge] + rank;
+    if (dst < 0 || dst >= total) {
+      flag_bounds_error();
+      continue;
+    }
+    p.seg_tok[dst] = static_cast<int32_t>(n);
+    if (p.row_map) p.row_map[i] = static_cast<int32_t>(dst);
+  }
+}
+
 }  // namespace gqe
