@@ -489,6 +489,71 @@ def long_context(names, steps: int, warmup: int, seed: int, peaks: dict, flush) 
     return out, routes
 
 
+def stage_study(workload: str, steps: int, warmup: int) -> None:
+    """Each stage entry point of the layer (route, qproj, attn, combine) on one
+    workload, called alone: one JSON line per stage with its CUDA-event time
+    (L2 flushed before each call) and its roofline (routing and the k > 1
+    combine against HBM bandwidth with their algorithmic bytes; the
+    projections, attention and Wo against the bf16 peak)."""
+    import torch
+    import moe_gqa_query_gqe_b200 as gqe
+    from gqe_inputs import CONFIGS, make_inputs
+
+    d = CONFIGS[workload]
+    inp = make_inputs(d, seed=0, device="cuda")
+    N, G, M, k = d.B * d.T, d.G, d.M, d.k
+    Ha = G * k + 1
+    sel = torch.empty(N, G, k, dtype=torch.int32, device="cuda")
+    wts = torch.empty(N, G, k, dtype=torch.float32, device="cuda")
+    margin = torch.empty(N, G, dtype=torch.float32, device="cuda")
+    seg_off = torch.empty(d.B * G * M + 1, dtype=torch.int32, device="cuda")
+    seg_tok = torch.empty(N * G * k, dtype=torch.int32, device="cuda")
+    row_map = torch.empty(N, G, k, dtype=torch.int32, device="cuda")
+    Q = torch.empty(N, Ha, 64, dtype=torch.bfloat16, device="cuda")
+    K = torch.empty(N, G, 64, dtype=torch.bfloat16, device="cuda")
+    V = torch.empty(N, G, 64, dtype=torch.bfloat16, device="cuda")
+    O = torch.empty(N, Ha, 64, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty(N, d.D, dtype=torch.bfloat16, device="cuda")
+    ws_route = gqe.workspace(d, gqe.OP_ROUTE)
+    ws_comb = gqe.workspace(d, gqe.OP_COMBINE)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    calls = {
+        "route": lambda: gqe.gqe_route(d, inp["x"], inp["Wr"], inp["br"], sel, wts, margin, seg_off, seg_tok, row_map,
+                                       ws_route),
+        "qproj": lambda: gqe.gqe_qproj(d, inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], sel, seg_off, seg_tok, Q, K, V),
+        "attention": lambda: gqe.gqe_attn(d, Q, K, V, O),
+        "combine": lambda: gqe.gqe_combine(d, O, wts, inp["Wo"], y, ws_comb),
+    }
+    peaks = load_peaks()
+    fl = flops_model(d)["gqe"]
+    Ka = (G * k + G + 1) * 64
+    for name, fn in calls.items():
+        evs = []
+        for i in range(warmup + steps):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            if i >= warmup:
+                evs.append((a, b))
+        torch.cuda.synchronize()
+        ms = sorted(a.elapsed_time(b) for a, b in evs)[len(evs) // 2]
+        line = {"study": "stages", "workload": workload, "stage": name, "us": ms * 1e3, "status": gqe.gqe_check_error()}
+        if name == "route":
+            by = 2 * N * d.D + 2 * d.D * G * M + 4 * N * G * k * 4 + 4 * N * G + 4 * (d.B * G * M + 1)
+            line.update(bound="hbm", algorithmic_bytes=by, achieved_gbs=by / (ms / 1e3) / 1e9, peak=peaks["hbm_gbs"])
+        elif name == "combine" and k > 1:
+            by = N * (Ha * 128 + G * k * 4) + N * Ka * 2 * 2 + Ka * d.D * 2 + N * d.D * 2  # O, w, A out+in, Wo, y
+            line.update(bound="hbm+tensor", algorithmic_bytes=by, achieved_gbs=by / (ms / 1e3) / 1e9,
+                        peak=peaks["hbm_gbs"], tflops=fl["wo"] / (ms / 1e3) / 1e12)
+        else:
+            flops = {"qproj": fl["q_proj"] + fl["kv_proj"], "attention": fl["attention"], "combine": fl["wo"]}[name]
+            line.update(bound="tensor", algorithmic_flops=flops, tflops=flops / (ms / 1e3) / 1e12,
+                        peak=peaks["bf16_tflops"])
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -500,8 +565,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--long", default="long_b1_t32768,million_b1_t1048576",
                     help="comma-separated long-context workloads timed after the headline (empty: none)")
-    ap.add_argument("--study", choices=["pools", "decode"],
-                    help="print the expert-pool or decode-step study lines instead of the bench line")
+    ap.add_argument("--study", choices=["pools", "decode", "stages"],
+                    help="print the expert-pool, decode-step or per-stage study lines instead of the bench line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -516,6 +581,9 @@ def main():
         return
     if args.study == "decode":
         decode_study(steps=min(args.steps, 20), warmup=args.warmup)
+        return
+    if args.study == "stages":
+        stage_study(args.workload, steps=min(args.steps, 20), warmup=args.warmup)
         return
     if args.impl == "reference":
         run_reference(args, d, rank, world)

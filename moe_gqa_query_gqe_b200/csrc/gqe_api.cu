@@ -21,6 +21,7 @@
 #include "attn2.cuh"
 #include "combine.cuh"
 #include "decode.cuh"
+#include "decode_proj.cuh"
 
 using namespace gqe;
 
@@ -411,10 +412,12 @@ int route_finish(const gqe_dims* d, int32_t* sel, int32_t* seg_off, int32_t* seg
   const long long blocks = std::min<long long>(cdiv(rows, 256), (long long)sm_count() * 8);
   const long long ncnt = (long long)nseg * rp.nch;
   if (ncnt <= kRouteFusedMax) {
-    // counts small enough for every block to scan them itself: one launch
+    // counts small enough for every block to scan them itself: one launch,
+    // one block per SM (each block scans once, then places its share)
     const int smem = (int)(ncnt + nseg + 1) * 4;
-    return launch_pdl(route_scan_finalize_kernel, dim3((unsigned)std::max<long long>(blocks, 1)), dim3(256), smem, st,
-                      rp);
+    const long long fblocks = std::min<long long>(cdiv(rows, 256), (long long)sm_count());
+    return launch_pdl(route_scan_finalize_kernel, dim3((unsigned)std::max<long long>(fblocks, 1)), dim3(1024), smem,
+                      st, rp);
   }
   GQE_TRY(launch_pdl(route_scan_kernel, dim3(1), dim3(1024), nseg * 4, st, rp));
   return launch_pdl(route_finalize_kernel, dim3((unsigned)std::max<long long>(blocks, 1)), dim3(256), 0, st, rp);
@@ -647,6 +650,12 @@ int host_pipe(HostPipe** out) {
 // head in group 0): one CTA per (chunk of keys, sequence).
 template <int KR>
 int launch_decode_attn_kr(const DecodeParams& dp, cudaStream_t st) {
+  if (dp.G <= 2 * kDecWarps) {
+    // cache rows by bulk copies through a shared-memory ring
+    const int smem = dec_ring_smem(dp.Ha, dp.rmax);
+    GQE_TRY(set_smem(decode_attn_ring_kernel<KR>, smem));
+    return launch_pdl(decode_attn_ring_kernel<KR>, dim3(dp.nsplit, dp.B), dim3(kDecThreads), smem, st, dp);
+  }
   const int smem = dec_smem_floats(dp.Ha, dp.rmax) * 4;
   GQE_TRY(set_smem(decode_attn_kernel<KR>, smem));
   return launch_pdl(decode_attn_kernel<KR>, dim3(dp.nsplit, dp.B), dim3(kDecThreads), smem, st, dp);
@@ -928,17 +937,60 @@ int gqe_decode(const gqe_dims* d, const int32_t* cache_len, const void* x_new, c
   Carver c{static_cast<uint8_t*>(ws)};
   DecodeWs f = carve_decode(c, d);
   const gqe_dims t = decode_token_dims(d);
+  const int ka_cols = (d->G * d->k + d->G + 1) * 64;
+  const bool skinny = d->B <= kSkinnyMaxTokens && skinny_proj_smem(d->B, d->D, d->G * d->M) <= 232448 &&
+                      skinny_out_smem(ka_cols) <= 232448;
+  DecodeProjParams pp;
+  memset(&pp, 0, sizeof(pp));
+  pp.x = static_cast<const __nv_bfloat16*>(x_new);
+  pp.Wq = static_cast<const __nv_bfloat16*>(Wq);
+  pp.Wk = static_cast<const __nv_bfloat16*>(Wk);
+  pp.Wv = static_cast<const __nv_bfloat16*>(Wv);
+  pp.Wr = static_cast<const __nv_bfloat16*>(Wr);
+  pp.br = br;
+  pp.cache_len = cache_len;
+  pp.Kc = static_cast<__nv_bfloat16*>(K_cache);
+  pp.Vc = static_cast<__nv_bfloat16*>(V_cache);
+  pp.Q = f.Q;
+  pp.sel = sel;
+  pp.w = w;
+  pp.margin = f.margin;
+  pp.O = f.O;
+  pp.Wo = static_cast<const __nv_bfloat16*>(Wo);
+  pp.y = static_cast<__nv_bfloat16*>(y);
+  pp.B = d->B;
+  pp.T = d->T;
+  pp.D = d->D;
+  pp.G = d->G;
+  pp.M = d->M;
+  pp.k = d->k;
+  if (skinny) {
+    // a few new tokens: routing, K/V (written straight into the caches at
+    // cache_len) and the queries as skinny products, one CTA per 64-column
+    // weight slice
+    const int GM = d->G * d->M, Ka = (d->G * d->k + d->G + 1) * 64;
+    GQE_TRY(tmap_rows(&pp.tmWq, Wq, d->D, (GM + 1) * 64, (GM + 1) * 64, kSkChunk));
+    GQE_TRY(tmap_rows(&pp.tmWk, Wk, d->D, d->G * 64, d->G * 64, kSkChunk));
+    GQE_TRY(tmap_rows(&pp.tmWv, Wv, d->D, d->G * 64, d->G * 64, kSkChunk));
+    GQE_TRY(tmap_rows(&pp.tmWr, Wr, d->D, GM, GM, kSkChunk));
+    GQE_TRY(tmap_rows(&pp.tmWo, Wo, Ka, d->D, d->D, kSkChunk));
+    const int smem = skinny_proj_smem(d->B, d->D, d->G * d->M);
+    GQE_TRY(set_smem(decode_proj_kernel, smem));
+    GQE_TRY(launch_pdl(decode_proj_kernel, dim3(2 * d->G + 1 + d->G * d->M), dim3(kSkinnyThreads), smem, st, pp));
+  }
   // one pair-GEMM launch over the new tokens: K, V, the shared query and the
   // router, then the compaction and the selected queries (prefill kernels)
   DenseSeg segs[3];
   kv_segments(&t, Wq, Wk, Wv, f.Q, f.Kn, f.Vn, segs);
-  GemmParams p;
-  long long dense_tiles = 0, route_tiles = 0;
-  GQE_TRY(dense_params(p, x_new, d->B, d->D, segs, 3, &dense_tiles));
-  GQE_TRY(add_route_tiles(p, &t, Wr, br, sel, w, f.margin, f.route, dense_tiles, &route_tiles));
-  GQE_TRY(launch_gemm_pair(p, dense_tiles + route_tiles, st));
-  GQE_TRY(route_finish(&t, sel, f.seg_off, f.seg_tok, nullptr, f.route, st));
-  GQE_TRY(do_qgather(&t, x_new, Wq, sel, f.seg_off, f.seg_tok, f.Q, st));
+  if (!skinny) {
+    GemmParams p;
+    long long dense_tiles = 0, route_tiles = 0;
+    GQE_TRY(dense_params(p, x_new, d->B, d->D, segs, 3, &dense_tiles));
+    GQE_TRY(add_route_tiles(p, &t, Wr, br, sel, w, f.margin, f.route, dense_tiles, &route_tiles));
+    GQE_TRY(launch_gemm_pair(p, dense_tiles + route_tiles, st));
+    GQE_TRY(route_finish(&t, sel, f.seg_off, f.seg_tok, nullptr, f.route, st));
+    GQE_TRY(do_qgather(&t, x_new, Wq, sel, f.seg_off, f.seg_tok, f.Q, st));
+  }
   // the cache side: append, split-K attention, merge
   DecodeParams dp;
   dp.Q = f.Q;
@@ -959,11 +1011,16 @@ int gqe_decode(const gqe_dims* d, const int32_t* cache_len, const void* x_new, c
   dp.nsplit = f.nsplit;
   dp.scale_log2 = 1.4426950408889634f / sqrtf(64.f);
   const long long pieces = (long long)d->B * d->G * 64 / 8 * 2;
-  GQE_TRY(launch_pdl(decode_append_kernel, dim3((unsigned)std::min<long long>(cdiv(pieces, 256), 4096)), dim3(256), 0,
-                     st, dp));
+  if (!skinny)
+    GQE_TRY(launch_pdl(decode_append_kernel, dim3((unsigned)std::min<long long>(cdiv(pieces, 256), 4096)), dim3(256),
+                       0, st, dp));
   GQE_TRY(launch_decode_attn(dp, st));
-  const long long warps = (long long)d->B * dp.Ha;
-  GQE_TRY(launch_pdl(decode_merge_kernel, dim3((unsigned)cdiv(warps * 32, 256)), dim3(256), 0, st, dp));
+  GQE_TRY(launch_pdl(decode_merge_kernel, dim3((unsigned)((long long)d->B * dp.Ha)), dim3(kDecMergeThreads), 0, st, dp));
+  if (skinny) {
+    const int smem = skinny_out_smem((d->G * d->k + d->G + 1) * 64);
+    GQE_TRY(set_smem(decode_out_kernel, smem));
+    return launch_pdl(decode_out_kernel, dim3((unsigned)(d->D / 64)), dim3(kSkinnyThreads), smem, st, pp);
+  }
   return do_combine(&t, f.O, w, Wo, y, f.A, st);
 }
 

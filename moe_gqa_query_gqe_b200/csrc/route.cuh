@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(256) route_finalize_kernel(const RouteParams p
 // per-block scan costs less than a second launch.
 constexpr int kRouteFusedMax = 4096;
 
-__global__ void __launch_bounds__(256) route_scan_finalize_kernel(const RouteParams p) {
+__global__ void __launch_bounds__(1024) route_scan_finalize_kernel(const RouteParams p) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ int sh[];

@@ -133,6 +133,12 @@ __device__ __forceinline__ void bulk_wait_read() {
 // All of this thread's bulk groups complete (writes performed).
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Bring `bytes` of global memory (16-byte aligned, a multiple of 16 bytes)
+// into L2 without waiting for it.
+__device__ __forceinline__ void l2_prefetch_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // cp.async (16-byte) for gathered operands.
 // ---------------------------------------------------------------------------
