@@ -355,20 +355,24 @@ def pool_study(steps: int, warmup: int) -> None:
             del g1, g2
 
 
-def decode_study(steps: int, warmup: int) -> None:
+def decode_study(steps: int, warmup: int, cases: str = "") -> None:
     """Decode step (gqe_decode): one new token per sequence against caches of
     L positions, for the main layer's shape (D 1024, G 8, M 2, k 1). Per
     configuration: one JSON line with the step time (CUDA-graph replays, L2
     flushed between them), tokens/s, the bytes the step must read (the K/V
     cache rows up to each new token, plus the weights) and that rate as a
-    fraction of the measured HBM bandwidth."""
+    fraction of the measured HBM bandwidth. `cases` ("8x32767,1x131071")
+    picks configurations by B x L; empty: all three."""
     import torch
     import moe_gqa_query_gqe_b200 as gqe
     from gqe_inputs import Dims, make_decode_inputs
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     peaks = load_peaks()
-    for (B, L) in [(8, 32767), (64, 4095), (1, 131071)]:
+    todo = [(8, 32767), (64, 4095), (1, 131071)]
+    if cases:
+        todo = [tuple(int(v) for v in c.split("x")) for c in cases.split(",")]
+    for (B, L) in todo:
         d = Dims(B=B, T=L + 1, D=1024, G=8, M=2, k=1)
         inp = {kk: v.cuda() for kk, v in make_decode_inputs(d, [L] * B, seed=0, device="cpu").items()}
         y = torch.empty(B, d.D, dtype=torch.bfloat16, device="cuda")
@@ -567,6 +571,8 @@ def main():
                     help="comma-separated long-context workloads timed after the headline (empty: none)")
     ap.add_argument("--study", choices=["pools", "decode", "stages"],
                     help="print the expert-pool, decode-step or per-stage study lines instead of the bench line")
+    ap.add_argument("--cases", default="",
+                    help="decode study: configurations as BxL, comma-separated (default: all three)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -580,7 +586,7 @@ def main():
         pool_study(steps=min(args.steps, 20), warmup=args.warmup)
         return
     if args.study == "decode":
-        decode_study(steps=min(args.steps, 20), warmup=args.warmup)
+        decode_study(steps=min(args.steps, 20), warmup=args.warmup, cases=args.cases)
         return
     if args.study == "stages":
         stage_study(args.workload, steps=min(args.steps, 20), warmup=args.warmup)

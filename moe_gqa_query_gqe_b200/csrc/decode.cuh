@@ -293,7 +293,6 @@ __host__ __device__ inline int dec_ring_smem(int Ha, int rmax) {
 
 template <int KR>
 __global__ void __launch_bounds__(kDecThreads) decode_attn_ring_kernel(const DecodeParams p) {
-  pdl_wait();
   pdl_trigger();
   extern __shared__ uint8_t dr_raw[];
   uint8_t* ring = dr_raw + ((1024u - (smem_u32(dr_raw) & 1023u)) & 1023u);
@@ -306,9 +305,13 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_ring_kernel(const Dec
   const int s = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = lane & 7, kq = lane >> 3;  // 16-byte piece of a row, key within the quad
+  // cache_len and the cache rows before the new token's depend on no launch
+  // of this step: a chunk without row L starts loading before the wait for
+  // the projection launch (which writes row L and the queries)
   const int L = dec_len(p, b);
   const int k0 = s * kDecChunk, k1 = min(k0 + kDecChunk, L + 1);
   if (L < 0 || k0 >= k1) {
+    pdl_wait();
     for (int i = tid; i < p.G * p.rmax; i += kDecThreads) {
       const size_t at = ((size_t)(b * p.G) * p.rmax + i) * p.nsplit + s;
       p.part_ml[at * 2] = -INFINITY;
@@ -320,14 +323,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_ring_kernel(const Dec
   const int SK = dec_stage_keys(p.G);
   const int nst = (n + SK - 1) / SK;  // stages per pass (K, then V)
   const size_t row_bytes = (size_t)p.G * 128;
-  if (tid == 0) {
-    for (int i = 0; i < kDecRingStages; ++i) mbar_init(&full[i], 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  for (int i = tid; i < p.Ha * 64; i += kDecThreads)
-    q[i] = __bfloat162float(p.Q[(size_t)b * p.Ha * 64 + i]) * p.scale_log2;
-  __syncthreads();
+  const bool has_new = k1 == L + 1;  // the chunk holds row L
   // stage i: pass i / nst (K or V), keys [k0 + (i % nst) * SK, +SK) clipped
   auto issue = [&](int i) {
     const int st = i % nst, key0 = k0 + st * SK, nk = min(SK, k1 - key0);
@@ -339,8 +335,19 @@ __global__ void __launch_bounds__(kDecThreads) decode_attn_ring_kernel(const Dec
                  "l"(src), "r"((uint32_t)(nk * row_bytes)), "r"(smem_u32(bar))
                  : "memory");
   };
-  if (tid == 0)
+  if (tid == 0) {
+    for (int i = 0; i < kDecRingStages; ++i) mbar_init(&full[i], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    if (!has_new)
+      for (int i = 0; i < kDecRingStages && i < 2 * nst; ++i) issue(i);
+  }
+  pdl_wait();
+  if (tid == 0 && has_new)
     for (int i = 0; i < kDecRingStages && i < 2 * nst; ++i) issue(i);
+  for (int i = tid; i < p.Ha * 64; i += kDecThreads)
+    q[i] = __bfloat162float(p.Q[(size_t)b * p.Ha * 64 + i]) * p.scale_log2;
+  __syncthreads();
   const int gs = min(p.G, kDecWarps), wpg = kDecWarps / gs;  // warps per group
   bool ok = true;
   uint32_t uses[kDecRingStages] = {};

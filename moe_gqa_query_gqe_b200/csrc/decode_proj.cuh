@@ -14,15 +14,16 @@
 // D x 64 per 64-column block. The tensor-core tiles of the prefill path would
 // pad the B rows to 256 and stream each weight through a few SMs; here every
 // 64-column weight slice is read by its own CTA, so all slices stream at once.
+//   decode_route_kernel: one block: router logits x Wr + br of the B tokens,
+//                        their decisions -> sel, w, margin
 //   decode_proj_kernel : block 0..G-1   K of group g -> cache row cache_len[b]
 //                        block G..2G-1  V of group g -> cache row cache_len[b]
 //                        block 2G       the shared head's query
 //                        block 2G+1+h   routed head h = g*M + e: the query of
 //                                       the tokens that selected it (only)
-//                        Every block that needs the routing decisions computes
-//                        them itself from x Wr + br (the same code and order in
-//                        every block, so they agree); block 0 also writes sel,
-//                        w and margin.
+//                        Its weight slices load while the routing launch runs
+//                        (programmatic dependent launch: the wait for it comes
+//                        after the loads are issued).
 //   decode_out_kernel  : block j: columns [64j, 64j + 64) of y = A Wo, with
 //                        A = [concat | per-group slot sum_j w_j O_j | shared]
 //                        built from O and w in shared memory (the slot rounded
@@ -70,12 +71,16 @@ struct DecodeProjParams {
 // Shared memory (from a 1024-aligned base): kSkBufs weight chunk buffers
 // [kSkBufs][kSkChunk][128 B], their mbarriers and the abort flag (1 KB), then the
 // tokens' rows xs [TB][K] (bf16), per-warp partials red [8][TB][64] (float),
-// and for decode_proj_kernel logits [B][G*M] (float) and the token list of a
-// routed head [kSkinnyMaxTokens + 1] (int; the last entry holds its length).
+// and for decode_route_kernel the logits [B][G*M] (float), for
+// decode_proj_kernel the token list of a routed head [kSkinnyMaxTokens + 1]
+// (int; the last entry holds its length).
 constexpr int kSkWbuf = kSkBufs * kSkChunk * 128;
 constexpr int kSkHead = kSkWbuf + 1024;
-__host__ __device__ inline int skinny_proj_smem(int B, int D, int GM) {
-  return 1024 + kSkHead + kSkinnyTB * D * 2 + 8 * kSkinnyTB * 64 * 4 + B * GM * 4 + (kSkinnyMaxTokens + 1) * 4;
+__host__ __device__ inline int skinny_route_smem(int B, int D, int GM) {
+  return 1024 + kSkHead + kSkinnyTB * D * 2 + 8 * kSkinnyTB * 64 * 4 + B * GM * 4;
+}
+__host__ __device__ inline int skinny_proj_smem(int D) {
+  return 1024 + kSkHead + kSkinnyTB * D * 2 + 8 * kSkinnyTB * 64 * 4 + (kSkinnyMaxTokens + 1) * 4;
 }
 __host__ __device__ inline int skinny_out_smem(int D_in) {
   return 1024 + kSkHead + kSkinnyTB * D_in * 2 + 8 * kSkinnyTB * 64 * 4;
@@ -97,18 +102,27 @@ struct SkPipe {
 // bytes each at column c8 = 8 (t % 8); columns at or past ncols are zeros and
 // skipped. The 32 row-partials of each (n, c) are summed: lanes 0..7 of every
 // warp leave the warp's sums in red[warp]. Returns false if a wait timed out.
+// Thread 0 issues the TMA loads of chunk ch of the slice into its buffer.
+__device__ __forceinline__ void skinny_issue(const CUtensorMap* tm, int col0, int ch, SkPipe& pp) {
+  const int bsel = ch % kSkBufs;
+  mbar_arrive_expect_tx(&pp.bar[bsel], kSkChunk * 128);
+  tma_load_2d(pp.wbuf + bsel * kSkChunk * 128, tm, &pp.bar[bsel], col0, ch * kSkChunk);
+}
+// The first kSkBufs chunks (thread 0), so they load before the data they
+// multiply is ready (skinny_block then takes preissued = true).
+__device__ __forceinline__ void skinny_prefetch(const CUtensorMap* tm, int col0, int K, SkPipe& pp) {
+  const int nch = (K + kSkChunk - 1) / kSkChunk;
+  if (threadIdx.x == 0)
+    for (int ch = 0; ch < kSkBufs && ch < nch; ++ch) skinny_issue(tm, col0, ch, pp);
+}
+
 __device__ __forceinline__ bool skinny_block(const CUtensorMap* tm, int col0, int ncols, const __nv_bfloat16* xs,
-                                             int K, float* red, SkPipe& pp) {
+                                             int K, float* red, SkPipe& pp, bool preissued = false) {
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int c8 = (t & 7) * 8, kr = t >> 3;
   const int nch = (K + kSkChunk - 1) / kSkChunk;
-  auto issue = [&](int ch) {
-    const int bsel = ch % kSkBufs;
-    mbar_arrive_expect_tx(&pp.bar[bsel], kSkChunk * 128);
-    tma_load_2d(pp.wbuf + bsel * kSkChunk * 128, tm, &pp.bar[bsel], col0, ch * kSkChunk);
-  };
-  if (t == 0)
-    for (int ch = 0; ch < kSkBufs && ch < nch; ++ch) issue(ch);
+  auto issue = [&](int ch) { skinny_issue(tm, col0, ch, pp); };
+  if (!preissued) skinny_prefetch(tm, col0, K, pp);
   float acc[kSkinnyTB][8];
 #pragma unroll
   for (int n = 0; n < kSkinnyTB; ++n)
@@ -212,17 +226,20 @@ __device__ __forceinline__ void skinny_stage_x(const DecodeProjParams& p, const 
   __syncthreads();
 }
 
+// Router logits x Wr + br of the B new tokens, then the decisions, written to
+// sel, w and margin.
 template <int RM>
-__device__ bool skinny_route(const DecodeProjParams& p, __nv_bfloat16* xs, float* logits, float* red, bool write,
-                             SkPipe& pp) {
+__device__ bool skinny_route(const DecodeProjParams& p, __nv_bfloat16* xs, float* logits, float* red, SkPipe& pp) {
   const int GM = p.G * RM;
+  bool pre = true;  // the first slice's chunks were issued by the caller
   for (int n0 = 0; n0 < p.B; n0 += kSkinnyTB) {
     int tok[kSkinnyTB];
 #pragma unroll
     for (int n = 0; n < kSkinnyTB; ++n) tok[n] = n0 + n;
     skinny_stage_x(p, tok, min(kSkinnyTB, p.B - n0), xs);
     for (int c0 = 0; c0 < GM; c0 += 64) {
-      if (!skinny_block(&p.tmWr, c0, GM - c0, xs, p.D, red, pp)) return false;
+      if (!skinny_block(&p.tmWr, c0, GM - c0, xs, p.D, red, pp, pre)) return false;
+      pre = false;
       for (int i = threadIdx.x; i < kSkinnyTB * 64; i += kSkinnyThreads) {
         const int n = i / 64, c = i % 64;
         if (n0 + n < p.B && c0 + c < GM)
@@ -231,8 +248,7 @@ __device__ bool skinny_route(const DecodeProjParams& p, __nv_bfloat16* xs, float
       __syncthreads();
     }
   }
-  // decisions: one thread per (token, group); sel/w/margin scratch in place
-  // of the outputs when this block does not write them
+  // decisions: one thread per (token, group)
   for (int i = threadIdx.x; i < p.B * p.G; i += kSkinnyThreads) {
     const int n = i / p.G, g = i % p.G;
     float l[RM];
@@ -242,24 +258,46 @@ __device__ bool skinny_route(const DecodeProjParams& p, __nv_bfloat16* xs, float
     float wl[8];
     float mg;
     route_decide<RM, false>(l, p.k, true, sl, wl, &mg);
-    // the selected experts, encoded for the routed blocks: bit e of the mask
-    uint32_t mask = 0;
-    for (int j = 0; j < p.k; ++j) mask |= 1u << sl[j];
-    reinterpret_cast<uint32_t*>(logits)[n * GM + g * RM] = mask;  // the group's first logit slot
-    if (write) {
-      for (int j = 0; j < p.k; ++j) {
-        p.sel[((size_t)n * p.G + g) * p.k + j] = sl[j];
-        p.w[((size_t)n * p.G + g) * p.k + j] = wl[j];
-      }
-      if (p.margin) p.margin[(size_t)n * p.G + g] = mg;
+    for (int j = 0; j < p.k; ++j) {
+      p.sel[((size_t)n * p.G + g) * p.k + j] = sl[j];
+      p.w[((size_t)n * p.G + g) * p.k + j] = wl[j];
     }
+    if (p.margin) p.margin[(size_t)n * p.G + g] = mg;
   }
   __syncthreads();
   return true;
 }
 
-__global__ void __launch_bounds__(kSkinnyThreads) decode_proj_kernel(const __grid_constant__ DecodeProjParams p) {
+// One CTA: the routing decisions of the B new tokens (sel, w, margin).
+__global__ void __launch_bounds__(kSkinnyThreads) decode_route_kernel(const __grid_constant__ DecodeProjParams p) {
+  extern __shared__ uint8_t sk_raw[];
+  uint8_t* sk = sk_raw + ((1024u - (smem_u32(sk_raw) & 1023u)) & 1023u);
+  SkPipe pp = skinny_pipe_init(sk);
+  skinny_prefetch(&p.tmWr, 0, p.D, pp);  // Wr depends on no launch
+  // the previous step's output kernel reads w: wait before writing it (and
+  // before letting the projection launch in)
   pdl_wait();
+  pdl_trigger();
+  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(sk + kSkHead);
+  float* red = reinterpret_cast<float*>(sk + kSkHead + kSkinnyTB * p.D * 2);
+  float* logits = red + 8 * kSkinnyTB * 64;
+  bool ok = true;
+  switch (p.M) {
+    case 1: ok = skinny_route<1>(p, xs, logits, red, pp); break;
+    case 2: ok = skinny_route<2>(p, xs, logits, red, pp); break;
+    case 4: ok = skinny_route<4>(p, xs, logits, red, pp); break;
+    default: ok = skinny_route<8>(p, xs, logits, red, pp); break;
+  }
+  if (!ok) {  // a wait ran out: let copies in flight land before the block exits
+    const unsigned long long t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 100000ull) {}
+  }
+}
+
+// The projections of the new tokens. The weight slice starts loading before
+// the wait for the routing launch (weights depend on no launch); routed
+// blocks read sel after the wait.
+__global__ void __launch_bounds__(kSkinnyThreads) decode_proj_kernel(const __grid_constant__ DecodeProjParams p) {
   pdl_trigger();
   extern __shared__ uint8_t sk_raw[];
   // aligned by pointer arithmetic on the shared array itself, so the
@@ -270,55 +308,62 @@ __global__ void __launch_bounds__(kSkinnyThreads) decode_proj_kernel(const __gri
   const int GM = p.G * p.M;
   __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(sk + kSkHead);
   float* red = reinterpret_cast<float*>(sk + kSkHead + kSkinnyTB * p.D * 2);
-  float* logits = red + 8 * kSkinnyTB * 64;
-  int* tlist = reinterpret_cast<int*>(logits + p.B * GM);
+  int* tlist = reinterpret_cast<int*>(red + 8 * kSkinnyTB * 64);
   const int blk = blockIdx.x;
   const int Ha = p.G * p.k + 1;
   const bool routed = blk > 2 * p.G;
-  bool ok = true;
-  if (routed || blk == 0) {
-    switch (p.M) {
-      case 1: ok = skinny_route<1>(p, xs, logits, red, blk == 0, pp); break;
-      case 2: ok = skinny_route<2>(p, xs, logits, red, blk == 0, pp); break;
-      case 4: ok = skinny_route<4>(p, xs, logits, red, blk == 0, pp); break;
-      default: ok = skinny_route<8>(p, xs, logits, red, blk == 0, pp); break;
-    }
-  }
-  // this block's weight slice and its tokens
+  // this block's weight slice
   const CUtensorMap* W;
-  int col0, g = 0, e = 0, ntok;
+  int col0, g = 0, e = 0;
   if (blk < 2 * p.G) {
     g = blk % p.G;
     W = blk < p.G ? &p.tmWk : &p.tmWv;
     col0 = g * 64;
-    ntok = p.B;
-    for (int i = threadIdx.x; i < p.B; i += kSkinnyThreads) tlist[i] = i;
   } else {
     W = &p.tmWq;
     if (!routed) {
       col0 = GM * 64;
-      ntok = p.B;
-      for (int i = threadIdx.x; i < p.B; i += kSkinnyThreads) tlist[i] = i;
     } else {
       const int h = blk - 2 * p.G - 1;
       g = h / p.M;
       e = h % p.M;
       col0 = h * 64;
-      // the tokens that selected expert e of group g, in order
-      if (threadIdx.x == 0) {
-        int c = 0;
-        for (int n = 0; n < p.B; ++n)
-          if (reinterpret_cast<const uint32_t*>(logits)[n * GM + g * p.M] & (1u << e)) tlist[c++] = n;
-        tlist[kSkinnyMaxTokens] = c;
-      }
     }
+  }
+  skinny_prefetch(W, col0, p.D, pp);
+  // The K/V and shared-query blocks compute their first pass before the
+  // wait (x and the weights depend on no launch) and wait before writing;
+  // the routed blocks need sel first.
+  bool waited = false;
+  int ntok;
+  if (!routed) {
+    ntok = p.B;
+    for (int i = threadIdx.x; i < p.B; i += kSkinnyThreads) tlist[i] = i;
+  } else {
+    pdl_wait();
+    waited = true;
+  }
+  if (routed && threadIdx.x == 0) {
+    // the tokens that selected expert e of group g, in order
+    int c = 0;
+    for (int n = 0; n < p.B; ++n)
+      for (int j = 0; j < p.k; ++j)
+        if (p.sel[((size_t)n * p.G + g) * p.k + j] == e) tlist[c++] = n;
+    tlist[kSkinnyMaxTokens] = c;
   }
   __syncthreads();
   if (routed) ntok = tlist[kSkinnyMaxTokens];
+  bool ok = true;
+  bool pre = true;  // the first chunks were issued above
   for (int n0 = 0; ok && n0 < ntok; n0 += kSkinnyTB) {
     const int nt = min(kSkinnyTB, ntok - n0);
     skinny_stage_x(p, tlist + n0, nt, xs);
-    if (!(ok = skinny_block(W, col0, 64, xs, p.D, red, pp))) break;
+    if (!(ok = skinny_block(W, col0, 64, xs, p.D, red, pp, pre))) break;
+    pre = false;
+    if (!waited) {
+      pdl_wait();  // earlier launches are done with the rows written below
+      waited = true;
+    }
     for (int i = threadIdx.x; i < nt * 64; i += kSkinnyThreads) {
       const int n = i / 64, c = i % 64;
       const int tok = tlist[n0 + n];
@@ -334,12 +379,19 @@ __global__ void __launch_bounds__(kSkinnyThreads) decode_proj_kernel(const __gri
         p.Q[((size_t)tok * Ha + p.G * p.k) * 64 + c] = v;
       } else {
         // slot of expert e among the token's selections (ascending experts)
-        const uint32_t mask = reinterpret_cast<const uint32_t*>(logits)[tok * GM + g * p.M];
-        const int j = __popc(mask & ((1u << e) - 1u));
+        int j = 0;
+        for (int jj = 0; jj < p.k; ++jj)
+          if (p.sel[((size_t)tok * p.G + g) * p.k + jj] == e) j = jj;
         p.Q[((size_t)tok * Ha + g * p.k + j) * 64 + c] = v;
       }
     }
     __syncthreads();
+  }
+  pdl_wait();  // on every path, so this grid completes after the ones it depends on
+  if (ntok == 0) {
+    // nothing consumed the chunks issued before the wait: let them land
+    for (int ch = 0; ch < kSkBufs && ch * kSkChunk < p.D; ++ch)
+      ok = ok && mbar_wait(&pp.bar[ch], 0, pp.abort_flag);
   }
   if (!ok) {  // a wait ran out: let copies in flight land before the block exits
     const unsigned long long t0 = globaltimer_ns();
@@ -349,7 +401,6 @@ __global__ void __launch_bounds__(kSkinnyThreads) decode_proj_kernel(const __gri
 
 // y = A Wo for the new tokens; A from O and w (see the file comment).
 __global__ void __launch_bounds__(kSkinnyThreads) decode_out_kernel(const __grid_constant__ DecodeProjParams p) {
-  pdl_wait();
   pdl_trigger();
   extern __shared__ uint8_t sk_raw[];
   // aligned by pointer arithmetic on the shared array itself, so the
@@ -362,7 +413,10 @@ __global__ void __launch_bounds__(kSkinnyThreads) decode_out_kernel(const __grid
   __nv_bfloat16* As = reinterpret_cast<__nv_bfloat16*>(sk + kSkHead);
   float* red = reinterpret_cast<float*>(sk + kSkHead + kSkinnyTB * Ka * 2);
   const int col0 = blockIdx.x * 64;
+  skinny_prefetch(&p.tmWo, col0, Ka, pp);  // Wo does not depend on the earlier launches
+  pdl_wait();
   bool ok = true;
+  bool pre = true;
   for (int n0 = 0; ok && n0 < p.B; n0 += kSkinnyTB) {
     const int nt = min(kSkinnyTB, p.B - n0);
     // A rows: 64-wide blocks [concat (G*k) | slot (G) | shared], built in
@@ -397,7 +451,8 @@ __global__ void __launch_bounds__(kSkinnyThreads) decode_out_kernel(const __grid
       reinterpret_cast<uint4*>(As)[i] = v;
     }
     __syncthreads();
-    if (!(ok = skinny_block(&p.tmWo, col0, 64, As, Ka, red, pp))) break;
+    if (!(ok = skinny_block(&p.tmWo, col0, 64, As, Ka, red, pp, pre))) break;
+    pre = false;
     for (int i = threadIdx.x; i < nt * 64; i += kSkinnyThreads) {
       const int n = i / 64, c = i % 64;
       p.y[(size_t)(n0 + n) * p.D + col0 + c] = __float2bfloat16_rn(skinny_sum(red, n, c));

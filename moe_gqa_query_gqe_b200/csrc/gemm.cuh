@@ -59,6 +59,11 @@ struct GemmParams {
   // A column remap for the k = 1 combine: A = [O_routed | O_routed | O_shared]
   // read straight from O ([N, (G+1)*64]); 0 disables the remap
   int amap_G;
+  // Selected-query segment: this segment's columns are the routed heads
+  // h = g*M + e of Wq (64 each); the epilogue writes head h's row of token n
+  // to Q slot g*k + j only where sel[n, g, j] is expert e, and drops the
+  // rest (sel from an earlier launch, read after the dependency wait). -1: none.
+  int sel_seg;
 };
 
 

@@ -176,9 +176,30 @@ __device__ void pair_route_epilogue(const GemmParams& p, uint32_t tm, int b, int
   }
 }
 
+// The same decisions as plain expert ids, without ranks and counts (for a
+// forward pass that does not build segment lists).
+template <int RM, bool PR>
+__device__ void pair_route_plain(const GemmParams& p, uint32_t tm, int b, int c, int q, int lane) {
+  const int t = c * kRouteChunk + q * 32 + lane;
+  const bool valid = t < p.r_T;
+  const size_t n = (size_t)b * p.r_T + (valid ? t : 0);
+  const int G = p.G, k = p.k;
+  for (int g = 0; g < G; ++g) {
+    float l[RM];
+    tmem_ld_cols<RM>(tm + g * RM, l);
+#pragma unroll
+    for (int e = 0; e < RM; ++e) l[e] += p.r_br ? p.r_br[g * RM + e] : 0.f;
+    const size_t o = (n * G + g) * k;
+    route_decide<RM, PR>(l, k, valid, p.r_sel + o, p.r_w + o, p.r_margin ? p.r_margin + n * G + g : nullptr,
+                         PR ? p.r_p + o : nullptr);
+  }
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     gemm_pair_kernel(const __grid_constant__ GemmParams p, int total_tiles) {
-  pdl_wait();
+  // A selected-query launch reads only inputs (x, Wq) in its main loop: the
+  // wait for the routing launch is left to the epilogue, before it reads sel.
+  if (p.sel_seg < 0) pdl_wait();
   pdl_trigger();
   using L = PairSmem;
   extern __shared__ uint8_t smem_raw[];
@@ -298,6 +319,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   } else {
     // ---- epilogue (both CTAs): this CTA's 128 rows ----------------------------------
     const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
+    if (p.sel_seg >= 0) pdl_wait();
     const uint32_t acce_c = mapa_shared(smem_u32(acc_empty), 0);
     uint8_t* stage_out = smem + L::kStageOut + q * 2 * L::kOutBytes;  // this warp's two staging buffers
     uint32_t nstore = 0;                                               // chunks staged by this warp
@@ -311,7 +333,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       // routing decisions of this CTA's 128 tokens (chunk c of sequence b)
       // from the logits at TMEM column tm
       auto route = [&](uint32_t tm, int b, int c) {
-        if (p.r_p == nullptr) {
+        if (p.r_counts == nullptr) {
+          if (p.r_p == nullptr) {
+            switch (p.M) {
+              case 1: pair_route_plain<1, false>(p, tm, b, c, q, lane); break;
+              case 2: pair_route_plain<2, false>(p, tm, b, c, q, lane); break;
+              case 4: pair_route_plain<4, false>(p, tm, b, c, q, lane); break;
+              default: pair_route_plain<8, false>(p, tm, b, c, q, lane); break;
+            }
+          } else {
+            switch (p.M) {
+              case 1: pair_route_plain<1, true>(p, tm, b, c, q, lane); break;
+              case 2: pair_route_plain<2, true>(p, tm, b, c, q, lane); break;
+              case 4: pair_route_plain<4, true>(p, tm, b, c, q, lane); break;
+              default: pair_route_plain<8, true>(p, tm, b, c, q, lane); break;
+            }
+          }
+        } else if (p.r_p == nullptr) {
           switch (p.M) {
             case 1: pair_route_epilogue<1, false>(p, tm, b, c, q, lane, s_tot); break;
             case 2: pair_route_epilogue<2, false>(p, tm, b, c, q, lane, s_tot); break;
@@ -336,12 +374,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         if (lane == 0) mbar_arrive_cluster(acce_c + 8 * a);
         continue;
       }
-      // 64-column chunks: TMEM -> registers -> bf16 -> swizzled staging rows (one
-      // row per lane, conflict-free) -> one TMA store of 32 rows x 64 columns
       const GemmSeg& sg = p.seg[t.seg];
       const int wrow0 = t.m0 + (int)rank * 128 + q * 32;  // first row of this warp
       const int ncols = min(t.nvalid, sg.n_cols - t.n0);
       const uint32_t tm = tmem_base + a * kPairBN + (static_cast<uint32_t>(q * 32) << 16);
+      if (t.seg == p.sel_seg) {
+        // routed heads: lane = token n; head h's 64 columns go to Q slot
+        // g*k + j if the token selected expert e = h % M of group g = h / M
+        // (slot j), else nowhere. Each lane stores its own 128-byte row.
+        const int n = wrow0 + lane;
+#pragma unroll 1
+        for (int ch = 0; ch < t.nvalid / 64; ++ch) {
+          uint32_t r[64];
+          tmem_ld64(tm + ch * 64, r);
+          if (ch * 64 >= ncols || n >= p.rows) continue;
+          const int h = (sg.b_col0 + t.n0) / 64 + ch;
+          const int g = h / p.M, e = h % p.M;
+          const int32_t* sl = p.sel + ((size_t)n * p.G + g) * p.k;
+          int j = -1;
+          for (int jj = 0; jj < p.k; ++jj)
+            if ((sl[jj] & 0xff) == e) j = jj;
+          if (j < 0) continue;
+          uint4* dst = reinterpret_cast<uint4*>(p.Q + ((size_t)n * p.Ha + g * p.k + j) * 64);
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            dst[c] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * c]), __uint_as_float(r[8 * c + 1])),
+                                pack_bf16x2(__uint_as_float(r[8 * c + 2]), __uint_as_float(r[8 * c + 3])),
+                                pack_bf16x2(__uint_as_float(r[8 * c + 4]), __uint_as_float(r[8 * c + 5])),
+                                pack_bf16x2(__uint_as_float(r[8 * c + 6]), __uint_as_float(r[8 * c + 7])));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acce_c + 8 * a);
+        continue;
+      }
+      // 64-column chunks: TMEM -> registers -> bf16 -> swizzled staging rows (one
+      // row per lane, conflict-free) -> one TMA store of 32 rows x 64 columns
       for (int ch = 0; ch < t.nvalid / 64; ++ch) {
         uint32_t r[64];
         tmem_ld64(tm + ch * 64, r);

@@ -240,6 +240,7 @@ int dense_params(GemmParams& p, const void* A, long long rows, int K, const Dens
   *tiles = nt > 0 ? cdiv(rows, kPairBM) * nt : 0;
   p.r_tile0 = 0x7fffffff;
   p.r_merge_seg = -1;
+  p.sel_seg = -1;
   return GQE_OK;
 }
 
@@ -428,6 +429,7 @@ int do_route(const gqe_dims* d, const void* x, const void* Wr, const float* br, 
   GemmParams p;
   memset(&p, 0, sizeof(p));
   p.r_merge_seg = -1;
+  p.sel_seg = -1;
   const long long N = (long long)d->B * d->T;
   GQE_TRY(tmap_rows(&p.tmA, x, N, d->D, d->D, kGemmBM));
   p.rows = (int)N;
@@ -448,6 +450,32 @@ void kv_segments(const gqe_dims* d, const void* Wq, const void* Wk, const void* 
   segs[2] = DenseSeg{Wq, wq_cols, G * M * 64, 64, Q, (long long)Ha * 64, G * k * 64};
 }
 
+// The selected queries of gqe_forward as one dense product over every
+// routed head (Wq columns 0 .. G*M*64), whose epilogue keeps each token's
+// selected experts' rows (gemm2sm.cuh, selected-query segment). Chosen when
+// M <= 2k: the tensor-core work on the unselected heads (at most as much
+// again) then costs less than gathering every (token, group)'s row of x per
+// expert, which the gather kernel is bound by. The results are the same
+// products, accumulated in the same order.
+bool qproj_dense_select(const gqe_dims* d) { return d->M <= 2 * d->k; }
+
+int do_qselect(const gqe_dims* d, const void* x, const void* Wq, const int32_t* sel, void* Q, cudaStream_t st) {
+  const int G = d->G, M = d->M, k = d->k, Ha = G * k + 1;
+  const int wq_cols = (G * M + 1) * 64;
+  const DenseSeg seg = {Wq, wq_cols, 0, G * M * 64, Q, (long long)Ha * 64, 0};
+  GemmParams p;
+  long long tiles = 0;
+  GQE_TRY(dense_params(p, x, (long long)d->B * d->T, d->D, &seg, 1, &tiles));
+  p.sel_seg = 0;
+  p.sel = sel;
+  p.Q = static_cast<__nv_bfloat16*>(Q);
+  p.G = G;
+  p.M = M;
+  p.k = k;
+  p.Ha = Ha;
+  return launch_gemm_pair(p, tiles, st);
+}
+
 // Selected experts: one segment per (b, g, e), rows gathered by seg_tok.
 int do_qgather(const gqe_dims* d, const void* x, const void* Wq, const int32_t* sel, const int32_t* seg_off,
                const int32_t* seg_tok, void* Q, cudaStream_t st) {
@@ -457,6 +485,7 @@ int do_qgather(const gqe_dims* d, const void* x, const void* Wq, const int32_t* 
   GemmParams p;
   memset(&p, 0, sizeof(p));
   p.r_merge_seg = -1;
+  p.sel_seg = -1;
   GQE_TRY(tmap_rows(&p.tmB[0], Wq, d->D, wq_cols, wq_cols, 64));
   GQE_TRY(tmap_rows(&p.tmA, x, N, d->D, d->D, 1));  // a valid map for the kernel's descriptor prefetch (rows are copied with cp.async)
   p.K = d->D;
@@ -554,6 +583,7 @@ int project_from_o(const gqe_dims* d, const void* O, const void* Wo, void* y, in
   p.amap_G = d->G;
   p.r_tile0 = 0x7fffffff;
   p.r_merge_seg = -1;
+  p.sel_seg = -1;
   return launch_gemm_pair(p, cdiv(N, kPairBM) * p.ntn, st);
 }
 
@@ -816,13 +846,17 @@ int do_forward(const gqe_dims* d, int mode, const void* x, const void* Wq, const
   // (its column of Q and O is left unwritten and is never read).
   const bool shared = mode != GQE_COMBINE_NO_SHARED;
   // one pair-GEMM launch over x: K, V, the shared head's query and the router
-  // (logits and decisions), then the compaction and the selected queries
+  // (logits and decisions), then the selected queries: a dense product over
+  // the routed heads that keeps the selected rows, or (M > 2k) the
+  // compaction and the gather
+  const bool qsel = qproj_dense_select(d);
   DenseSeg segs[3];
   kv_segments(d, Wq, Wk, Wv, f.Q, f.K, f.V, segs);
   GemmParams p;
   long long dense_tiles = 0, route_tiles = 0;
   GQE_TRY(dense_params(p, x, (long long)d->B * d->T, d->D, segs, shared ? 3 : 2, &dense_tiles));
   GQE_TRY(add_route_tiles(p, d, Wr, br, f.sel, f.w, f.margin, f.route, dense_tiles, &route_tiles));
+  if (qsel) p.r_counts = nullptr;  // plain decisions, no segment lists
   p.r_p = (mode == GQE_COMBINE_WEIGHTED || mode == GQE_COMBINE_GLOBAL_SLOT) ? p_sel : nullptr;
   if (shared && d->T % kRouteChunk == 0) {
     // the router logits fill the second half of the shared head's 128-column
@@ -832,8 +866,12 @@ int do_forward(const gqe_dims* d, int mode, const void* x, const void* Wq, const
     route_tiles = 0;
   }
   GQE_TRY(launch_gemm_pair(p, dense_tiles + route_tiles, st));
-  GQE_TRY(route_finish(d, f.sel, f.seg_off, f.seg_tok, f.row_map, f.route, st));
-  GQE_TRY(do_qgather(d, x, Wq, f.sel, f.seg_off, f.seg_tok, f.Q, st));
+  if (qsel) {
+    GQE_TRY(do_qselect(d, x, Wq, f.sel, f.Q, st));
+  } else {
+    GQE_TRY(route_finish(d, f.sel, f.seg_off, f.seg_tok, f.row_map, f.route, st));
+    GQE_TRY(do_qgather(d, x, Wq, f.sel, f.seg_off, f.seg_tok, f.Q, st));
+  }
   if (mode == GQE_COMBINE_SLOT && d->k > 1) {
     // the attention writes A itself (concatenation, per-group slots, shared
     // head), then y = A Wo: no separate combine pass over O
@@ -938,8 +976,8 @@ int gqe_decode(const gqe_dims* d, const int32_t* cache_len, const void* x_new, c
   DecodeWs f = carve_decode(c, d);
   const gqe_dims t = decode_token_dims(d);
   const int ka_cols = (d->G * d->k + d->G + 1) * 64;
-  const bool skinny = d->B <= kSkinnyMaxTokens && skinny_proj_smem(d->B, d->D, d->G * d->M) <= 232448 &&
-                      skinny_out_smem(ka_cols) <= 232448;
+  const bool skinny = d->B <= kSkinnyMaxTokens && skinny_route_smem(d->B, d->D, d->G * d->M) <= 232448 &&
+                      skinny_proj_smem(d->D) <= 232448 && skinny_out_smem(ka_cols) <= 232448;
   DecodeProjParams pp;
   memset(&pp, 0, sizeof(pp));
   pp.x = static_cast<const __nv_bfloat16*>(x_new);
@@ -974,9 +1012,12 @@ int gqe_decode(const gqe_dims* d, const int32_t* cache_len, const void* x_new, c
     GQE_TRY(tmap_rows(&pp.tmWv, Wv, d->D, d->G * 64, d->G * 64, kSkChunk));
     GQE_TRY(tmap_rows(&pp.tmWr, Wr, d->D, GM, GM, kSkChunk));
     GQE_TRY(tmap_rows(&pp.tmWo, Wo, Ka, d->D, d->D, kSkChunk));
-    const int smem = skinny_proj_smem(d->B, d->D, d->G * d->M);
+    const int rsmem = skinny_route_smem(d->B, d->D, GM);
+    GQE_TRY(set_smem(decode_route_kernel, rsmem));
+    GQE_TRY(launch_pdl(decode_route_kernel, dim3(1), dim3(kSkinnyThreads), rsmem, st, pp));
+    const int smem = skinny_proj_smem(d->D);
     GQE_TRY(set_smem(decode_proj_kernel, smem));
-    GQE_TRY(launch_pdl(decode_proj_kernel, dim3(2 * d->G + 1 + d->G * d->M), dim3(kSkinnyThreads), smem, st, pp));
+    GQE_TRY(launch_pdl(decode_proj_kernel, dim3(2 * d->G + 1 + GM), dim3(kSkinnyThreads), smem, st, pp));
   }
   // one pair-GEMM launch over the new tokens: K, V, the shared query and the
   // router, then the compaction and the selected queries (prefill kernels)
@@ -987,9 +1028,15 @@ int gqe_decode(const gqe_dims* d, const int32_t* cache_len, const void* x_new, c
     long long dense_tiles = 0, route_tiles = 0;
     GQE_TRY(dense_params(p, x_new, d->B, d->D, segs, 3, &dense_tiles));
     GQE_TRY(add_route_tiles(p, &t, Wr, br, sel, w, f.margin, f.route, dense_tiles, &route_tiles));
+    const bool qsel = qproj_dense_select(&t);
+    if (qsel) p.r_counts = nullptr;
     GQE_TRY(launch_gemm_pair(p, dense_tiles + route_tiles, st));
-    GQE_TRY(route_finish(&t, sel, f.seg_off, f.seg_tok, nullptr, f.route, st));
-    GQE_TRY(do_qgather(&t, x_new, Wq, sel, f.seg_off, f.seg_tok, f.Q, st));
+    if (qsel) {
+      GQE_TRY(do_qselect(&t, x_new, Wq, sel, f.Q, st));
+    } else {
+      GQE_TRY(route_finish(&t, sel, f.seg_off, f.seg_tok, nullptr, f.route, st));
+      GQE_TRY(do_qgather(&t, x_new, Wq, sel, f.seg_off, f.seg_tok, f.Q, st));
+    }
   }
   // the cache side: append, split-K attention, merge
   DecodeParams dp;

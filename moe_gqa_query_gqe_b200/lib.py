@@ -209,7 +209,10 @@ def _align(v: int) -> int:
 def forward_views(dims, ws: torch.Tensor) -> dict:
     """Typed views of the intermediates gqe_forward leaves in its workspace
     (same carving order as the library: sel, w, margin, seg_off, seg_tok,
-    row_map, route counts x2, Q, K, V, O, A)."""
+    row_map, route counts x2, Q, K, V, O, A). seg_off, seg_tok and row_map are
+    written only when the forward gathers the selected queries (M > 2k);
+    for M <= 2k it projects every routed head and keeps the selected rows,
+    without segment lists."""
     d = dims_struct(dims)
     N = d.B * d.T
     nch = (d.T + 127) // 128

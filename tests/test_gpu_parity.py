@@ -167,9 +167,13 @@ def _sampled_parity(d, n_uniform, seed=0, dense=True, case=None):
     sel = views["sel"].cpu()
     rows = ref.sample_rows(d.B, d.T, n_uniform=n_uniform, seed=seed)
     chk = check_selection(d, inp["x"], inp["Wr"], inp["br"], sel, rows=rows, case=case)
-    seg_off = views["seg_off"].cpu().numpy()
-    assert seg_off[-1] == d.B * d.T * d.G * d.k
-    counts = np.diff(seg_off)
+    # tokens per (b, g, e) from the decisions (the forward writes segment
+    # lists only on its gather path)
+    s8 = (sel.numpy() & 0xFF).reshape(d.B, d.T, d.G, d.k)
+    counts = np.stack([np.bincount((s8[:, :, g, :] + d.M * np.arange(d.B)[:, None, None]).ravel(),
+                                   minlength=d.B * d.M) for g in range(d.G)], axis=1).reshape(d.B, d.M, d.G)
+    counts = counts.transpose(0, 2, 1).ravel()
+    assert counts.sum() == d.B * d.T * d.G * d.k
     full = ref.gqe_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"], inp["Wo"], d,
                            rows=rows, forced_sel=sel.numpy()[rows])
     e = assert_close_bf16(y.cpu()[rows], full["y"], "y-sampled", case=case)
