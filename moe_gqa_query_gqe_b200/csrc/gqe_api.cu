@@ -700,6 +700,28 @@ int launch_decode_attn(const DecodeParams& dp, cudaStream_t st) {
   }
 }
 
+// The persistent tensor-core decode attention over the caches (decode.cuh).
+// dp.nsplit: the splits the workspace holds; the launch sets its own count
+// (*nsplit_used), which the merge must take.
+int launch_decode_attn_mma(const DecodeParams& dp, int* nsplit_used, cudaStream_t st) {
+  DecodeMmaParams P;
+  memset(&P, 0, sizeof(P));
+  GQE_TRY(tmap_heads(&P.tmK, dp.Kc, (long long)dp.B * dp.T, dp.G, 1, kDmSK));
+  GQE_TRY(tmap_heads(&P.tmV, dp.Vc, (long long)dp.B * dp.T, dp.G, 1, kDmSK));
+  P.d = dp;
+  P.nitem = (int)cdiv(dp.T, kDmItem);
+  P.items = (long long)dp.B * P.nitem;
+  P.wpg = dm_wpg(dp.G);
+  P.gpw = dp.G > kDmWarps ? dp.G / kDmWarps : 1;
+  const int grid = (int)std::min<long long>(std::min<long long>(P.items, kDmGridMax), sm_count());
+  // the workspace holds dm_nsplit(B, G, kDmGridMax) splits, at least this grid's
+  P.d.nsplit = dm_nsplit(dp.B, dp.G, grid);
+  if (P.d.nsplit > dp.nsplit || dp.rmax > 16) return GQE_ERR_UNSUPPORTED;
+  *nsplit_used = P.d.nsplit;
+  GQE_TRY(set_smem(decode_attn_mma_kernel, dm_smem()));
+  return launch_pdl(decode_attn_mma_kernel, dim3(std::max(grid, 1)), dim3(kDmThreads), dm_smem(), st, P);
+}
+
 int check_ptrs(std::initializer_list<const void*> ps) {
   for (const void* p : ps)
     if (p == nullptr || !aligned16(p)) return GQE_ERR_INVALID_ARG;
@@ -748,7 +770,7 @@ DecodeWs carve_decode(Carver& c, const gqe_dims* d) {
   f.Q = c.take<__nv_bfloat16>(B * Ha * 64);
   f.O = c.take<__nv_bfloat16>(B * Ha * 64);
   f.A = d->k == 1 ? nullptr : c.take<__nv_bfloat16>(B * (size_t)(d->G * d->k + d->G + 1) * 64);
-  f.nsplit = (int)cdiv(d->T, kDecChunk);
+  f.nsplit = dm_nsplit(d->B, d->G, kDmGridMax);
   f.rmax = d->k + 1;
   const size_t parts = B * d->G * f.rmax * (size_t)f.nsplit;
   f.part_ml = c.take<float>(parts * 2);
@@ -1061,7 +1083,7 @@ int gqe_decode(const gqe_dims* d, const int32_t* cache_len, const void* x_new, c
   if (!skinny)
     GQE_TRY(launch_pdl(decode_append_kernel, dim3((unsigned)std::min<long long>(cdiv(pieces, 256), 4096)), dim3(256),
                        0, st, dp));
-  GQE_TRY(launch_decode_attn(dp, st));
+  GQE_TRY(launch_decode_attn_mma(dp, &dp.nsplit, st));
   GQE_TRY(launch_pdl(decode_merge_kernel, dim3((unsigned)((long long)d->B * dp.Ha)), dim3(kDecMergeThreads), 0, st, dp));
   if (skinny) {
     const int smem = skinny_out_smem((d->G * d->k + d->G + 1) * 64);
