@@ -998,15 +998,10 @@ int gqe_decode(const gqe_dims* d, const int32_t* cache_len, const void* x_new, c
   DecodeWs f = carve_decode(c, d);
   const gqe_dims t = decode_token_dims(d);
   const int ka_cols = (d->G * d->k + d->G + 1) * 64;
-  const bool skinny = d->B <= kSkinnyMaxTokens && skinny_route_smem(d->B, d->D, d->G * d->M) <= 232448 &&
-                      skinny_proj_smem(d->D) <= 232448 && skinny_out_smem(ka_cols) <= 232448;
+  const bool skinny = d->B <= kSkinnyMaxTokens && sk_smem(d->D) <= 232448 && sk_smem(ka_cols) <= 232448;
   DecodeProjParams pp;
   memset(&pp, 0, sizeof(pp));
   pp.x = static_cast<const __nv_bfloat16*>(x_new);
-  pp.Wq = static_cast<const __nv_bfloat16*>(Wq);
-  pp.Wk = static_cast<const __nv_bfloat16*>(Wk);
-  pp.Wv = static_cast<const __nv_bfloat16*>(Wv);
-  pp.Wr = static_cast<const __nv_bfloat16*>(Wr);
   pp.br = br;
   pp.cache_len = cache_len;
   pp.Kc = static_cast<__nv_bfloat16*>(K_cache);
@@ -1016,7 +1011,6 @@ int gqe_decode(const gqe_dims* d, const int32_t* cache_len, const void* x_new, c
   pp.w = w;
   pp.margin = f.margin;
   pp.O = f.O;
-  pp.Wo = static_cast<const __nv_bfloat16*>(Wo);
   pp.y = static_cast<__nv_bfloat16*>(y);
   pp.B = d->B;
   pp.T = d->T;
@@ -1026,20 +1020,21 @@ int gqe_decode(const gqe_dims* d, const int32_t* cache_len, const void* x_new, c
   pp.k = d->k;
   if (skinny) {
     // a few new tokens: routing, K/V (written straight into the caches at
-    // cache_len) and the queries as skinny products, one CTA per 64-column
-    // weight slice
+    // cache_len) and the queries as skinny products, one 8-CTA cluster per
+    // 64-column weight slice
     const int GM = d->G * d->M, Ka = (d->G * d->k + d->G + 1) * 64;
-    GQE_TRY(tmap_rows(&pp.tmWq, Wq, d->D, (GM + 1) * 64, (GM + 1) * 64, kSkChunk));
-    GQE_TRY(tmap_rows(&pp.tmWk, Wk, d->D, d->G * 64, d->G * 64, kSkChunk));
-    GQE_TRY(tmap_rows(&pp.tmWv, Wv, d->D, d->G * 64, d->G * 64, kSkChunk));
-    GQE_TRY(tmap_rows(&pp.tmWr, Wr, d->D, GM, GM, kSkChunk));
-    GQE_TRY(tmap_rows(&pp.tmWo, Wo, Ka, d->D, d->D, kSkChunk));
-    const int rsmem = skinny_route_smem(d->B, d->D, GM);
-    GQE_TRY(set_smem(decode_route_kernel, rsmem));
-    GQE_TRY(launch_pdl(decode_route_kernel, dim3(1), dim3(kSkinnyThreads), rsmem, st, pp));
-    const int smem = skinny_proj_smem(d->D);
+    GQE_TRY(tmap_rows(&pp.tmWq, Wq, d->D, (GM + 1) * 64, (GM + 1) * 64, kSkBoxRows));
+    GQE_TRY(tmap_rows(&pp.tmWk, Wk, d->D, d->G * 64, d->G * 64, kSkBoxRows));
+    GQE_TRY(tmap_rows(&pp.tmWv, Wv, d->D, d->G * 64, d->G * 64, kSkBoxRows));
+    GQE_TRY(tmap_rows(&pp.tmWr, Wr, d->D, GM, GM, kSkBoxRows));
+    GQE_TRY(tmap_rows(&pp.tmWo, Wo, Ka, d->D, d->D, kSkBoxRows));
+    const int smem = sk_smem(d->D);
+    GQE_TRY(set_smem(decode_route_kernel, smem));
+    GQE_TRY(launch_pdl(decode_route_kernel, dim3((unsigned)cdiv(GM, 64) * kSkCluster), dim3(kSkinnyThreads), smem,
+                       st, pp));
     GQE_TRY(set_smem(decode_proj_kernel, smem));
-    GQE_TRY(launch_pdl(decode_proj_kernel, dim3(2 * d->G + 1 + GM), dim3(kSkinnyThreads), smem, st, pp));
+    GQE_TRY(launch_pdl(decode_proj_kernel, dim3((2 * d->G + 1 + GM) * kSkCluster), dim3(kSkinnyThreads), smem, st,
+                       pp));
   }
   // one pair-GEMM launch over the new tokens: K, V, the shared query and the
   // router, then the compaction and the selected queries (prefill kernels)
@@ -1086,9 +1081,10 @@ int gqe_decode(const gqe_dims* d, const int32_t* cache_len, const void* x_new, c
   GQE_TRY(launch_decode_attn_mma(dp, &dp.nsplit, st));
   GQE_TRY(launch_pdl(decode_merge_kernel, dim3((unsigned)((long long)d->B * dp.Ha)), dim3(kDecMergeThreads), 0, st, dp));
   if (skinny) {
-    const int smem = skinny_out_smem((d->G * d->k + d->G + 1) * 64);
+    const int smem = sk_smem(ka_cols);
     GQE_TRY(set_smem(decode_out_kernel, smem));
-    return launch_pdl(decode_out_kernel, dim3((unsigned)(d->D / 64)), dim3(kSkinnyThreads), smem, st, pp);
+    return launch_pdl(decode_out_kernel, dim3((unsigned)(d->D / 64) * kSkCluster), dim3(kSkinnyThreads), smem, st,
+                      pp);
   }
   return do_combine(&t, f.O, w, Wo, y, f.A, st);
 }

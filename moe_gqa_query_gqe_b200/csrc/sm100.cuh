@@ -302,6 +302,13 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
 }
 // TMA tile load into this CTA's shared memory; the bytes are counted on an
 // mbarrier given by its cluster address (the pair's leader barrier).
+// 32-bit load from distributed shared memory (a cluster address from mapa_shared).
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t cluster_addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* tm, uint32_t bar_cluster, int c0,
                                                  int c1) {
   asm volatile(
