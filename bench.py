@@ -662,11 +662,13 @@ def main():
         return g
 
     # kernels launched per forward step: K/V + shared-query + router pair GEMM,
-    # routing scan and compaction (one launch when the per-chunk counts fit a
-    # block's shared memory, else two), selected-query gather, attention
-    # (which also builds the output operand when k > 1), Wo
+    # the selected queries, attention (which also builds the output operand
+    # when k > 1), Wo. The selected queries are one dense pair GEMM over the
+    # routed heads when M <= 2k; otherwise the routing scan and compaction
+    # (one launch when the per-chunk counts fit a block's shared memory, else
+    # two) and the gather.
     n_counts = d.B * d.G * d.M * ((d.T + 127) // 128)
-    launches_per_step = 4 + (1 if n_counts <= 4096 else 2)
+    launches_per_step = 4 if d.M <= 2 * d.k else 4 + (1 if n_counts <= 4096 else 2)
 
     def barrier():
         if world > 1:
