@@ -676,30 +676,6 @@ int host_pipe(HostPipe** out) {
   return GQE_OK;
 }
 
-// decode_attn_kernel instantiated for the rows of a group (k, plus the shared
-// head in group 0): one CTA per (chunk of keys, sequence).
-template <int KR>
-int launch_decode_attn_kr(const DecodeParams& dp, cudaStream_t st) {
-  if (dp.G <= 2 * kDecWarps) {
-    // cache rows by bulk copies through a shared-memory ring
-    const int smem = dec_ring_smem(dp.Ha, dp.rmax);
-    GQE_TRY(set_smem(decode_attn_ring_kernel<KR>, smem));
-    return launch_pdl(decode_attn_ring_kernel<KR>, dim3(dp.nsplit, dp.B), dim3(kDecThreads), smem, st, dp);
-  }
-  const int smem = dec_smem_floats(dp.Ha, dp.rmax) * 4;
-  GQE_TRY(set_smem(decode_attn_kernel<KR>, smem));
-  return launch_pdl(decode_attn_kernel<KR>, dim3(dp.nsplit, dp.B), dim3(kDecThreads), smem, st, dp);
-}
-int launch_decode_attn(const DecodeParams& dp, cudaStream_t st) {
-  switch (dp.k) {
-    case 1: return launch_decode_attn_kr<2>(dp, st);
-    case 2: return launch_decode_attn_kr<3>(dp, st);
-    case 4: return launch_decode_attn_kr<5>(dp, st);
-    case 8: return launch_decode_attn_kr<9>(dp, st);
-    default: return GQE_ERR_UNSUPPORTED;
-  }
-}
-
 // The persistent tensor-core decode attention over the caches (decode.cuh).
 // dp.nsplit: the splits the workspace holds; the launch sets its own count
 // (*nsplit_used), which the merge must take.

@@ -66,11 +66,15 @@ def test_variant_workspace_holds_the_widest_variant():
         assert extra <= N * d.G * d.k * 4 + N * widest * 2 + 512  # two 256-byte alignments
 
 
-def test_decode_workspace_grows_with_the_cache_capacity():
+def test_decode_workspace_does_not_grow_with_the_cache_capacity():
+    # the attention's partial results are per CTA and sequence (one key range
+    # each), not per key chunk: the workspace depends on B, G and k only
     d = Dims(B=4, T=1024, D=256, G=4, M=2, k=1)
     small = gqe.workspace_bytes(d, gqe.OP_DECODE)
-    assert gqe.workspace_bytes(d.with_(T=32 * 1024), gqe.OP_DECODE) > small
+    assert gqe.workspace_bytes(d.with_(T=32 * 1024), gqe.OP_DECODE) == small
+    assert gqe.workspace_bytes(d.with_(T=1 << 20), gqe.OP_DECODE) == small
     assert gqe.workspace_bytes(d.with_(k=2), gqe.OP_DECODE) > small
+    assert gqe.workspace_bytes(d.with_(B=8), gqe.OP_DECODE) > small
 
 
 @pytest.mark.parametrize("bad,code", [

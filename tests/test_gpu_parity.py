@@ -80,11 +80,18 @@ def test_combine_stage(cases, name):
 
 @pytest.mark.parametrize("name", list(SMALL))
 def test_layer_end_to_end(cases, name):
+    import moe_gqa_query_gqe_b200 as gqe
     d, inp, dev, st = cases[name]
-    y, _, status = run_forward(d, dev)
+    y, ws, status = run_forward(d, dev)
     assert status == 0
-    # the one-call forward runs the same kernels on the same inputs: identical bits
+    # identical bits to the stage path: for M > 2k the forward runs the same
+    # kernels; for M <= 2k its selected queries come from the dense product
+    # over all routed heads instead of the gather, the same dot products
+    # accumulated in the same order, so Q (and all that follows) is the same
     assert torch.equal(y.cpu(), st["y"])
+    if d.M <= 2 * d.k:
+        Q = gqe.forward_views(d, ws)["Q"].cpu()
+        assert torch.equal(Q[:, : d.G * d.k], st["Q"][:, : d.G * d.k])
     full = ref.gqe_forward(inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], inp["Wr"], inp["br"], inp["Wo"], d,
                            forced_sel=st["sel"].numpy())
     assert_close_bf16(y, full["y"], "y", case=name)
