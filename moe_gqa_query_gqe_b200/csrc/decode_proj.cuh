@@ -19,13 +19,13 @@
 // rows of the tokens' inputs; the eight partial sums meet in distributed
 // shared memory, where rank q adds up token q's 64 columns of a pass of
 // eight tokens (ranks in order, so the sum is the same on every run).
-//   decode_route_kernel: cdiv(G*M, 64) clusters: router logits x Wr + br;
-//                        rank q decides token q of a pass for the groups of
-//                        its slice -> sel, w, margin
 //   decode_proj_kernel : 2G + 1 + G*M clusters: K and V of group g (written
 //                        into the caches at cache_len[b]), the shared head's
-//                        query, routed head h = g*M + e's query for only the
-//                        tokens that selected it
+//                        query, and routed head h = g*M + e: its query and
+//                        group g's router logits x Wr + br for every token;
+//                        rank q decides token q of a pass for group g and
+//                        keeps the query row if the token selected e (the
+//                        e = 0 cluster writes sel, w, margin)
 //   decode_out_kernel  : D / 64 clusters: y = A Wo, A = [concat | per-group
 //                        slot sum_j w_j O_j | shared] built for the CTA's rows
 //                        (A's columns) from O and w (the slot rounded to
@@ -73,26 +73,28 @@ __host__ __device__ inline int sk_rows(int K) {
   return (r + kSkBoxRows - 1) / kSkBoxRows * kSkBoxRows;
 }
 // Shared memory (from a 1024-aligned base): the CTA's weight rows wbuf
-// [RR][128 B], the barrier and abort flag (64 B), the inputs' rows xs
-// [TB][RR] (bf16), per-warp partials red [8][TB][64], the CTA's partial part
-// [TB][64] (read by the cluster), the token list of a routed head
-// [kSkinnyMaxTokens + 1] (int, the last entry its length) and the reduced
-// logits of a routing CTA [64] (float).
+// [RR][128 B] and, for a routed head, its router rows wbuf_r [RR][128 B];
+// their barriers and the abort flag (64 B); the inputs' rows xs [TB][RR]
+// (bf16); per-warp partials red [8][TB][64]; the CTA's partials part and
+// part_r [TB][64] (read by the cluster); the decision area (64 B: a group's
+// logits, the selected slot).
 __host__ __device__ inline int sk_smem(int K) {
   const int RR = sk_rows(K);
-  return 1024 + RR * 128 + 64 + kSkinnyTB * RR * 2 + 8 * kSkinnyTB * 64 * 4 + kSkinnyTB * 64 * 4 +
-         (kSkinnyMaxTokens + 1) * 4 + 64 * 4;
+  return 1024 + 2 * RR * 128 + 64 + kSkinnyTB * RR * 2 + 8 * kSkinnyTB * 64 * 4 + 2 * kSkinnyTB * 64 * 4 + 64;
 }
 
 struct SkCta {
   uint8_t* wbuf;
+  uint8_t* wbuf_r;
   uint64_t* bar;
+  uint64_t* bar_r;
   volatile int* abort_flag;
   __nv_bfloat16* xs;
   float* red;
   float* part;
-  int* tlist;
-  float* logits;
+  float* part_r;
+  float* logits;  // [8]
+  int* slot;      // [1]
   int RR, row0, rank;
 };
 
@@ -103,15 +105,20 @@ __device__ __forceinline__ SkCta sk_init(uint8_t* raw, int K) {
   s.rank = (int)cluster_ctarank();
   s.row0 = s.rank * s.RR;
   s.wbuf = b;
-  s.bar = reinterpret_cast<uint64_t*>(b + s.RR * 128);
-  s.abort_flag = reinterpret_cast<volatile int*>(b + s.RR * 128 + 8);
-  s.xs = reinterpret_cast<__nv_bfloat16*>(b + s.RR * 128 + 64);
-  s.red = reinterpret_cast<float*>(b + s.RR * 128 + 64 + kSkinnyTB * s.RR * 2);
+  s.wbuf_r = b + s.RR * 128;
+  uint8_t* h = b + 2 * s.RR * 128;
+  s.bar = reinterpret_cast<uint64_t*>(h);
+  s.bar_r = s.bar + 1;
+  s.abort_flag = reinterpret_cast<volatile int*>(h + 16);
+  s.xs = reinterpret_cast<__nv_bfloat16*>(h + 64);
+  s.red = reinterpret_cast<float*>(h + 64 + kSkinnyTB * s.RR * 2);
   s.part = s.red + 8 * kSkinnyTB * 64;
-  s.tlist = reinterpret_cast<int*>(s.part + kSkinnyTB * 64);
-  s.logits = reinterpret_cast<float*>(s.tlist + kSkinnyMaxTokens + 1);
+  s.part_r = s.part + kSkinnyTB * 64;
+  s.logits = s.part_r + kSkinnyTB * 64;
+  s.slot = reinterpret_cast<int*>(s.logits + 8);
   if (threadIdx.x == 0) {
     mbar_init(s.bar, 1);
+    mbar_init(s.bar_r, 1);
     *s.abort_flag = 0;
     fence_mbar_init();
   }
@@ -120,25 +127,28 @@ __device__ __forceinline__ SkCta sk_init(uint8_t* raw, int K) {
 }
 
 // Thread 0: TMA loads of this CTA's rows of the slice starting at column
-// col0 (all boxes on the one barrier; rows past the weight read as zero).
-__device__ __forceinline__ void sk_load(const SkCta& s, const CUtensorMap* tm, int col0) {
+// col0 into wbuf (all boxes on barrier bar; rows past the weight read as zero).
+__device__ __forceinline__ void sk_load(const SkCta& s, uint8_t* wbuf, uint64_t* bar, const CUtensorMap* tm,
+                                        int col0) {
   if (threadIdx.x == 0) {
     const int nbox = s.RR / kSkBoxRows;
-    mbar_arrive_expect_tx(s.bar, nbox * kSkBoxRows * 128);
+    mbar_arrive_expect_tx(bar, nbox * kSkBoxRows * 128);
     for (int i = 0; i < nbox; ++i)
-      tma_load_2d(s.wbuf + i * kSkBoxRows * 128, tm, s.bar, col0, s.row0 + i * kSkBoxRows);
+      tma_load_2d(wbuf + i * kSkBoxRows * 128, tm, bar, col0, s.row0 + i * kSkBoxRows);
   }
 }
 
 // part[n][c] = sum over this CTA's rows r of xs[n][r] * W[row0 + r][col0 + c]
-// (columns at or past ncols are zeros). The first call waits for the weights
-// (*loaded tracks it). Returns false if that wait ran out (part is then zero).
-__device__ __forceinline__ bool sk_product(const SkCta& s, int ncols, bool* loaded) {
+// for the slice in wbuf (columns at or past ncols are zeros). The first call
+// for a buffer waits for its weights (*loaded tracks it). Returns false if that
+// wait ran out (part is then zero).
+__device__ __forceinline__ bool sk_product(const SkCta& s, const uint8_t* wbuf, uint64_t* bar, int ncols,
+                                           bool* loaded, float* part) {
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int c8 = (t & 7) * 8, kr = t >> 3;
   bool ok = true;
   if (!*loaded) {
-    ok = __syncthreads_and(mbar_wait(s.bar, 0, s.abort_flag));
+    ok = __syncthreads_and(mbar_wait(bar, 0, s.abort_flag));
     *loaded = true;
   }
   float acc[kSkinnyTB][8];
@@ -147,7 +157,7 @@ __device__ __forceinline__ bool sk_product(const SkCta& s, int ncols, bool* load
 #pragma unroll
     for (int c = 0; c < 8; ++c) acc[n][c] = 0.f;
   if (ok && c8 < ncols) {
-    const uint32_t base = smem_u32(s.wbuf);
+    const uint32_t base = smem_u32(wbuf);
     for (int r = kr; r < s.RR; r += 32) {
       uint32_t w4[4];
       asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
@@ -184,15 +194,16 @@ __device__ __forceinline__ bool sk_product(const SkCta& s, int ncols, bool* load
     float v = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) v += s.red[w * kSkinnyTB * 64 + i];
-    s.part[i] = v;
+    part[i] = v;
   }
+  __syncthreads();  // red is reused by the next product
   return ok;
 }
 
 // After a cluster barrier: the sum over the cluster's ranks (in rank order)
-// of part[token rank][col].
-__device__ __forceinline__ float sk_cluster_sum(const SkCta& s, int col) {
-  const uint32_t a = smem_u32(s.part + s.rank * 64 + col);
+// of part[token rank][col] (part: this CTA's s.part or s.part_r).
+__device__ __forceinline__ float sk_cluster_sum(const SkCta& s, const float* part, int col) {
+  const uint32_t a = smem_u32(part + s.rank * 64 + col);
   float v = 0.f;
 #pragma unroll
   for (int r = 0; r < kSkCluster; ++r) v += ld_dsmem_f32(mapa_shared(a, (uint32_t)r));
@@ -222,77 +233,36 @@ __device__ __forceinline__ void sk_stage_x(const SkCta& s, const DecodeProjParam
   __syncthreads();
 }
 
-// Router decisions for the groups of slice `sl` (columns [64 sl, 64 sl + 64)
-// of Wr): token n, groups [64 sl / RM, ...), one thread each.
+// Thread 0 of rank q, for token n of a pass: the decision of group g from
+// the logits in s.logits; the slot of expert e among the selections (-1:
+// not selected) into *s.slot; the e = 0 cluster writes sel, w and margin.
 template <int RM>
-__device__ __forceinline__ void sk_decide(const SkCta& s, const DecodeProjParams& p, int sl, int n) {
-  const int gpsl = 64 / RM;  // groups per slice
-  const int g = sl * gpsl + (int)threadIdx.x;
-  if ((int)threadIdx.x >= gpsl || g >= p.G) return;
+__device__ __forceinline__ void sk_decide(const SkCta& s, const DecodeProjParams& p, int g, int e, int n) {
   float l[RM];
 #pragma unroll
-  for (int e = 0; e < RM; ++e) l[e] = s.logits[threadIdx.x * RM + e];
-  int32_t sl_[8];
+  for (int i = 0; i < RM; ++i) l[i] = s.logits[i];
+  int32_t sl[8];
   float wl[8];
   float mg;
-  route_decide<RM, false>(l, p.k, true, sl_, wl, &mg);
-  for (int j = 0; j < p.k; ++j) {
-    p.sel[((size_t)n * p.G + g) * p.k + j] = sl_[j];
-    p.w[((size_t)n * p.G + g) * p.k + j] = wl[j];
-  }
-  if (p.margin) p.margin[(size_t)n * p.G + g] = mg;
-}
-
-// Cluster sl: router logits of slice sl for the B new tokens, then the
-// decisions of the slice's groups.
-__global__ void __cluster_dims__(kSkCluster, 1, 1) __launch_bounds__(kSkinnyThreads)
-    decode_route_kernel(const __grid_constant__ DecodeProjParams p) {
-  extern __shared__ uint8_t sk_raw[];
-  SkCta s = sk_init(sk_raw, p.D);
-  const int sl = blockIdx.x / kSkCluster;
-  const int GM = p.G * p.M;
-  sk_load(s, &p.tmWr, sl * 64);
-  // the previous step's output kernel reads w: wait before writing it (and
-  // before letting the projection launch in)
-  pdl_wait();
-  pdl_trigger();
-  bool loaded = false, ok = true;
-  int tok[kSkinnyTB];
-  for (int n0 = 0; n0 < p.B; n0 += kSkinnyTB) {
-    const int nt = min(kSkinnyTB, p.B - n0);
-#pragma unroll
-    for (int n = 0; n < kSkinnyTB; ++n) tok[n] = n0 + n;
-    sk_stage_x(s, p, tok, nt);
-    ok = sk_product(s, GM - sl * 64, &loaded) && ok;
-    cluster_sync();  // every rank's part is ready
-    if (threadIdx.x < 64) {
-      const int col = sl * 64 + (int)threadIdx.x;
-      s.logits[threadIdx.x] = sk_cluster_sum(s, threadIdx.x) + (p.br && col < GM ? p.br[col] : 0.f);
+  route_decide<RM, false>(l, p.k, true, sl, wl, &mg);
+  int slot = -1;
+  for (int j = 0; j < p.k; ++j)
+    if (sl[j] == e) slot = j;
+  *s.slot = slot;
+  if (e == 0) {
+    for (int j = 0; j < p.k; ++j) {
+      p.sel[((size_t)n * p.G + g) * p.k + j] = sl[j];
+      p.w[((size_t)n * p.G + g) * p.k + j] = wl[j];
     }
-    __syncthreads();
-    if (ok && s.rank < nt) {
-      switch (p.M) {
-        case 1: sk_decide<1>(s, p, sl, n0 + s.rank); break;
-        case 2: sk_decide<2>(s, p, sl, n0 + s.rank); break;
-        case 4: sk_decide<4>(s, p, sl, n0 + s.rank); break;
-        default: sk_decide<8>(s, p, sl, n0 + s.rank); break;
-      }
-    }
-    cluster_sync();  // the ranks are done reading part
-  }
-  if (!ok) {  // a wait ran out: let copies in flight land before the block exits
-    const unsigned long long t0 = globaltimer_ns();
-    while (globaltimer_ns() - t0 < 100000ull) {}
+    if (p.margin) p.margin[(size_t)n * p.G + g] = mg;
   }
 }
 
 // Cluster h: the projection of one 64-column weight slice (see the file
-// comment). The K/V and shared-query clusters stage x and multiply before
-// the wait for the routing launch, and wait before writing; the routed
-// clusters need sel first.
+// comment); a routed head's cluster also multiplies the 64-column slice of
+// Wr that holds its group's logits and decides.
 __global__ void __cluster_dims__(kSkCluster, 1, 1) __launch_bounds__(kSkinnyThreads)
     decode_proj_kernel(const __grid_constant__ DecodeProjParams p) {
-  pdl_trigger();
   extern __shared__ uint8_t sk_raw[];
   SkCta s = sk_init(sk_raw, p.D);
   const int GM = p.G * p.M;
@@ -316,56 +286,59 @@ __global__ void __cluster_dims__(kSkCluster, 1, 1) __launch_bounds__(kSkinnyThre
       col0 = h * 64;
     }
   }
-  sk_load(s, W, col0);
-  int ntok;
-  if (!routed) {
-    ntok = p.B;
-    for (int i = threadIdx.x; i < p.B; i += kSkinnyThreads) s.tlist[i] = i;
-  } else {
-    pdl_wait();  // sel of the routing launch
-    if (threadIdx.x == 0) {
-      // the tokens that selected expert e of group g, in order
-      int c = 0;
-      for (int n = 0; n < p.B; ++n)
-        for (int j = 0; j < p.k; ++j)
-          if (p.sel[((size_t)n * p.G + g) * p.k + j] == e) s.tlist[c++] = n;
-      s.tlist[kSkinnyMaxTokens] = c;
+  const int rcol = (g * p.M / 64) * 64;  // Wr slice holding group g's logits
+  const int roff = g * p.M - rcol;
+  // weights depend on no launch; x, and the buffers the previous step's
+  // launches read (caches, Q, sel, w), only after the wait
+  sk_load(s, s.wbuf, s.bar, W, col0);
+  if (routed) sk_load(s, s.wbuf_r, s.bar_r, &p.tmWr, rcol);
+  pdl_wait();
+  pdl_trigger();
+  bool loaded = false, loaded_r = false, ok = true;
+  int tok[kSkinnyTB];
+  for (int n0 = 0; n0 < p.B; n0 += kSkinnyTB) {
+    const int nt = min(kSkinnyTB, p.B - n0);
+#pragma unroll
+    for (int n = 0; n < kSkinnyTB; ++n) tok[n] = n0 + n;
+    sk_stage_x(s, p, tok, nt);
+    ok = sk_product(s, s.wbuf, s.bar, 64, &loaded, s.part) && ok;
+    if (routed) ok = sk_product(s, s.wbuf_r, s.bar_r, roff + p.M, &loaded_r, s.part_r) && ok;
+    cluster_sync();  // every rank's partials are ready
+    const int n = n0 + s.rank;  // this rank's token
+    int slot = 0;
+    if (routed) {
+      if ((int)threadIdx.x < p.M)
+        s.logits[threadIdx.x] = sk_cluster_sum(s, s.part_r, roff + threadIdx.x) + (p.br ? p.br[g * p.M + threadIdx.x] : 0.f);
+      __syncthreads();
+      if (threadIdx.x == 0 && s.rank < nt && ok) {
+        switch (p.M) {
+          case 1: sk_decide<1>(s, p, g, e, n); break;
+          case 2: sk_decide<2>(s, p, g, e, n); break;
+          case 4: sk_decide<4>(s, p, g, e, n); break;
+          default: sk_decide<8>(s, p, g, e, n); break;
+        }
+      }
+      __syncthreads();
+      slot = *s.slot;
     }
-  }
-  __syncthreads();
-  if (routed) ntok = s.tlist[kSkinnyMaxTokens];
-  bool loaded = false, ok = true;
-  for (int n0 = 0; n0 < ntok; n0 += kSkinnyTB) {
-    const int nt = min(kSkinnyTB, ntok - n0);
-    sk_stage_x(s, p, s.tlist + n0, nt);
-    ok = sk_product(s, 64, &loaded) && ok;
-    pdl_wait();      // earlier launches are done with the rows written below
-    cluster_sync();  // every rank's part is ready
-    if (ok && threadIdx.x < 64 && s.rank < nt) {
+    if (ok && threadIdx.x < 64 && s.rank < nt && slot >= 0) {
       const int c = threadIdx.x;
-      const int tok = s.tlist[n0 + s.rank];
-      const __nv_bfloat16 v = __float2bfloat16_rn(sk_cluster_sum(s, c));
+      const __nv_bfloat16 v = __float2bfloat16_rn(sk_cluster_sum(s, s.part, c));
       if (blk < 2 * p.G) {
-        const int L = p.cache_len[tok];
+        const int L = p.cache_len[n];
         if (L < 0 || L >= p.T) {
           if (c == 0) flag_bounds_error();
         } else {
-          (blk < p.G ? p.Kc : p.Vc)[(((size_t)tok * p.T + L) * p.G + g) * 64 + c] = v;
+          (blk < p.G ? p.Kc : p.Vc)[(((size_t)n * p.T + L) * p.G + g) * 64 + c] = v;
         }
       } else if (!routed) {
-        p.Q[((size_t)tok * Ha + p.G * p.k) * 64 + c] = v;
+        p.Q[((size_t)n * Ha + p.G * p.k) * 64 + c] = v;
       } else {
-        // slot of expert e among the token's selections
-        int j = 0;
-        for (int jj = 0; jj < p.k; ++jj)
-          if (p.sel[((size_t)tok * p.G + g) * p.k + jj] == e) j = jj;
-        p.Q[((size_t)tok * Ha + g * p.k + j) * 64 + c] = v;
+        p.Q[((size_t)n * Ha + g * p.k + slot) * 64 + c] = v;
       }
     }
-    cluster_sync();  // the ranks are done reading part
+    cluster_sync();  // the ranks are done reading the partials
   }
-  pdl_wait();  // on every path, so this grid completes after the ones it depends on
-  if (!loaded) ok = __syncthreads_and(mbar_wait(s.bar, 0, s.abort_flag));  // a slice no token used
   if (!ok) {  // a wait ran out: let copies in flight land before the block exits
     const unsigned long long t0 = globaltimer_ns();
     while (globaltimer_ns() - t0 < 100000ull) {}
@@ -382,7 +355,7 @@ __global__ void __cluster_dims__(kSkCluster, 1, 1) __launch_bounds__(kSkinnyThre
   const int Ka = (Gk + p.G + 1) * 64;
   SkCta s = sk_init(sk_raw, Ka);
   const int col0 = (blockIdx.x / kSkCluster) * 64;
-  sk_load(s, &p.tmWo, col0);  // Wo depends on no launch
+  sk_load(s, s.wbuf, s.bar, &p.tmWo, col0);  // Wo depends on no launch
   pdl_wait();
   bool loaded = false, ok = true;
   for (int n0 = 0; n0 < p.B; n0 += kSkinnyTB) {
@@ -419,10 +392,11 @@ __global__ void __cluster_dims__(kSkCluster, 1, 1) __launch_bounds__(kSkinnyThre
       reinterpret_cast<uint4*>(s.xs)[i] = v;
     }
     __syncthreads();
-    ok = sk_product(s, 64, &loaded) && ok;
+    ok = sk_product(s, s.wbuf, s.bar, 64, &loaded, s.part) && ok;
     cluster_sync();  // every rank's part is ready
     if (ok && threadIdx.x < 64 && s.rank < nt)
-      p.y[(size_t)(n0 + s.rank) * p.D + col0 + threadIdx.x] = __float2bfloat16_rn(sk_cluster_sum(s, threadIdx.x));
+      p.y[(size_t)(n0 + s.rank) * p.D + col0 + threadIdx.x] =
+          __float2bfloat16_rn(sk_cluster_sum(s, s.part, threadIdx.x));
     cluster_sync();  // the ranks are done reading part
   }
   if (!ok) {  // a wait ran out: let copies in flight land before the block exits

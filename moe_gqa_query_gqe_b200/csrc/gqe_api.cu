@@ -995,9 +995,9 @@ int gqe_decode(const gqe_dims* d, const int32_t* cache_len, const void* x_new, c
   pp.M = d->M;
   pp.k = d->k;
   if (skinny) {
-    // a few new tokens: routing, K/V (written straight into the caches at
-    // cache_len) and the queries as skinny products, one 8-CTA cluster per
-    // 64-column weight slice
+    // a few new tokens: K/V (written straight into the caches at
+    // cache_len), the routing and the queries as skinny products in one
+    // launch, one 8-CTA cluster per 64-column weight slice
     const int GM = d->G * d->M, Ka = (d->G * d->k + d->G + 1) * 64;
     GQE_TRY(tmap_rows(&pp.tmWq, Wq, d->D, (GM + 1) * 64, (GM + 1) * 64, kSkBoxRows));
     GQE_TRY(tmap_rows(&pp.tmWk, Wk, d->D, d->G * 64, d->G * 64, kSkBoxRows));
@@ -1005,9 +1005,6 @@ int gqe_decode(const gqe_dims* d, const int32_t* cache_len, const void* x_new, c
     GQE_TRY(tmap_rows(&pp.tmWr, Wr, d->D, GM, GM, kSkBoxRows));
     GQE_TRY(tmap_rows(&pp.tmWo, Wo, Ka, d->D, d->D, kSkBoxRows));
     const int smem = sk_smem(d->D);
-    GQE_TRY(set_smem(decode_route_kernel, smem));
-    GQE_TRY(launch_pdl(decode_route_kernel, dim3((unsigned)cdiv(GM, 64) * kSkCluster), dim3(kSkinnyThreads), smem,
-                       st, pp));
     GQE_TRY(set_smem(decode_proj_kernel, smem));
     GQE_TRY(launch_pdl(decode_proj_kernel, dim3((2 * d->G + 1 + GM) * kSkCluster), dim3(kSkinnyThreads), smem, st,
                        pp));
