@@ -728,6 +728,25 @@ def main():
     torch.cuda.synchronize()
     dense_ms = sum(a.elapsed_time(b) for a, b in devs) / args.steps
 
+    # ---- the same layer with the selected heads' queries only (per-expert
+    # gather; gqe_forward takes the dense product when M <= 2k): same y, bit
+    # for bit, reported beside the headline --------------------------------
+    ws_var = gqe.workspace(d, gqe.OP_FORWARD_VARIANT)
+    y_sel = torch.empty_like(y)
+
+    def gather_step():
+        gqe.gqe_forward_variant(d, gqe.COMBINE_SLOT | gqe.QPROJ_GATHER, inp["x"], inp["Wq"], inp["Wk"], inp["Wv"],
+                                inp["Wr"], inp["br"], inp["Wo"], y_sel, ws_var)
+
+    g_gather = as_graph(gather_step)
+    timed(g_gather.replay, args.warmup)
+    gevs = timed(g_gather.replay, args.steps)
+    torch.cuda.synchronize()
+    gather_ms = sum(a.elapsed_time(b) for a, b in gevs) / args.steps
+    gather_ms = reduce_max([gather_ms], world, dev)[0]
+    gather_same = bool(torch.equal(y_sel, y))
+    del g_gather
+
     # ---- end to end through the host-buffer entry point ---------------------
     x_host = inp["x"].cpu().pin_memory()
     y_host = torch.empty(N, d.D, dtype=torch.bfloat16).pin_memory()
@@ -773,6 +792,11 @@ def main():
                     "h2d_bytes_per_step": N * d.D * 2, "d2h_bytes_per_step": N * d.D * 2,
                     "entry": "gqe_forward_host"},
             "gpu_launches": launches_per_step * args.steps,
+            "qproj_path": "dense product over all routed heads, selected rows kept" if d.M <= 2 * d.k
+                          else "selected heads only (per-expert gather)",
+            "selected_heads_only": {"ms_per_step": gather_ms, "tokens_per_s": job_throughput(world, N, gather_ms),
+                                    "speedup_vs_dense": dense_ms / gather_ms, "same_y_bits": gather_same,
+                                    "entry": "gqe_forward_variant(COMBINE_SLOT | QPROJ_GATHER)"},
             "timing": "each step one CUDA-graph replay of gqe_forward; stage_ms from the four stage calls"}
 
     # long-context keys: one GPU, headline workload only (a scaling run keeps its timed work short)

@@ -91,6 +91,24 @@ enum gqe_combine_mode {
                                    is computed)                                               */
 };
 
+/* How gqe_forward_variant computes the selected experts' queries, or'ed into
+ * its `mode`. Both give the same Q (the same dot products, accumulated in the
+ * same order); they differ in the work done.
+ *   GQE_QPROJ_AUTO   : GQE_QPROJ_DENSE when M <= 2k, else GQE_QPROJ_GATHER
+ *                      (what gqe_forward does)
+ *   GQE_QPROJ_GATHER : selected heads only: the tokens of every (sequence,
+ *                      group, expert) are compacted and their rows of x
+ *                      gathered per expert (gqe_route + gqe_qproj)
+ *   GQE_QPROJ_DENSE  : every routed head's query is projected on the tensor
+ *                      cores and each token's selected rows are kept (at
+ *                      most M/k times the selected heads' flops, no
+ *                      compaction and no gather) */
+enum gqe_qproj_path {
+  GQE_QPROJ_AUTO = 0,
+  GQE_QPROJ_GATHER = 0x100,
+  GQE_QPROJ_DENSE = 0x200
+};
+
 /* Workspace bytes the operation needs for these dims (0 if none); returns 0
  * and nothing else for invalid dims (check with gqe_validate_dims). */
 size_t gqe_workspace_bytes(const gqe_dims* d, int op);
@@ -217,6 +235,11 @@ int gqe_combine(const gqe_dims* d, const void* O, const float* w,
 
 /*
  * gqe_forward -- route -> qproj -> attn -> combine on one stream.
+ * The selected queries follow GQE_QPROJ_AUTO (enum gqe_qproj_path): for
+ * M <= 2k a dense product over all routed heads keeps each token's selected
+ * rows, and the segment lists (seg_off, seg_tok, row_map) are not built;
+ * for M > 2k the selected tokens are gathered per expert. Either way Q, and
+ * so y, is the same as gqe_route + gqe_qproj + gqe_attn + gqe_combine give.
  * ws: gqe_workspace_bytes(d, GQE_OP_FORWARD); it holds every intermediate
  * (sel, w, margin, segments, Q, K, V, O, ...).
  */
@@ -261,6 +284,7 @@ int gqe_forward_host(const gqe_dims* d, const void* x_host, const void* Wq,
  *     GQE_COMBINE_WEIGHTED     (G*k + 1)*dh
  *     GQE_COMBINE_GLOBAL_SLOT  (G*k + 2)*dh
  *     GQE_COMBINE_NO_SHARED    (G*k + G)*dh
+ * `mode` may also carry one enum gqe_qproj_path value (or'ed in).
  * ws: gqe_workspace_bytes(d, GQE_OP_FORWARD_VARIANT). An unknown mode returns
  * GQE_ERR_INVALID_ARG. Everything else as gqe_forward.
  */

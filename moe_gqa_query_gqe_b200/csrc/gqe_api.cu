@@ -829,8 +829,9 @@ int gqe_combine(const gqe_dims* d, const void* O, const float* w, const void* Wo
 
 // The layer: mode GQE_COMBINE_SLOT is the GQE output construction; the other
 // modes are the ablation variants (see gqe_forward_variant).
-int do_forward(const gqe_dims* d, int mode, const void* x, const void* Wq, const void* Wk, const void* Wv,
+int do_forward(const gqe_dims* d, int mode_bits, const void* x, const void* Wq, const void* Wk, const void* Wv,
                const void* Wr, const float* br, const void* Wo, void* y, void* ws, cudaStream_t st) {
+  const int mode = mode_bits & 0xff, qpath = mode_bits & (GQE_QPROJ_GATHER | GQE_QPROJ_DENSE);
   Carver c{static_cast<uint8_t*>(ws)};
   FwdWs f = carve_forward(c, d);
   const size_t N = (size_t)d->B * d->T;
@@ -847,7 +848,7 @@ int do_forward(const gqe_dims* d, int mode, const void* x, const void* Wq, const
   // (logits and decisions), then the selected queries: a dense product over
   // the routed heads that keeps the selected rows, or (M > 2k) the
   // compaction and the gather
-  const bool qsel = qproj_dense_select(d);
+  const bool qsel = qpath == GQE_QPROJ_DENSE || (qpath == GQE_QPROJ_AUTO && qproj_dense_select(d));
   DenseSeg segs[3];
   kv_segments(d, Wq, Wk, Wv, f.Q, f.K, f.V, segs);
   GemmParams p;
@@ -896,7 +897,9 @@ int gqe_forward_variant(const gqe_dims* d, int mode, const void* x, const void* 
                         const void* Wr, const float* br, const void* Wo, void* y, void* ws, size_t ws_bytes,
                         void* stream) {
   GQE_TRY(check_dims(d));
-  if (mode < GQE_COMBINE_SLOT || mode > GQE_COMBINE_NO_SHARED) return GQE_ERR_INVALID_ARG;
+  const int cmode = mode & 0xff, qpath = mode & ~0xff;
+  if (cmode < GQE_COMBINE_SLOT || cmode > GQE_COMBINE_NO_SHARED) return GQE_ERR_INVALID_ARG;
+  if (qpath != GQE_QPROJ_AUTO && qpath != GQE_QPROJ_GATHER && qpath != GQE_QPROJ_DENSE) return GQE_ERR_INVALID_ARG;
   GQE_TRY(check_ptrs({x, Wq, Wk, Wv, Wr, Wo, y}));
   if (br && !aligned16(br)) return GQE_ERR_INVALID_ARG;
   GQE_TRY(check_ws(ws, ws_bytes, gqe_workspace_bytes(d, GQE_OP_FORWARD_VARIANT)));

@@ -21,6 +21,8 @@ STATUS = {0: "GQE_OK", -1: "GQE_ERR_INVALID_ARG", -2: "GQE_ERR_UNSUPPORTED", -3:
 OP_ROUTE, OP_QPROJ, OP_ATTN, OP_COMBINE, OP_FORWARD, OP_DENSE, OP_FORWARD_HOST, OP_DECODE, OP_FORWARD_VARIANT = \
     1, 2, 3, 4, 5, 6, 7, 8, 9
 COMBINE_SLOT, COMBINE_HARD, COMBINE_WEIGHTED, COMBINE_GLOBAL_SLOT, COMBINE_NO_SHARED = 0, 1, 2, 3, 4
+# selected-query path of gqe_forward_variant, or'ed into the mode (enum gqe_qproj_path)
+QPROJ_AUTO, QPROJ_GATHER, QPROJ_DENSE = 0, 0x100, 0x200
 
 # every symbol include/gqe.h declares
 EXPORTS = ("gqe_workspace_bytes", "gqe_validate_dims", "gqe_route", "gqe_route_noalloc", "gqe_qproj", "gqe_attn", "gqe_combine",
@@ -158,8 +160,10 @@ def gqe_forward(dims, x, Wq, Wk, Wv, Wr, br, Wo, y, ws, stream=None) -> None:
 
 def gqe_forward_variant(dims, mode, x, Wq, Wk, Wv, Wr, br, Wo, y, ws, stream=None) -> None:
     """gqe_forward with the output construction `mode` (COMBINE_SLOT, _HARD,
-    _WEIGHTED, _GLOBAL_SLOT, _NO_SHARED). Wo has (G*k + G + 1), (G*k + 1),
-    (G*k + 1), (G*k + 2) or (G*k + G) blocks of 64 rows respectively."""
+    _WEIGHTED, _GLOBAL_SLOT, _NO_SHARED), optionally or'ed with a selected-query
+    path (QPROJ_AUTO, QPROJ_GATHER, QPROJ_DENSE). Wo has (G*k + G + 1),
+    (G*k + 1), (G*k + 1), (G*k + 2) or (G*k + G) blocks of 64 rows
+    respectively."""
     _call("gqe_forward_variant", ctypes.byref(dims_struct(dims)), int(mode), _ptr(x), _ptr(Wq), _ptr(Wk), _ptr(Wv),
           _ptr(Wr), _ptr(br), _ptr(Wo), _ptr(y), _ptr(ws), ws.numel(), _stream(stream))
 

@@ -105,10 +105,12 @@ def test_null_and_misaligned_pointers_are_rejected_before_any_launch():
     assert _raw("gqa_dense_forward", dp, P, P, P, P, P, None, P, 1 << 30, None) == -1
     # gqe_forward_variant: unknown combine mode, then a valid mode without workspace
     vargs = [P, P, P, P, P, None, P, P]
-    for bad_mode in (-1, 5, 7):
+    # (or an unknown selected-query path: both, or a bit outside the enum)
+    for bad_mode in (-1, 5, 7, 0x300, 0x400, 0x105):
         assert _raw("gqe_forward_variant", dp, bad_mode, *vargs, P, 1 << 30, None) == -1
     for mode in range(5):
-        assert _raw("gqe_forward_variant", dp, mode, *vargs, None, 0, None) == -3
+        for qpath in (gqe.QPROJ_AUTO, gqe.QPROJ_GATHER, gqe.QPROJ_DENSE):
+            assert _raw("gqe_forward_variant", dp, mode | qpath, *vargs, None, 0, None) == -3
     # gqe_decode: null cache_len, misaligned x_new, missing workspace
     args = [P, P, P, P, P, P, None, P, P, P, P, P, P]
     assert _raw("gqe_decode", dp, None, *args[1:], P, 1 << 30, None) == -1

@@ -98,6 +98,23 @@ def test_layer_end_to_end(cases, name):
 
 
 @pytest.mark.parametrize("name", ["tiny_b2_t256", "ragged_b3_t300", "pool4_k2_skewed_t384", "pool8_k4_t136",
+                                  "single_token_b4", "one_group_g1_m8_k2", "k_equals_m_t260"])
+def test_selected_query_paths_agree_bitwise(cases, name):
+    """The two ways of computing the selected queries (the per-expert gather,
+    selected heads only; the dense product over all routed heads with the
+    selected rows kept) give the stage path's y, bit for bit, on every shape."""
+    import moe_gqa_query_gqe_b200 as gqe
+    d, inp, dev, st = cases[name]
+    ws = gqe.workspace(d, gqe.OP_FORWARD_VARIANT)
+    for qpath in (gqe.QPROJ_GATHER, gqe.QPROJ_DENSE):
+        y = torch.full((d.B * d.T, d.D), float("nan"), dtype=torch.bfloat16, device="cuda")
+        gqe.gqe_forward_variant(d, gqe.COMBINE_SLOT | qpath, dev["x"], dev["Wq"], dev["Wk"], dev["Wv"], dev["Wr"],
+                                dev["br"], dev["Wo"], y, ws)
+        assert gqe.gqe_check_error() == 0
+        assert torch.equal(y.cpu(), st["y"]), f"qpath {qpath:#x}"
+
+
+@pytest.mark.parametrize("name", ["tiny_b2_t256", "ragged_b3_t300", "pool4_k2_skewed_t384", "pool8_k4_t136",
                                   "single_token_b4"])
 def test_dense_gqa_baseline(cases, name):
     d, inp, dev, st = cases[name]
