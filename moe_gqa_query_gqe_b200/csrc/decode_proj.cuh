@@ -16,16 +16,17 @@
 // slice is read by its own cluster of kSkCluster CTAs. CTA rank q loads rows
 // [q RR, q RR + RR) of the slice by TMA (RR: the slice's rows / kSkCluster,
 // rounded up to whole kSkBoxRows boxes) and multiplies them with the same
-// rows of the tokens' inputs; the eight partial sums meet in distributed
-// shared memory, where rank q adds up token q's 64 columns of a pass of
-// eight tokens (ranks in order, so the sum is the same on every run).
+// rows of all the tokens' inputs (staged once, up to kSkinnyMaxTokens); the
+// eight partial sums meet in distributed shared memory, where rank q adds up
+// tokens [2q, 2q + 2) (ranks in order, so the sum is the same on every run).
+// A launch takes two cluster barriers whatever the token count.
 //   decode_proj_kernel : 2G + 1 + G*M clusters: K and V of group g (written
 //                        into the caches at cache_len[b]), the shared head's
 //                        query, and routed head h = g*M + e: its query and
 //                        group g's router logits x Wr + br for every token;
-//                        rank q decides token q of a pass for group g and
-//                        keeps the query row if the token selected e (the
-//                        e = 0 cluster writes sel, w, margin)
+//                        rank q decides its tokens for group g and keeps a
+//                        token's query row if it selected e (the e = 0
+//                        cluster writes sel, w, margin)
 //   decode_out_kernel  : D / 64 clusters: y = A Wo, A = [concat | per-group
 //                        slot sum_j w_j O_j | shared] built for the CTA's rows
 //                        (A's columns) from O and w (the slot rounded to
@@ -43,12 +44,15 @@
 
 namespace gqe {
 
+// Above 16 new tokens the CUDA-core products cost more than the prefill
+// path's tensor-core tiles (64 tokens: 52 + 31 us against three 17 us GEMMs).
 constexpr int kSkinnyMaxTokens = 16;
 constexpr int kSkCluster = 8;
 constexpr int kSkinnyThreads = 256;
-constexpr int kSkinnyTB = 8;     // tokens per pass (rank q adds token q)
-constexpr int kSkBoxRows = 32;   // TMA box: 64 columns x 32 rows, 4 KB
-static_assert(kSkinnyTB == kSkCluster, "rank q reduces token q of a pass");
+constexpr int kSkinnyTB = 8;   // tokens per register block of a product
+constexpr int kSkPerRank = kSkinnyMaxTokens / kSkCluster;  // tokens a rank adds up
+constexpr int kSkBoxRows = 32; // TMA box: 64 columns x 32 rows, 4 KB
+static_assert(kSkPerRank <= 8 && kSkinnyMaxTokens % kSkinnyTB == 0, "decision area and register blocks");
 
 struct DecodeProjParams {
   // weights as TMA tensor maps: box 64 columns x kSkBoxRows rows, 128-byte swizzle
@@ -73,14 +77,15 @@ __host__ __device__ inline int sk_rows(int K) {
   return (r + kSkBoxRows - 1) / kSkBoxRows * kSkBoxRows;
 }
 // Shared memory (from a 1024-aligned base): the CTA's weight rows wbuf
-// [RR][128 B] and, for a routed head, its router rows wbuf_r [RR][128 B];
-// their barriers and the abort flag (64 B); the inputs' rows xs [TB][RR]
-// (bf16); per-warp partials red [8][TB][64]; the CTA's partials part and
-// part_r [TB][64] (read by the cluster); the decision area (64 B: a group's
-// logits, the selected slot).
-__host__ __device__ inline int sk_smem(int K) {
+// [RR][128 B] and, with `router`, the router rows wbuf_r [RR][128 B]; their
+// barriers and the abort flag (64 B); all tokens' input rows xs
+// [kSkinnyMaxTokens][RR] (bf16); per-warp partials red [8][TB][64]; the CTA's
+// partials part (and, with `router`, part_r) [kSkinnyMaxTokens][64] (read by
+// the cluster); the decision area: logits [8][8] and slots [8].
+__host__ __device__ inline int sk_smem(int K, bool router) {
   const int RR = sk_rows(K);
-  return 1024 + 2 * RR * 128 + 64 + kSkinnyTB * RR * 2 + 8 * kSkinnyTB * 64 * 4 + 2 * kSkinnyTB * 64 * 4 + 64;
+  return 1024 + (router ? 2 : 1) * RR * 128 + 64 + kSkinnyMaxTokens * RR * 2 + 8 * kSkinnyTB * 64 * 4 +
+         (router ? 2 : 1) * kSkinnyMaxTokens * 64 * 4 + 64 * 4 + 8 * 4;
 }
 
 struct SkCta {
@@ -93,12 +98,12 @@ struct SkCta {
   float* red;
   float* part;
   float* part_r;
-  float* logits;  // [8]
-  int* slot;      // [1]
+  float* logits;  // [8 tokens][8]
+  int* slot;      // [8 tokens]
   int RR, row0, rank;
 };
 
-__device__ __forceinline__ SkCta sk_init(uint8_t* raw, int K) {
+__device__ __forceinline__ SkCta sk_init(uint8_t* raw, int K, bool router) {
   SkCta s;
   uint8_t* b = raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
   s.RR = sk_rows(K);
@@ -106,16 +111,16 @@ __device__ __forceinline__ SkCta sk_init(uint8_t* raw, int K) {
   s.row0 = s.rank * s.RR;
   s.wbuf = b;
   s.wbuf_r = b + s.RR * 128;
-  uint8_t* h = b + 2 * s.RR * 128;
+  uint8_t* h = b + (router ? 2 : 1) * s.RR * 128;
   s.bar = reinterpret_cast<uint64_t*>(h);
   s.bar_r = s.bar + 1;
   s.abort_flag = reinterpret_cast<volatile int*>(h + 16);
   s.xs = reinterpret_cast<__nv_bfloat16*>(h + 64);
-  s.red = reinterpret_cast<float*>(h + 64 + kSkinnyTB * s.RR * 2);
+  s.red = reinterpret_cast<float*>(h + 64 + kSkinnyMaxTokens * s.RR * 2);
   s.part = s.red + 8 * kSkinnyTB * 64;
-  s.part_r = s.part + kSkinnyTB * 64;
-  s.logits = s.part_r + kSkinnyTB * 64;
-  s.slot = reinterpret_cast<int*>(s.logits + 8);
+  s.part_r = s.part + kSkinnyMaxTokens * 64;  // (router only)
+  s.logits = s.part + (router ? 2 : 1) * kSkinnyMaxTokens * 64;
+  s.slot = reinterpret_cast<int*>(s.logits + 64);
   if (threadIdx.x == 0) {
     mbar_init(s.bar, 1);
     mbar_init(s.bar_r, 1);
@@ -139,90 +144,88 @@ __device__ __forceinline__ void sk_load(const SkCta& s, uint8_t* wbuf, uint64_t*
 }
 
 // part[n][c] = sum over this CTA's rows r of xs[n][r] * W[row0 + r][col0 + c]
-// for the slice in wbuf (columns at or past ncols are zeros). The first call
-// for a buffer waits for its weights (*loaded tracks it). Returns false if that
-// wait ran out (part is then zero).
-__device__ __forceinline__ bool sk_product(const SkCta& s, const uint8_t* wbuf, uint64_t* bar, int ncols,
-                                           bool* loaded, float* part) {
+// for tokens n < ntok and the slice in wbuf (columns at or past ncols are
+// zeros), eight tokens per register block. Waits for the weights first.
+// Returns false if that wait ran out (part is then zero).
+__device__ __forceinline__ bool sk_product(const SkCta& s, const uint8_t* wbuf, uint64_t* bar, int ncols, int ntok,
+                                           float* part) {
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int c8 = (t & 7) * 8, kr = t >> 3;
-  bool ok = true;
-  if (!*loaded) {
-    ok = __syncthreads_and(mbar_wait(bar, 0, s.abort_flag));
-    *loaded = true;
-  }
-  float acc[kSkinnyTB][8];
-#pragma unroll
-  for (int n = 0; n < kSkinnyTB; ++n)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[n][c] = 0.f;
-  if (ok && c8 < ncols) {
-    const uint32_t base = smem_u32(wbuf);
-    for (int r = kr; r < s.RR; r += 32) {
-      uint32_t w4[4];
-      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                   : "=r"(w4[0]), "=r"(w4[1]), "=r"(w4[2]), "=r"(w4[3])
-                   : "r"(base + r * 128 + ((((c8 >> 3) ^ (r & 7))) << 4)));
-      float wf[8];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        wf[2 * e] = bf16lo_to_f32(w4[e]);
-        wf[2 * e + 1] = bf16hi_to_f32(w4[e]);
-      }
-#pragma unroll
-      for (int n = 0; n < kSkinnyTB; ++n) {
-        const float xv = __bfloat162float(s.xs[n * s.RR + r]);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[n][c] = fmaf(xv, wf[c], acc[n][c]);
-      }
-    }
-  }
-#pragma unroll
-  for (int n = 0; n < kSkinnyTB; ++n)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      acc[n][c] += __shfl_xor_sync(0xffffffffu, acc[n][c], 8);
-      acc[n][c] += __shfl_xor_sync(0xffffffffu, acc[n][c], 16);
-    }
-  if (lane < 8)
+  const bool ok = __syncthreads_and(mbar_wait(bar, 0, s.abort_flag));
+  const uint32_t base = smem_u32(wbuf);
+  for (int n0 = 0; n0 < ntok; n0 += kSkinnyTB) {
+    float acc[kSkinnyTB][8];
 #pragma unroll
     for (int n = 0; n < kSkinnyTB; ++n)
 #pragma unroll
-      for (int c = 0; c < 8; ++c) s.red[(warp * kSkinnyTB + n) * 64 + c8 + c] = acc[n][c];
-  __syncthreads();
-  for (int i = t; i < kSkinnyTB * 64; i += kSkinnyThreads) {
-    float v = 0.f;
+      for (int c = 0; c < 8; ++c) acc[n][c] = 0.f;
+    if (ok && c8 < ncols) {
+      for (int r = kr; r < s.RR; r += 32) {
+        uint32_t w4[4];
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w4[0]), "=r"(w4[1]), "=r"(w4[2]), "=r"(w4[3])
+                     : "r"(base + r * 128 + ((((c8 >> 3) ^ (r & 7))) << 4)));
+        float wf[8];
 #pragma unroll
-    for (int w = 0; w < 8; ++w) v += s.red[w * kSkinnyTB * 64 + i];
-    part[i] = v;
+        for (int e = 0; e < 4; ++e) {
+          wf[2 * e] = bf16lo_to_f32(w4[e]);
+          wf[2 * e + 1] = bf16hi_to_f32(w4[e]);
+        }
+#pragma unroll
+        for (int n = 0; n < kSkinnyTB; ++n) {
+          const float xv = __bfloat162float(s.xs[(n0 + n) * s.RR + r]);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) acc[n][c] = fmaf(xv, wf[c], acc[n][c]);
+        }
+      }
+    }
+#pragma unroll
+    for (int n = 0; n < kSkinnyTB; ++n)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        acc[n][c] += __shfl_xor_sync(0xffffffffu, acc[n][c], 8);
+        acc[n][c] += __shfl_xor_sync(0xffffffffu, acc[n][c], 16);
+      }
+    if (lane < 8)
+#pragma unroll
+      for (int n = 0; n < kSkinnyTB; ++n)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) s.red[(warp * kSkinnyTB + n) * 64 + c8 + c] = acc[n][c];
+    __syncthreads();
+    for (int i = t; i < kSkinnyTB * 64; i += kSkinnyThreads) {
+      float v = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) v += s.red[w * kSkinnyTB * 64 + i];
+      part[n0 * 64 + i] = v;
+    }
+    __syncthreads();  // red is reused by the next block
   }
-  __syncthreads();  // red is reused by the next product
   return ok;
 }
 
 // After a cluster barrier: the sum over the cluster's ranks (in rank order)
-// of part[token rank][col] (part: this CTA's s.part or s.part_r).
-__device__ __forceinline__ float sk_cluster_sum(const SkCta& s, const float* part, int col) {
-  const uint32_t a = smem_u32(part + s.rank * 64 + col);
+// of part[i] (part: this CTA's s.part or s.part_r; i = token * 64 + column).
+__device__ __forceinline__ float sk_cluster_sum(const float* part, int i) {
+  const uint32_t a = smem_u32(part + i);
   float v = 0.f;
 #pragma unroll
   for (int r = 0; r < kSkCluster; ++r) v += ld_dsmem_f32(mapa_shared(a, (uint32_t)r));
   return v;
 }
 
-// Stage rows [row0, row0 + RR) of x for tokens tok[0..nt) into xs (zeros past
-// nt or past D); 16-byte pieces, four loaded before any is stored.
-__device__ __forceinline__ void sk_stage_x(const SkCta& s, const DecodeProjParams& p, const int* tok, int nt) {
+// Stage rows [row0, row0 + RR) of x for tokens 0..B-1 into xs (zeros past B
+// or past D); 16-byte pieces, four loaded before any is stored.
+__device__ __forceinline__ void sk_stage_x(const SkCta& s, const DecodeProjParams& p) {
   const int per = s.RR / 8;  // 16-byte pieces of a row
-  const int total = kSkinnyTB * per;
+  const int total = kSkinnyMaxTokens * per;
   for (int i0 = threadIdx.x; i0 < total; i0 += 4 * kSkinnyThreads) {
     uint4 v[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int i = i0 + u * kSkinnyThreads;
       const int n = i / per, col = s.row0 + (i % per) * 8;
-      v[u] = (i < total && n < nt && col < p.D) ? *reinterpret_cast<const uint4*>(p.x + (size_t)tok[n] * p.D + col)
-                                                : make_uint4(0u, 0u, 0u, 0u);
+      v[u] = (i < total && n < p.B && col < p.D) ? *reinterpret_cast<const uint4*>(p.x + (size_t)n * p.D + col)
+                                                 : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -233,14 +236,14 @@ __device__ __forceinline__ void sk_stage_x(const SkCta& s, const DecodeProjParam
   __syncthreads();
 }
 
-// Thread 0 of rank q, for token n of a pass: the decision of group g from
-// the logits in s.logits; the slot of expert e among the selections (-1:
-// not selected) into *s.slot; the e = 0 cluster writes sel, w and margin.
+// Thread i < kSkPerRank of rank q: the decision of group g for token n = n0 + i from
+// the logits in s.logits[i][.]; the slot of expert e among the selections
+// (-1: not selected) into s.slot[i]; the e = 0 cluster writes sel, w, margin.
 template <int RM>
-__device__ __forceinline__ void sk_decide(const SkCta& s, const DecodeProjParams& p, int g, int e, int n) {
+__device__ __forceinline__ void sk_decide(const SkCta& s, const DecodeProjParams& p, int g, int e, int i, int n) {
   float l[RM];
 #pragma unroll
-  for (int i = 0; i < RM; ++i) l[i] = s.logits[i];
+  for (int x = 0; x < RM; ++x) l[x] = s.logits[i * 8 + x];
   int32_t sl[8];
   float wl[8];
   float mg;
@@ -248,7 +251,7 @@ __device__ __forceinline__ void sk_decide(const SkCta& s, const DecodeProjParams
   int slot = -1;
   for (int j = 0; j < p.k; ++j)
     if (sl[j] == e) slot = j;
-  *s.slot = slot;
+  s.slot[i] = slot;
   if (e == 0) {
     for (int j = 0; j < p.k; ++j) {
       p.sel[((size_t)n * p.G + g) * p.k + j] = sl[j];
@@ -264,11 +267,11 @@ __device__ __forceinline__ void sk_decide(const SkCta& s, const DecodeProjParams
 __global__ void __cluster_dims__(kSkCluster, 1, 1) __launch_bounds__(kSkinnyThreads)
     decode_proj_kernel(const __grid_constant__ DecodeProjParams p) {
   extern __shared__ uint8_t sk_raw[];
-  SkCta s = sk_init(sk_raw, p.D);
   const int GM = p.G * p.M;
   const int blk = blockIdx.x / kSkCluster;
   const int Ha = p.G * p.k + 1;
   const bool routed = blk > 2 * p.G;
+  SkCta s = sk_init(sk_raw, p.D, routed);
   const CUtensorMap* W;
   int col0, g = 0, e = 0;
   if (blk < 2 * p.G) {
@@ -294,51 +297,49 @@ __global__ void __cluster_dims__(kSkCluster, 1, 1) __launch_bounds__(kSkinnyThre
   if (routed) sk_load(s, s.wbuf_r, s.bar_r, &p.tmWr, rcol);
   pdl_wait();
   pdl_trigger();
-  bool loaded = false, loaded_r = false, ok = true;
-  int tok[kSkinnyTB];
-  for (int n0 = 0; n0 < p.B; n0 += kSkinnyTB) {
-    const int nt = min(kSkinnyTB, p.B - n0);
-#pragma unroll
-    for (int n = 0; n < kSkinnyTB; ++n) tok[n] = n0 + n;
-    sk_stage_x(s, p, tok, nt);
-    ok = sk_product(s, s.wbuf, s.bar, 64, &loaded, s.part) && ok;
-    if (routed) ok = sk_product(s, s.wbuf_r, s.bar_r, roff + p.M, &loaded_r, s.part_r) && ok;
-    cluster_sync();  // every rank's partials are ready
-    const int n = n0 + s.rank;  // this rank's token
-    int slot = 0;
-    if (routed) {
-      if ((int)threadIdx.x < p.M)
-        s.logits[threadIdx.x] = sk_cluster_sum(s, s.part_r, roff + threadIdx.x) + (p.br ? p.br[g * p.M + threadIdx.x] : 0.f);
-      __syncthreads();
-      if (threadIdx.x == 0 && s.rank < nt && ok) {
-        switch (p.M) {
-          case 1: sk_decide<1>(s, p, g, e, n); break;
-          case 2: sk_decide<2>(s, p, g, e, n); break;
-          case 4: sk_decide<4>(s, p, g, e, n); break;
-          default: sk_decide<8>(s, p, g, e, n); break;
-        }
-      }
-      __syncthreads();
-      slot = *s.slot;
+  sk_stage_x(s, p);
+  bool ok = sk_product(s, s.wbuf, s.bar, 64, p.B, s.part);
+  if (routed) ok = sk_product(s, s.wbuf_r, s.bar_r, roff + p.M, p.B, s.part_r) && ok;
+  cluster_sync();  // every rank's partials are ready
+  const int n0 = s.rank * kSkPerRank;  // this rank's tokens [n0, n0 + kSkPerRank)
+  const int nr = max(0, min(kSkPerRank, p.B - n0));
+  if (routed) {
+    for (int i = threadIdx.x; i < nr * p.M; i += kSkinnyThreads) {
+      const int ti = i / p.M, x = i % p.M;
+      s.logits[ti * 8 + x] =
+          sk_cluster_sum(s.part_r, (n0 + ti) * 64 + roff + x) + (p.br ? p.br[g * p.M + x] : 0.f);
     }
-    if (ok && threadIdx.x < 64 && s.rank < nt && slot >= 0) {
-      const int c = threadIdx.x;
-      const __nv_bfloat16 v = __float2bfloat16_rn(sk_cluster_sum(s, s.part, c));
-      if (blk < 2 * p.G) {
-        const int L = p.cache_len[n];
-        if (L < 0 || L >= p.T) {
-          if (c == 0) flag_bounds_error();
-        } else {
-          (blk < p.G ? p.Kc : p.Vc)[(((size_t)n * p.T + L) * p.G + g) * 64 + c] = v;
-        }
-      } else if (!routed) {
-        p.Q[((size_t)n * Ha + p.G * p.k) * 64 + c] = v;
-      } else {
-        p.Q[((size_t)n * Ha + g * p.k + slot) * 64 + c] = v;
+    __syncthreads();
+    if ((int)threadIdx.x < nr && ok) {
+      const int i = threadIdx.x;
+      switch (p.M) {
+        case 1: sk_decide<1>(s, p, g, e, i, n0 + i); break;
+        case 2: sk_decide<2>(s, p, g, e, i, n0 + i); break;
+        case 4: sk_decide<4>(s, p, g, e, i, n0 + i); break;
+        default: sk_decide<8>(s, p, g, e, i, n0 + i); break;
       }
     }
-    cluster_sync();  // the ranks are done reading the partials
+    __syncthreads();
   }
+  for (int i = threadIdx.x; ok && i < nr * 64; i += kSkinnyThreads) {
+    const int ti = i / 64, c = i % 64, n = n0 + ti;
+    const int slot = routed ? s.slot[ti] : 0;
+    if (slot < 0) continue;
+    const __nv_bfloat16 v = __float2bfloat16_rn(sk_cluster_sum(s.part, n * 64 + c));
+    if (blk < 2 * p.G) {
+      const int L = p.cache_len[n];
+      if (L < 0 || L >= p.T) {
+        if (c == 0) flag_bounds_error();
+      } else {
+        (blk < p.G ? p.Kc : p.Vc)[(((size_t)n * p.T + L) * p.G + g) * 64 + c] = v;
+      }
+    } else if (!routed) {
+      p.Q[((size_t)n * Ha + p.G * p.k) * 64 + c] = v;
+    } else {
+      p.Q[((size_t)n * Ha + g * p.k + slot) * 64 + c] = v;
+    }
+  }
+  cluster_sync();  // the ranks are done reading the partials
   if (!ok) {  // a wait ran out: let copies in flight land before the block exits
     const unsigned long long t0 = globaltimer_ns();
     while (globaltimer_ns() - t0 < 100000ull) {}
@@ -353,52 +354,51 @@ __global__ void __cluster_dims__(kSkCluster, 1, 1) __launch_bounds__(kSkinnyThre
   extern __shared__ uint8_t sk_raw[];
   const int Gk = p.G * p.k, Ha = Gk + 1;
   const int Ka = (Gk + p.G + 1) * 64;
-  SkCta s = sk_init(sk_raw, Ka);
+  SkCta s = sk_init(sk_raw, Ka, false);
   const int col0 = (blockIdx.x / kSkCluster) * 64;
   sk_load(s, s.wbuf, s.bar, &p.tmWo, col0);  // Wo depends on no launch
   pdl_wait();
-  bool loaded = false, ok = true;
-  for (int n0 = 0; n0 < p.B; n0 += kSkinnyTB) {
-    const int nt = min(kSkinnyTB, p.B - n0);
-    // A's columns of this CTA: 64-wide blocks [concat (G*k) | slot (G) |
-    // shared], in 16-byte pieces of 8 columns; a thread loads all of a
-    // piece's inputs before storing it
-    const int per = s.RR / 8;
-    for (int i = threadIdx.x; i < kSkinnyTB * per; i += kSkinnyThreads) {
-      const int n = i / per, col = s.row0 + (i % per) * 8, blkc = col / 64, d = col % 64;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (n < nt && col < Ka) {
-        const size_t orow = (size_t)(n0 + n) * Ha;
-        if (blkc < Gk || blkc >= Gk + p.G) {
-          const int src = blkc < Gk ? blkc : Gk;  // concatenation, or the shared head
-          v = *reinterpret_cast<const uint4*>(p.O + (orow + src) * 64 + d);
-        } else {
-          const int g = blkc - Gk;
-          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-          for (int j = 0; j < p.k; ++j) {
-            const float wj = p.w[((size_t)(n0 + n) * p.G + g) * p.k + j];
-            const uint4 o = *reinterpret_cast<const uint4*>(p.O + (orow + g * p.k + j) * 64 + d);
-            const uint32_t ou[4] = {o.x, o.y, o.z, o.w};
+  // A's columns of this CTA for every token: 64-wide blocks [concat (G*k) |
+  // slot (G) | shared], in 16-byte pieces of 8 columns; a thread loads all of
+  // a piece's inputs before storing it
+  const int per = s.RR / 8;
+  for (int i = threadIdx.x; i < kSkinnyMaxTokens * per; i += kSkinnyThreads) {
+    const int n = i / per, col = s.row0 + (i % per) * 8, blkc = col / 64, d = col % 64;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (n < p.B && col < Ka) {
+      const size_t orow = (size_t)n * Ha;
+      if (blkc < Gk || blkc >= Gk + p.G) {
+        const int src = blkc < Gk ? blkc : Gk;  // concatenation, or the shared head
+        v = *reinterpret_cast<const uint4*>(p.O + (orow + src) * 64 + d);
+      } else {
+        const int g = blkc - Gk;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int j = 0; j < p.k; ++j) {
+          const float wj = p.w[((size_t)n * p.G + g) * p.k + j];
+          const uint4 o = *reinterpret_cast<const uint4*>(p.O + (orow + g * p.k + j) * 64 + d);
+          const uint32_t ou[4] = {o.x, o.y, o.z, o.w};
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              acc[2 * q] = fmaf(wj, bf16lo_to_f32(ou[q]), acc[2 * q]);
-              acc[2 * q + 1] = fmaf(wj, bf16hi_to_f32(ou[q]), acc[2 * q + 1]);
-            }
+          for (int q = 0; q < 4; ++q) {
+            acc[2 * q] = fmaf(wj, bf16lo_to_f32(ou[q]), acc[2 * q]);
+            acc[2 * q + 1] = fmaf(wj, bf16hi_to_f32(ou[q]), acc[2 * q + 1]);
           }
-          v = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
-                         pack_bf16x2(acc[6], acc[7]));
         }
+        v = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                       pack_bf16x2(acc[6], acc[7]));
       }
-      reinterpret_cast<uint4*>(s.xs)[i] = v;
     }
-    __syncthreads();
-    ok = sk_product(s, s.wbuf, s.bar, 64, &loaded, s.part) && ok;
-    cluster_sync();  // every rank's part is ready
-    if (ok && threadIdx.x < 64 && s.rank < nt)
-      p.y[(size_t)(n0 + s.rank) * p.D + col0 + threadIdx.x] =
-          __float2bfloat16_rn(sk_cluster_sum(s, s.part, threadIdx.x));
-    cluster_sync();  // the ranks are done reading part
+    reinterpret_cast<uint4*>(s.xs)[i] = v;
   }
+  __syncthreads();
+  const bool ok = sk_product(s, s.wbuf, s.bar, 64, p.B, s.part);
+  cluster_sync();  // every rank's part is ready
+  const int n0 = s.rank * kSkPerRank;
+  const int nr = max(0, min(kSkPerRank, p.B - n0));
+  for (int i = threadIdx.x; ok && i < nr * 64; i += kSkinnyThreads) {
+    const int n = n0 + i / 64, c = i % 64;
+    p.y[(size_t)n * p.D + col0 + c] = __float2bfloat16_rn(sk_cluster_sum(s.part, n * 64 + c));
+  }
+  cluster_sync();  // the ranks are done reading part
   if (!ok) {  // a wait ran out: let copies in flight land before the block exits
     const unsigned long long t0 = globaltimer_ns();
     while (globaltimer_ns() - t0 < 100000ull) {}
