@@ -10,7 +10,7 @@
 // attention, inference section (the new token's key/value rows are appended
 // to the cache).
 //
-// With a handful of rows a projection is a read of its weights: B x K times
+// With a few dozen rows a projection is a read of its weights: B x K times
 // K x 64 per 64-column slice. The tensor-core tiles of the prefill path would
 // pad the B rows to 256 and stream each weight through a few SMs; here every
 // slice is read by its own cluster of kSkCluster CTAs. CTA rank q loads rows
@@ -18,7 +18,7 @@
 // rounded up to whole kSkBoxRows boxes) and multiplies them with the same
 // rows of all the tokens' inputs (staged once, up to kSkinnyMaxTokens); the
 // eight partial sums meet in distributed shared memory, where rank q adds up
-// tokens [2q, 2q + 2) (ranks in order, so the sum is the same on every run).
+// tokens [8q, 8q + 8) (ranks in order, so the sum is the same on every run).
 // A launch takes two cluster barriers whatever the token count.
 //   decode_proj_kernel : 2G + 1 + G*M clusters: K and V of group g (written
 //                        into the caches at cache_len[b]), the shared head's
@@ -31,11 +31,12 @@
 //                        slot sum_j w_j O_j | shared] built for the CTA's rows
 //                        (A's columns) from O and w (the slot rounded to
 //                        bf16, as the combine kernel does)
-// Thread t of a 256-thread CTA owns 8 consecutive columns (t % 8) and the
-// rows t / 8 (mod 32) of the CTA's share; the 32 row-partial sums of each
-// column are added by shuffles within a warp and through shared memory across
-// warps. Every launch issues its weight loads before its dependency wait
-// (weights depend on no launch).
+// A CTA's product is mma.sync m16n8k16 (bf16 in, fp32 accumulate): warp w
+// takes the slice's columns [8w, 8w + 8) for every 16-token tile, A (the
+// tokens' rows) by matrix loads from a padded buffer, B (the weight rows,
+// [k][n] in the TMA's 128-byte swizzle) by transposing matrix loads. Every
+// launch issues its weight loads before its dependency wait (weights depend
+// on no launch).
 #pragma once
 
 #include "decode.cuh"
@@ -44,15 +45,12 @@
 
 namespace gqe {
 
-// Above 16 new tokens the CUDA-core products cost more than the prefill
-// path's tensor-core tiles (64 tokens: 52 + 31 us against three 17 us GEMMs).
-constexpr int kSkinnyMaxTokens = 16;
+constexpr int kSkinnyMaxTokens = 64;
 constexpr int kSkCluster = 8;
-constexpr int kSkinnyThreads = 256;
-constexpr int kSkinnyTB = 8;   // tokens per register block of a product
+constexpr int kSkinnyThreads = 256;  // 8 warps: one 8-column tile of the slice each
 constexpr int kSkPerRank = kSkinnyMaxTokens / kSkCluster;  // tokens a rank adds up
 constexpr int kSkBoxRows = 32; // TMA box: 64 columns x 32 rows, 4 KB
-static_assert(kSkPerRank <= 8 && kSkinnyMaxTokens % kSkinnyTB == 0, "decision area and register blocks");
+static_assert(kSkPerRank <= 8 && kSkinnyMaxTokens % 16 == 0, "decision area and 16-token tiles");
 
 struct DecodeProjParams {
   // weights as TMA tensor maps: box 64 columns x kSkBoxRows rows, 128-byte swizzle
@@ -79,12 +77,13 @@ __host__ __device__ inline int sk_rows(int K) {
 // Shared memory (from a 1024-aligned base): the CTA's weight rows wbuf
 // [RR][128 B] and, with `router`, the router rows wbuf_r [RR][128 B]; their
 // barriers and the abort flag (64 B); all tokens' input rows xs
-// [kSkinnyMaxTokens][RR] (bf16); per-warp partials red [8][TB][64]; the CTA's
-// partials part (and, with `router`, part_r) [kSkinnyMaxTokens][64] (read by
-// the cluster); the decision area: logits [8][8] and slots [8].
+// [kSkinnyMaxTokens][RR + 8] (bf16; the 16-byte pad makes the rows of a
+// matrix load fall in different banks); the CTA's partials part (and, with
+// `router`, part_r) [kSkinnyMaxTokens][64] (read by the cluster); the decision
+// area: logits [8][8] and slots [8].
 __host__ __device__ inline int sk_smem(int K, bool router) {
   const int RR = sk_rows(K);
-  return 1024 + (router ? 2 : 1) * RR * 128 + 64 + kSkinnyMaxTokens * RR * 2 + 8 * kSkinnyTB * 64 * 4 +
+  return 1024 + (router ? 2 : 1) * RR * 128 + 64 + kSkinnyMaxTokens * (RR + 8) * 2 +
          (router ? 2 : 1) * kSkinnyMaxTokens * 64 * 4 + 64 * 4 + 8 * 4;
 }
 
@@ -94,8 +93,7 @@ struct SkCta {
   uint64_t* bar;
   uint64_t* bar_r;
   volatile int* abort_flag;
-  __nv_bfloat16* xs;
-  float* red;
+  __nv_bfloat16* xs;  // [kSkinnyMaxTokens][RR + 8]
   float* part;
   float* part_r;
   float* logits;  // [8 tokens][8]
@@ -116,8 +114,7 @@ __device__ __forceinline__ SkCta sk_init(uint8_t* raw, int K, bool router) {
   s.bar_r = s.bar + 1;
   s.abort_flag = reinterpret_cast<volatile int*>(h + 16);
   s.xs = reinterpret_cast<__nv_bfloat16*>(h + 64);
-  s.red = reinterpret_cast<float*>(h + 64 + kSkinnyMaxTokens * s.RR * 2);
-  s.part = s.red + 8 * kSkinnyTB * 64;
+  s.part = reinterpret_cast<float*>(h + 64 + kSkinnyMaxTokens * (s.RR + 8) * 2);
   s.part_r = s.part + kSkinnyMaxTokens * 64;  // (router only)
   s.logits = s.part + (router ? 2 : 1) * kSkinnyMaxTokens * 64;
   s.slot = reinterpret_cast<int*>(s.logits + 64);
@@ -144,62 +141,51 @@ __device__ __forceinline__ void sk_load(const SkCta& s, uint8_t* wbuf, uint64_t*
 }
 
 // part[n][c] = sum over this CTA's rows r of xs[n][r] * W[row0 + r][col0 + c]
-// for tokens n < ntok and the slice in wbuf (columns at or past ncols are
-// zeros), eight tokens per register block. Waits for the weights first.
+// for tokens n < ntok (rounded up to 16, the rest zero) and the slice in wbuf
+// (columns at or past ncols are zeros). Warp w computes columns [8w, 8w + 8)
+// for every 16-token tile on mma.sync m16n8k16. Waits for the weights first.
 // Returns false if that wait ran out (part is then zero).
 __device__ __forceinline__ bool sk_product(const SkCta& s, const uint8_t* wbuf, uint64_t* bar, int ncols, int ntok,
                                            float* part) {
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int c8 = (t & 7) * 8, kr = t >> 3;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const bool ok = __syncthreads_and(mbar_wait(bar, 0, s.abort_flag));
-  const uint32_t base = smem_u32(wbuf);
-  for (int n0 = 0; n0 < ntok; n0 += kSkinnyTB) {
-    float acc[kSkinnyTB][8];
+  const int RRp = s.RR + 8;
+  const int nmt = (ntok + 15) / 16;  // 16-token tiles
+  const int col = warp * 8;
+  float acc[kSkinnyMaxTokens / 16][4];
 #pragma unroll
-    for (int n = 0; n < kSkinnyTB; ++n)
+  for (int mt = 0; mt < kSkinnyMaxTokens / 16; ++mt)
 #pragma unroll
-      for (int c = 0; c < 8; ++c) acc[n][c] = 0.f;
-    if (ok && c8 < ncols) {
-      for (int r = kr; r < s.RR; r += 32) {
-        uint32_t w4[4];
-        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(w4[0]), "=r"(w4[1]), "=r"(w4[2]), "=r"(w4[3])
-                     : "r"(base + r * 128 + ((((c8 >> 3) ^ (r & 7))) << 4)));
-        float wf[8];
+    for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
+  if (ok && col < ncols) {
+    const uint32_t wb = smem_u32(wbuf), xb = smem_u32(s.xs);
+    const int mi = lane >> 3, mr = lane & 7;
+    for (int ks = 0; ks < s.RR / 16; ++ks) {
+      // B: weight rows k = 16 ks .. 16 ks + 15 (lanes 0-15 address them),
+      // this warp's 16-byte column chunk, transposed into the (k, n) fragment
+      const int kb = ks * 16 + (lane & 15);
+      uint32_t b0, b1;
+      ldsm_x2_t(wb + kb * 128 + (((col >> 3) ^ (kb & 7)) << 4), b0, b1);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          wf[2 * e] = bf16lo_to_f32(w4[e]);
-          wf[2 * e + 1] = bf16hi_to_f32(w4[e]);
-        }
-#pragma unroll
-        for (int n = 0; n < kSkinnyTB; ++n) {
-          const float xv = __bfloat162float(s.xs[(n0 + n) * s.RR + r]);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) acc[n][c] = fmaf(xv, wf[c], acc[n][c]);
-        }
+      for (int mt = 0; mt < kSkinnyMaxTokens / 16; ++mt) {
+        if (mt >= nmt) break;
+        // A: tokens 16 mt .. 16 mt + 15 x k 16 ks .. 16 ks + 15
+        const int row = mt * 16 + (mi & 1) * 8 + mr, kc = ks * 16 + (mi >> 1) * 8;
+        uint32_t a[4];
+        ldsm_x4(xb + (row * RRp + kc) * 2, a[0], a[1], a[2], a[3]);
+        mma_bf16_16816(acc[mt], a, b0, b1);
       }
     }
-#pragma unroll
-    for (int n = 0; n < kSkinnyTB; ++n)
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        acc[n][c] += __shfl_xor_sync(0xffffffffu, acc[n][c], 8);
-        acc[n][c] += __shfl_xor_sync(0xffffffffu, acc[n][c], 16);
-      }
-    if (lane < 8)
-#pragma unroll
-      for (int n = 0; n < kSkinnyTB; ++n)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) s.red[(warp * kSkinnyTB + n) * 64 + c8 + c] = acc[n][c];
-    __syncthreads();
-    for (int i = t; i < kSkinnyTB * 64; i += kSkinnyThreads) {
-      float v = 0.f;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) v += s.red[w * kSkinnyTB * 64 + i];
-      part[n0 * 64 + i] = v;
-    }
-    __syncthreads();  // red is reused by the next block
   }
+  // accumulator fragment: tokens 16 mt + lane / 4 (+ 8), columns col + 2 (lane % 4) (+ 1)
+  const int tr = lane >> 2, tc = col + 2 * (lane & 3);
+#pragma unroll
+  for (int mt = 0; mt < kSkinnyMaxTokens / 16; ++mt) {
+    if (mt >= nmt) break;
+    *reinterpret_cast<float2*>(part + (mt * 16 + tr) * 64 + tc) = make_float2(acc[mt][0], acc[mt][1]);
+    *reinterpret_cast<float2*>(part + (mt * 16 + tr + 8) * 64 + tc) = make_float2(acc[mt][2], acc[mt][3]);
+  }
+  __syncthreads();
   return ok;
 }
 
@@ -230,7 +216,7 @@ __device__ __forceinline__ void sk_stage_x(const SkCta& s, const DecodeProjParam
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int i = i0 + u * kSkinnyThreads;
-      if (i < total) reinterpret_cast<uint4*>(s.xs)[i] = v[u];
+      if (i < total) reinterpret_cast<uint4*>(s.xs)[(i / per) * (per + 1) + i % per] = v[u];
     }
   }
   __syncthreads();
@@ -387,7 +373,7 @@ __global__ void __cluster_dims__(kSkCluster, 1, 1) __launch_bounds__(kSkinnyThre
                        pack_bf16x2(acc[6], acc[7]));
       }
     }
-    reinterpret_cast<uint4*>(s.xs)[i] = v;
+    reinterpret_cast<uint4*>(s.xs)[n * (per + 1) + i % per] = v;
   }
   __syncthreads();
   const bool ok = sk_product(s, s.wbuf, s.bar, 64, p.B, s.part);

@@ -24,12 +24,10 @@ CASES = [
     ("b3_d512_g8m4k2_skewed", Dims(B=3, T=1500, D=512, G=8, M=4, k=2, bias0=2.0), [1024, 1, 700]),
     ("b2_d256_g2m8k4", Dims(B=2, T=300, D=256, G=2, M=8, k=4), [5, 299]),
     ("b5_d256_g1m8k2_mqa", Dims(B=5, T=130, D=256, G=1, M=8, k=2), [0, 63, 64, 128, 129]),
-    # 13 and 16 new tokens: the cluster kernels' largest register blocks, ranks
-    # with partial and empty token pairs
+    # 13, 16, 37 and 64 new tokens on the cluster kernels (ranks with partial
+    # and empty token blocks, partial 16-token tiles), 65 on the prefill kernels
     ("b13_d256_g4m2k1", Dims(B=13, T=260, D=256, G=4, M=2, k=1), [(i * 53) % 260 for i in range(13)]),
     ("b16_d512_g8m4k2", Dims(B=16, T=200, D=512, G=8, M=4, k=2), [(i * 37) % 200 for i in range(16)]),
-    # more new tokens than the cluster kernels take (16): the prefill kernels
-    # on the new tokens, then the same attention
     ("b37_d256_g4m2k1", Dims(B=37, T=260, D=256, G=4, M=2, k=1), [(i * 53) % 260 for i in range(37)]),
     ("b64_d256_g8m4k2", Dims(B=64, T=200, D=256, G=8, M=4, k=2), [(i * 37) % 200 for i in range(64)]),
     ("b65_d256_g4m2k1", Dims(B=65, T=150, D=256, G=4, M=2, k=1), [(i * 29) % 150 for i in range(65)]),
