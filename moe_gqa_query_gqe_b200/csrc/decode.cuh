@@ -105,7 +105,10 @@ constexpr int kDmWarps = 8;
 constexpr int kDmThreads = kDmWarps * 32;
 constexpr int kDmSK = 32;                       // keys per stage
 constexpr int kDmItem = 64;                     // keys per item (the unit of the split)
-constexpr int kDmStages = 3;                    // ring depth per warp
+// ring depth per warp: 2 keeps the CTA at 129 KB of shared memory, so it
+// fits on an SM beside two of the projection launch's CTAs and starts
+// streaming the cache while they run (3 stages: 8 us slower per step)
+constexpr int kDmStages = 2;
 constexpr int kDmGridMax = 148;                 // CTAs at most (one per SM of a B200)
 constexpr int kDmBlock = kDmSK * 128;           // one K (or V) block of a stage, bytes
 constexpr int kDmStageBytes = 2 * kDmBlock;

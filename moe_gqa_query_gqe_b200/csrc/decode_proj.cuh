@@ -76,15 +76,17 @@ __host__ __device__ inline int sk_rows(int K) {
 }
 // Shared memory (from a 1024-aligned base): the CTA's weight rows wbuf
 // [RR][128 B] and, with `router`, the router rows wbuf_r [RR][128 B]; their
-// barriers and the abort flag (64 B); all tokens' input rows xs
-// [kSkinnyMaxTokens][RR + 8] (bf16; the 16-byte pad makes the rows of a
-// matrix load fall in different banks); the CTA's partials part (and, with
-// `router`, part_r) [kSkinnyMaxTokens][64] (read by the cluster); the decision
-// area: logits [8][8] and slots [8].
-__host__ __device__ inline int sk_smem(int K, bool router) {
-  const int RR = sk_rows(K);
-  return 1024 + (router ? 2 : 1) * RR * 128 + 64 + kSkinnyMaxTokens * (RR + 8) * 2 +
-         (router ? 2 : 1) * kSkinnyMaxTokens * 64 * 4 + 64 * 4 + 8 * 4;
+// barriers and the abort flag (64 B); all tokens' input rows xs [cap][RR + 8]
+// (bf16; the 16-byte pad makes the rows of a matrix load fall in different
+// banks); the CTA's partials part (and, with `router`, part_r) [cap][64] (read
+// by the cluster); the decision area: logits [8][8] and slots [8]. cap is B
+// rounded up to a 16-token tile, so a small step leaves room on the SM for
+// the attention launch's CTAs.
+__host__ __device__ inline int sk_cap(int B) { return (B + 15) / 16 * 16; }
+__host__ __device__ inline int sk_smem(int K, bool router, int B) {
+  const int RR = sk_rows(K), cap = sk_cap(B);
+  return 1024 + (router ? 2 : 1) * RR * 128 + 64 + cap * (RR + 8) * 2 + (router ? 2 : 1) * cap * 64 * 4 + 64 * 4 +
+         8 * 4;
 }
 
 struct SkCta {
@@ -93,18 +95,19 @@ struct SkCta {
   uint64_t* bar;
   uint64_t* bar_r;
   volatile int* abort_flag;
-  __nv_bfloat16* xs;  // [kSkinnyMaxTokens][RR + 8]
+  __nv_bfloat16* xs;  // [cap][RR + 8]
   float* part;
   float* part_r;
   float* logits;  // [8 tokens][8]
   int* slot;      // [8 tokens]
-  int RR, row0, rank;
+  int RR, row0, rank, cap;
 };
 
-__device__ __forceinline__ SkCta sk_init(uint8_t* raw, int K, bool router) {
+__device__ __forceinline__ SkCta sk_init(uint8_t* raw, int K, bool router, int B) {
   SkCta s;
   uint8_t* b = raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
   s.RR = sk_rows(K);
+  s.cap = sk_cap(B);
   s.rank = (int)cluster_ctarank();
   s.row0 = s.rank * s.RR;
   s.wbuf = b;
@@ -114,9 +117,9 @@ __device__ __forceinline__ SkCta sk_init(uint8_t* raw, int K, bool router) {
   s.bar_r = s.bar + 1;
   s.abort_flag = reinterpret_cast<volatile int*>(h + 16);
   s.xs = reinterpret_cast<__nv_bfloat16*>(h + 64);
-  s.part = reinterpret_cast<float*>(h + 64 + kSkinnyMaxTokens * (s.RR + 8) * 2);
-  s.part_r = s.part + kSkinnyMaxTokens * 64;  // (router only)
-  s.logits = s.part + (router ? 2 : 1) * kSkinnyMaxTokens * 64;
+  s.part = reinterpret_cast<float*>(h + 64 + s.cap * (s.RR + 8) * 2);
+  s.part_r = s.part + s.cap * 64;  // (router only)
+  s.logits = s.part + (router ? 2 : 1) * s.cap * 64;
   s.slot = reinterpret_cast<int*>(s.logits + 64);
   if (threadIdx.x == 0) {
     mbar_init(s.bar, 1);
@@ -203,7 +206,7 @@ __device__ __forceinline__ float sk_cluster_sum(const float* part, int i) {
 // or past D); 16-byte pieces, four loaded before any is stored.
 __device__ __forceinline__ void sk_stage_x(const SkCta& s, const DecodeProjParams& p) {
   const int per = s.RR / 8;  // 16-byte pieces of a row
-  const int total = kSkinnyMaxTokens * per;
+  const int total = s.cap * per;
   for (int i0 = threadIdx.x; i0 < total; i0 += 4 * kSkinnyThreads) {
     uint4 v[4];
 #pragma unroll
@@ -257,7 +260,7 @@ __global__ void __cluster_dims__(kSkCluster, 1, 1) __launch_bounds__(kSkinnyThre
   const int blk = blockIdx.x / kSkCluster;
   const int Ha = p.G * p.k + 1;
   const bool routed = blk > 2 * p.G;
-  SkCta s = sk_init(sk_raw, p.D, routed);
+  SkCta s = sk_init(sk_raw, p.D, routed, p.B);
   const CUtensorMap* W;
   int col0, g = 0, e = 0;
   if (blk < 2 * p.G) {
@@ -340,7 +343,7 @@ __global__ void __cluster_dims__(kSkCluster, 1, 1) __launch_bounds__(kSkinnyThre
   extern __shared__ uint8_t sk_raw[];
   const int Gk = p.G * p.k, Ha = Gk + 1;
   const int Ka = (Gk + p.G + 1) * 64;
-  SkCta s = sk_init(sk_raw, Ka, false);
+  SkCta s = sk_init(sk_raw, Ka, false, p.B);
   const int col0 = (blockIdx.x / kSkCluster) * 64;
   sk_load(s, s.wbuf, s.bar, &p.tmWo, col0);  // Wo depends on no launch
   pdl_wait();
@@ -348,7 +351,7 @@ __global__ void __cluster_dims__(kSkCluster, 1, 1) __launch_bounds__(kSkinnyThre
   // slot (G) | shared], in 16-byte pieces of 8 columns; a thread loads all of
   // a piece's inputs before storing it
   const int per = s.RR / 8;
-  for (int i = threadIdx.x; i < kSkinnyMaxTokens * per; i += kSkinnyThreads) {
+  for (int i = threadIdx.x; i < s.cap * per; i += kSkinnyThreads) {
     const int n = i / per, col = s.row0 + (i % per) * 8, blkc = col / 64, d = col % 64;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (n < p.B && col < Ka) {

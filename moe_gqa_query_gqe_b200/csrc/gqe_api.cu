@@ -977,7 +977,7 @@ int gqe_decode(const gqe_dims* d, const int32_t* cache_len, const void* x_new, c
   DecodeWs f = carve_decode(c, d);
   const gqe_dims t = decode_token_dims(d);
   const int ka_cols = (d->G * d->k + d->G + 1) * 64;
-  const bool skinny = d->B <= kSkinnyMaxTokens && sk_smem(d->D, true) <= 232448 && sk_smem(ka_cols, false) <= 232448;
+  const bool skinny = d->B <= kSkinnyMaxTokens && sk_smem(d->D, true, d->B) <= 232448 && sk_smem(ka_cols, false, d->B) <= 232448;
   DecodeProjParams pp;
   memset(&pp, 0, sizeof(pp));
   pp.x = static_cast<const __nv_bfloat16*>(x_new);
@@ -1007,7 +1007,7 @@ int gqe_decode(const gqe_dims* d, const int32_t* cache_len, const void* x_new, c
     GQE_TRY(tmap_rows(&pp.tmWv, Wv, d->D, d->G * 64, d->G * 64, kSkBoxRows));
     GQE_TRY(tmap_rows(&pp.tmWr, Wr, d->D, GM, GM, kSkBoxRows));
     GQE_TRY(tmap_rows(&pp.tmWo, Wo, Ka, d->D, d->D, kSkBoxRows));
-    const int smem = sk_smem(d->D, true);
+    const int smem = sk_smem(d->D, true, d->B);
     GQE_TRY(set_smem(decode_proj_kernel, smem));
     GQE_TRY(launch_pdl(decode_proj_kernel, dim3((2 * d->G + 1 + GM) * kSkCluster), dim3(kSkinnyThreads), smem, st,
                        pp));
@@ -1057,7 +1057,7 @@ int gqe_decode(const gqe_dims* d, const int32_t* cache_len, const void* x_new, c
   GQE_TRY(launch_decode_attn_mma(dp, &dp.nsplit, st));
   GQE_TRY(launch_pdl(decode_merge_kernel, dim3((unsigned)((long long)d->B * dp.Ha)), dim3(kDecMergeThreads), 0, st, dp));
   if (skinny) {
-    const int smem = sk_smem(ka_cols, false);
+    const int smem = sk_smem(ka_cols, false, d->B);
     GQE_TRY(set_smem(decode_out_kernel, smem));
     return launch_pdl(decode_out_kernel, dim3((unsigned)(d->D / 64) * kSkCluster), dim3(kSkinnyThreads), smem, st,
                       pp);
