@@ -1,7 +1,7 @@
-// decode_proj.cuh -- the token-side work of one decode step for a few new
-// tokens (B <= kSkinnyMaxTokens): routing, the K/V and query projections and
-// the output construction with its projection, as skinny products on CUDA
-// cores, each 64-column weight slice split over the rows of a cluster.
+// decode_proj.cuh -- the token-side work of one decode step for up to
+// kSkinnyMaxTokens new tokens: routing, the K/V and query projections and the
+// output construction with its projection, as skinny products, each 64-column
+// weight slice split over the rows of a cluster.
 //
 // Method: the layer of the gist.science summary ("Architecture and routing":
 // conditional activation, renormalised weighted sum, dense K/V, output
