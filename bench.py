@@ -344,7 +344,12 @@ def pool_study(steps: int, warmup: int) -> None:
                                                      y2, wd))
             t_gqe, t_dense = timed(g1), timed(g2)
             status = gqe.gqe_check_error()
-            seg = gqe.forward_views(d, ws)["seg_off"].diff().double()
+            # tokens per (sequence, group, expert) from the decisions (the
+            # forward builds segment lists only on its gather path)
+            sel = gqe.forward_views(d, ws)["sel"].long() & 0xFF                   # [N, G, k]
+            gidx = torch.arange(d.G, device=sel.device).view(1, d.G, 1) * M
+            bidx = (torch.arange(N, device=sel.device) // d.T).view(N, 1, 1) * (d.G * M)
+            seg = torch.bincount((sel + gidx + bidx).flatten(), minlength=d.B * d.G * M).double()
             mean = N * k / M
             fl = flops_model(d)
             print(json.dumps({"study": "expert_pool", "M": M, "k": k, "bias0": bias0, "T": d.T, "G": d.G,
