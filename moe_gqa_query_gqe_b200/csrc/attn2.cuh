@@ -11,8 +11,8 @@
 // so the routed attention of a group is causal attention with rr rows per
 // position and stays balanced under any routing skew.
 //
-// Per CTA (persistent, one per SM, 640 threads), work item = two adjacent
-// 128-row Q tiles (A, B) of one row set; items are visited heaviest first:
+// Per CTA (persistent, one per SM), work item = two adjacent 128-row Q tiles
+// (A, B) of one row set; items are visited heaviest first:
 //   warp 0      TMA producer: Q_A, Q_B once per item (two item buffers, so
 //               the next item's Q arrives while this one runs), K/V blocks of
 //               128 positions through a STAGES-deep ring
@@ -22,13 +22,12 @@
 //                 O_t     += P_t(j) V_j     (TS MMA: P read from TMEM, N=64)
 //               so neither tile's pipeline waits on the other's barriers
 //   warp 3      idle
-//   warps 4..19 softmax, eight warps a tile, 16 rows a warp, four threads a
-//               row (so each SM sub-partition runs four softmax warps, whose
-//               dependency chains hide one another's latency): S read from
-//               TMEM (then released at once so the next S can be computed
-//               under this block's softmax), lazily rescaled online softmax
-//               in the exp2 domain, P written back to TMEM as bf16 pairs,
-//               final O / l stored as bf16.
+//   warps 4..   softmax: S read from TMEM (then released at once so the next
+//               S can be computed under this block's softmax), lazily
+//               rescaled online softmax in the exp2 domain, P written back to
+//               TMEM as bf16 pairs, final O / l stored as bf16. Row layout:
+//               warps 4..11, one thread per row. Quad layout: warps 4..19,
+//               16 rows a warp, four threads a row.
 // TMEM columns: S_A [0,128) S_B [128,256) O_A [256,320) O_B [320,384)
 //               P_A [384,448) P_B [448,512).
 // Exponentials: MUFU ex2 delivers 16/clk/SM while each score needs 1/32 clk
@@ -44,8 +43,20 @@
 namespace gqe {
 
 constexpr int kA2Stages = 3;
-constexpr int kA2Threads = 640;
-constexpr int kA2SoftmaxPerTile = 256;  // softmax threads of one Q tile (8 warps x 16 rows x 4 threads a row)
+// Two softmax layouts (template parameter kQuad of attn2_fwd_kernel):
+//   row layout,  384 threads: one thread per row, two softmax warps per SM
+//                sub-partition, 88/208 register split after set-up
+//                (88*128 + 208*256 = 168*384, the registers of the launch);
+//   quad layout, 640 threads: four threads per row, four softmax warps per
+//                sub-partition.
+// The host takes the quad layout when every row set has one row per token
+// (GQE with k = 1): there it measured as fast at 2K tokens and 4% faster at
+// 32K. With two rows per token (the dense baseline's M = 2 heads, GQE with
+// k = 2) the row layout measured faster from 2K to 16K and equal at 32K.
+constexpr int kA2ThreadsRow = 384;
+constexpr int kA2ThreadsQuad = 640;
+constexpr int kA2RegsLow = 88;
+constexpr int kA2RegsHigh = 208;
 constexpr int kA2PolyEvery = 8;  // every n-th column pair uses the FMA-pipe exp2 (0: none)
 
 struct Attn2Params {
@@ -240,7 +251,10 @@ __device__ __forceinline__ int a2_item_of(int round) {
   return round * g + ((round & 1) ? (g - 1 - (int)blockIdx.x) : (int)blockIdx.x);
 }
 
-__global__ void __launch_bounds__(kA2Threads, 1) attn2_fwd_kernel(const __grid_constant__ Attn2Params p) {
+template <bool kQuad>
+__global__ void __launch_bounds__(kQuad ? kA2ThreadsQuad : kA2ThreadsRow, 1)
+    attn2_fwd_kernel(const __grid_constant__ Attn2Params p) {
+  constexpr int kSoftmaxPerTile = kQuad ? 256 : 128;  // softmax threads of one Q tile
   pdl_wait();
   pdl_trigger();
   using L = A2Smem;
@@ -273,8 +287,8 @@ __global__ void __launch_bounds__(kA2Threads, 1) attn2_fwd_kernel(const __grid_c
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&s_free[t], kA2SoftmaxPerTile);
-      mbar_init(&p_full[t], kA2SoftmaxPerTile);
+      mbar_init(&s_free[t], kSoftmaxPerTile);
+      mbar_init(&p_full[t], kSoftmaxPerTile);
       mbar_init(&pv_done[t], 1);
     }
     *abort_flag = 0;
@@ -293,6 +307,7 @@ __global__ void __launch_bounds__(kA2Threads, 1) attn2_fwd_kernel(const __grid_c
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t sbase = smem_u32(smem);
   if (warp < 4) {
+    if constexpr (!kQuad) setmaxnreg_dec<kA2RegsLow>();
     if (warp == 0 && lane == 0) {
       // ---- producer ------------------------------------------------------------
       uint32_t kv = 0, n_items = 0;
@@ -381,7 +396,7 @@ __global__ void __launch_bounds__(kA2Threads, 1) attn2_fwd_kernel(const __grid_c
         ++n_items;
       }
     }
-  } else {
+  } else if constexpr (kQuad) {
     // ---- softmax: 16 warps, four on each SM sub-partition -----------------------
     // Warp w (4..19) takes lane quadrant q = w % 4 (the TMEM lanes it may
     // access), tile t = ((w - 4) / 4) % 2 and half h = (w - 4) / 8 of the
@@ -559,6 +574,155 @@ __global__ void __launch_bounds__(kA2Threads, 1) attn2_fwd_kernel(const __grid_c
             __nv_bfloat16* sd = p.O + ((r ? n_tok1 : n_tok0) * p.o_ld + p.slot_blk0 + it.rs.kvg) * 64 + 2 * c4;
 #pragma unroll
             for (int m = 0; m < 8; ++m) st_global_b32(sd + 8 * m, pack_bf16x2(acc[2 * m], acc[2 * m + 1]));
+          }
+        }
+      }
+      tc_fence_before();
+    }
+  } else {
+    setmaxnreg_inc<kA2RegsHigh>();
+    // ---- softmax warpgroups: warps 4..7 -> tile A, 8..11 -> tile B --------------
+    const int t = (warp - 4) >> 2;
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int row = q * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t tm_s = tmem_base + lane_off + t * 128;
+    const uint32_t tm_o = tmem_base + lane_off + 256 + t * 64;
+    const uint32_t tm_p = tmem_base + lane_off + 384 + t * 64;
+    const float sl2 = p.scale_log2;
+    uint32_t cnt = 0;  // blocks processed by this tile so far (barrier phases)
+    bool ok = true;
+    for (int round = 0, item = a2_item_of(0); ok && item < p.total_items; item = a2_item_of(++round)) {
+      const A2Item it = a2_decode(p, item);
+      if (!it.valid) continue;
+      const int nblk = t == 0 ? it.nA : it.nB;
+      if (nblk == 0) continue;
+      const int tfirst = it.t0 + t * it.tpt;      // first token of this tile
+      const int tok = tfirst + row / it.rs.rr;    // token of this row (>= T: not stored)
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int j = 0; j < nblk; ++j, ++cnt) {
+        bool w_ok = mbar_wait(&s_full[t], cnt & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+        tc_fence_after();
+        float s[128];
+        tmem_ld128f(tm_s, s);
+        tc_fence_before();
+        mbar_arrive(&s_free[t]);  // S may be overwritten by the next block's QK^T now
+
+        const int kv0 = j * 128;
+        if (kv0 + 127 > tfirst) {
+          const int lim = tok - kv0;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c > lim) s[c] = -INFINITY;
+        }
+        float m4[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+        for (int c = 4; c < 128; c += 8) {
+          m4[0] = fmax3(m4[0], s[c], s[c + 1]);
+          m4[1] = fmax3(m4[1], s[c + 2], s[c + 3]);
+          m4[2] = fmax3(m4[2], s[c + 4], s[c + 5]);
+          m4[3] = fmax3(m4[3], s[c + 6], s[c + 7]);
+        }
+        const float mx = fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
+        const float m_new = fmaxf(m_run, mx * sl2);
+        const float m_use = (m_new > m_run + kRescaleThreshold) ? m_new : m_run;
+        const float alpha = ex2_approx(m_run - m_use);
+        const bool rescale = (j > 0) && (m_use != m_run);
+        m_run = m_use;
+
+        // x = s * scale_log2 - m, then 2^x: MUFU for most pairs, FMA pipe for some
+        float sm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 4 independent pair chains
+        uint32_t pk[64];
+#pragma unroll
+        for (int pi = 0; pi < 64; ++pi) {
+          float x0, x1, y0, y1;
+          ffma2(x0, x1, s[2 * pi], s[2 * pi + 1], sl2, sl2, -m_use, -m_use);
+          bool poly = false;
+          if constexpr (kA2PolyEvery > 0) poly = (pi % kA2PolyEvery) == kA2PolyEvery - 1;
+          if (poly) {
+            exp2_poly2(y0, y1, x0, x1);
+          } else {
+            y0 = ex2_approx(x0);
+            y1 = ex2_approx(x1);
+          }
+          fadd2(sm[2 * (pi & 3)], sm[2 * (pi & 3) + 1], sm[2 * (pi & 3)], sm[2 * (pi & 3) + 1], y0, y1);
+          pk[pi] = pack_bf16x2(y0, y1);
+        }
+        l_run = l_run * alpha + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
+
+        // P(j) overwrites P(j-1) and O may need rescaling: both need PV(j-1) done
+        if (j > 0) {
+          w_ok = mbar_wait(&pv_done[t], (cnt - 1) & 1, abort_flag);
+          if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              uint32_t o[16];
+              tmem_ld16(tm_o + h * 16, o);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+              tmem_st16(tm_o + h * 16, o);
+            }
+          }
+        }
+        tmem_st64(tm_p, pk);
+        tc_fence_before();
+        mbar_arrive(&p_full[t]);
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l -> bf16 ------------------------------------------------
+      const int rr = it.rs.rr, jslot = row % rr;
+      const size_t n_tok = (size_t)it.b * p.T + (tok < p.T ? tok : 0);
+      // slot weights of this row's token (fused output construction)
+      const bool slot = p.w != nullptr && it.rs.ob < p.slot_blk0;
+      float wj[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        wj[i] = (slot && i < rr && tok < p.T) ? p.w[(n_tok * p.G + it.rs.kvg) * rr + i] : 0.f;
+      const bool w_ok = mbar_wait(&pv_done[t], (cnt - 1) & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+      tc_fence_after();
+      const float inv = 1.f / l_run;
+      __nv_bfloat16* dst = (tok < p.T) ? p.O + (n_tok * p.o_ld + it.rs.ob + jslot) * 64 : nullptr;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t o[32];
+        tmem_ld32(tm_o + h * 32, o);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+        if (dst) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            st_global_v4(dst + h * 32 + i * 8, pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+        if (slot) {
+          // The token's rr rows are lanes base .. base+rr-1 of this warp.
+          // Every one of them sums the rr bf16 outputs (fp32, in slot
+          // order, as the separate combine kernel does); the first stores.
+          const int base = lane - jslot;
+          float acc[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) acc[c] = 0.f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if (i >= rr) break;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const uint32_t u = __shfl_sync(0xffffffffu, pk[c], base + i);
+              acc[2 * c] = fmaf(wj[i], bf16lo_to_f32(u), acc[2 * c]);
+              acc[2 * c + 1] = fmaf(wj[i], bf16hi_to_f32(u), acc[2 * c + 1]);
+            }
+          }
+          if (dst && jslot == 0) {
+            __nv_bfloat16* sd = p.O + (n_tok * p.o_ld + p.slot_blk0 + it.rs.kvg) * 64 + h * 32;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              st_global_v4(sd + i * 8, pack_bf16x2(acc[8 * i], acc[8 * i + 1]), pack_bf16x2(acc[8 * i + 2], acc[8 * i + 3]),
+                           pack_bf16x2(acc[8 * i + 4], acc[8 * i + 5]), pack_bf16x2(acc[8 * i + 6], acc[8 * i + 7]));
           }
         }
       }

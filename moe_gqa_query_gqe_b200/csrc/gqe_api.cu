@@ -558,9 +558,13 @@ int do_attn2(const gqe_dims* d, const void* Q, int Hq, const void* K, const void
   if (items > 0x7fffffffll) return GQE_ERR_UNSUPPORTED;
   p.total_items = (int)items;
   p.scale_log2 = 1.4426950408889634f / sqrtf(64.f);
-  GQE_TRY(set_smem(attn2_fwd_kernel, A2Smem::kBytes));
   const int grid = (int)std::min<long long>(items, sm_count());
-  return launch_pdl(attn2_fwd_kernel, dim3(grid), dim3(kA2Threads), A2Smem::kBytes, st, p);
+  if (rr == 1) {  // every row set one row per token: the quad softmax layout
+    GQE_TRY(set_smem(attn2_fwd_kernel<true>, A2Smem::kBytes));
+    return launch_pdl(attn2_fwd_kernel<true>, dim3(grid), dim3(kA2ThreadsQuad), A2Smem::kBytes, st, p);
+  }
+  GQE_TRY(set_smem(attn2_fwd_kernel<false>, A2Smem::kBytes));
+  return launch_pdl(attn2_fwd_kernel<false>, dim3(grid), dim3(kA2ThreadsRow), A2Smem::kBytes, st, p);
 }
 
 // k = 1: the renormalised weight of the one selected expert is exactly 1, so
