@@ -559,7 +559,7 @@ int do_attn2(const gqe_dims* d, const void* Q, int Hq, const void* K, const void
   p.total_items = (int)items;
   p.scale_log2 = 1.4426950408889634f / sqrtf(64.f);
   const int grid = (int)std::min<long long>(items, sm_count());
-  if (rr == 1) {  // every row set one row per token: the quad softmax layout
+  if (rr == 1 && slot_w == nullptr) {  // one row per token in every set, no slots: the quad softmax layout
     GQE_TRY(set_smem(attn2_fwd_kernel<true>, A2Smem::kBytes));
     return launch_pdl(attn2_fwd_kernel<true>, dim3(grid), dim3(kA2ThreadsQuad), A2Smem::kBytes, st, p);
   }
